@@ -1,0 +1,273 @@
+"""CPU oracle for the KV selection / compaction path (double precision).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may use this package; the product library
+never does. It shares no code with the CUDA path and does not import it.
+
+The arithmetic lives in ``kvcomp_oracle.c`` (plain C, double, no FMA
+contraction); this module compiles it with gcc on first use and wraps it with
+numpy. Each wrapper names the page passage it restates:
+
+* ``score``     AudioKV blog §1.2 (raw importance scores), window-softmax sum.
+* ``sss``       AudioKV blog §2.2 (Spectral Score Smoothing) via a direct DFT.
+* ``allocate``  AudioKV blog §3.1 / §5.1 (head-aware budget allocation).
+* ``select``    AudioKV blog §3.1 (local window kept) + top-k by smoothed score.
+* ``decode_*``  VoxZip, second stage (temporally decayed cumulative attention,
+                Concat(K[:T], K[I_hist], K[-M:]) eviction).
+
+Parity status: pinned (see tests/test_oracle_*.py); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvcomp_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC", "-pthread"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into liboracle.so (gcc); returns the path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _get():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = C.CDLL(build())
+            P = C.c_void_p
+            I64, I32, D = C.c_int64, C.c_int, C.c_double
+            lib.orc_score_rows.argtypes = [I64, P, P, P, I32, I32, P, P, I32]
+            lib.orc_rdft.argtypes = [P, I64, P, P]
+            lib.orc_kstar.argtypes = [P, P, I64, D, P]
+            lib.orc_kstar.restype = I64
+            lib.orc_irdft_lowpass.argtypes = [P, P, I64, I64, P]
+            lib.orc_sss_rows.argtypes = [I64, P, P, P, D, D, P, P, P, I32]
+            lib.orc_allocate.argtypes = [I32, P, I32, I32, I32, I32, C.c_float, P, P]
+            lib.orc_allocate.restype = I32
+            lib.orc_select_rows.argtypes = [I64, P, P, P, I32, P, P, P, I32]
+            lib.orc_decode_step.argtypes = [P, I32, I32, P, P, P, P, P, P, P, I64, D, I32, I32, I64, P]
+            lib.orc_decode_step.restype = I64
+            lib.orc_decode_run_heads.argtypes = [I64, P, I32, I32, P, P, P, P, P, I64, P, P, P, P, D, I32, P, P,
+                                                 P, P, I32]
+            _lib = lib
+        return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- step 1 ----
+def score(qwin: np.ndarray, K: np.ndarray, L_rows: Sequence[int], n_threads: int = 0) -> np.ndarray:
+    """Window scores of every row (AudioKV blog §1.2 raw importance scores).
+
+    qwin [rows][R][d]; K concatenated [sum L][d] in row order. Returns the
+    concatenated scores [sum L] (float64): s_j = sum_r softmax_j(q_r.K_j/sqrt d).
+    """
+    qwin = _c(qwin, np.float32)
+    K = _c(K, np.float32)
+    L = _c(L_rows, np.int64)
+    off = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+    rows, R, d = qwin.shape
+    assert K.shape == (off[-1], d)
+    s = np.zeros(off[-1], np.float64)
+    _get().orc_score_rows(rows, _p(L), _p(off), _p(qwin), R, d, _p(K), _p(s), n_threads or default_threads())
+    return s
+
+
+# ---------------------------------------------------------------- step 2 ----
+def rdft(s: np.ndarray) -> np.ndarray:
+    """One-sided DFT bins 0..L/2 of a real row, by direct summation (complex128)."""
+    s = _c(s, np.float64)
+    L = s.shape[0]
+    re = np.zeros(L // 2 + 1)
+    im = np.zeros(L // 2 + 1)
+    _get().orc_rdft(_p(s), L, _p(re), _p(im))
+    return re + 1j * im
+
+
+def kstar(F: np.ndarray, L: int, rho: float) -> Tuple[int, np.ndarray]:
+    """Smallest k with E(k) >= rho E(L/2); returns (k*, E prefix)."""
+    re = _c(F.real, np.float64)
+    im = _c(F.imag, np.float64)
+    E = np.zeros(L // 2 + 1)
+    k = _get().orc_kstar(_p(re), _p(im), L, rho, _p(E))
+    return int(k), E
+
+
+def irdft_lowpass(F: np.ndarray, L: int, k: int) -> np.ndarray:
+    """IRFFT (length L, 1/L scaling) of the spectrum kept up to bin k, by direct sums."""
+    re = _c(F.real, np.float64)
+    im = _c(F.imag, np.float64)
+    y = np.zeros(L)
+    _get().orc_irdft_lowpass(_p(re), _p(im), L, k, _p(y))
+    return y
+
+
+def sss(s: np.ndarray, L_rows: Sequence[int], alpha: float, rho: float,
+        kstar_force: Optional[Sequence[int]] = None, n_threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Spectral Score Smoothing of every row (AudioKV blog §2.2).
+
+    s is the concatenated scores; returns (s_hat concatenated, k* per row).
+    ``kstar_force[i] >= 0`` smooths row i at that cutoff instead of its own.
+    """
+    s = _c(s, np.float64)
+    L = _c(L_rows, np.int64)
+    off = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+    assert s.shape[0] == off[-1]
+    s_hat = np.zeros_like(s)
+    ks = np.zeros(len(L), np.int64)
+    kf = None if kstar_force is None else _c(kstar_force, np.int64)
+    _get().orc_sss_rows(len(L), _p(L), _p(off), _p(s), alpha, rho, None if kf is None else _p(kf), _p(s_hat),
+                        _p(ks), n_threads or default_threads())
+    return s_hat, ks
+
+
+# ---------------------------------------------------------------- step 3 ----
+class BudgetError(ValueError):
+    pass
+
+
+def allocate(S: np.ndarray, L_seq: Sequence[int], w: int, budget_pct: int, r: float) -> np.ndarray:
+    """Per-head budgets b [n_seq][layers][H] (AudioKV blog §3.1, §5.1)."""
+    S = _c(S, np.float32)
+    n_layers, H = S.shape
+    L = _c(L_seq, np.int64)
+    b = np.zeros((len(L), n_layers, H), np.int32)
+    st = _get().orc_allocate(len(L), _p(L), n_layers, H, w, budget_pct, C.c_float(r), _p(S), _p(b))
+    if st == 3:
+        raise BudgetError("budget below H*w")
+    if st:
+        raise ValueError(f"allocate failed ({st})")
+    return b
+
+
+# ---------------------------------------------------------------- step 4 ----
+def select(s_hat: np.ndarray, L_rows: Sequence[int], w: int, b_rows: Sequence[int],
+           n_threads: int = 0) -> list:
+    """Kept positions per row, ascending: last w + top-(b-w) of s_hat over [0, L-w)."""
+    s_hat = _c(s_hat, np.float64)
+    L = _c(L_rows, np.int64)
+    off = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+    b = _c(b_rows, np.int32)
+    keep = np.minimum(b.astype(np.int64), L)
+    ioff = np.concatenate([[0], np.cumsum(keep)]).astype(np.int64)
+    idx = np.zeros(max(1, ioff[-1]), np.int32)
+    _get().orc_select_rows(len(L), _p(L), _p(off), _p(s_hat), w, _p(b), _p(ioff), _p(idx),
+                           n_threads or default_threads())
+    return [idx[ioff[i]:ioff[i + 1]].copy() for i in range(len(L))]
+
+
+def gather(X: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """Compacted rows X[idx] (an index copy)."""
+    return np.ascontiguousarray(X[np.asarray(idx, np.int64)])
+
+
+# ---------------------------------------------------------------- step 5 ----
+class DecodeList:
+    """One KV head's kept cache as the ordered list of the VoxZip eviction rule.
+
+    Entries are in position order; arrays have room for one appended entry.
+    """
+
+    def __init__(self, K: np.ndarray, V: np.ndarray, pos: np.ndarray, A: Optional[np.ndarray] = None,
+                 extra: int = 1):
+        n, d = K.shape
+        cap = n + extra
+        self.d = d
+        self.n = C.c_int64(n)
+        self.K = np.zeros((cap, d), np.float32)
+        self.V = np.zeros((cap, d), np.float32)
+        self.A = np.zeros(cap, np.float64)
+        self.pos = np.zeros(cap, np.int64)
+        order = np.argsort(np.asarray(pos, np.int64), kind="stable")
+        self.K[:n] = np.asarray(K, np.float32)[order]
+        self.V[:n] = np.asarray(V, np.float32)[order]
+        self.pos[:n] = np.asarray(pos, np.int64)[order]
+        if A is not None:
+            self.A[:n] = np.asarray(A, np.float64)[order]
+
+    @property
+    def size(self) -> int:
+        return self.n.value
+
+    def step(self, q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray, pos_new: int, gamma: float, T: int,
+             M: int, b: int) -> Tuple[np.ndarray, int]:
+        """Append, attend, update A, evict (VoxZip second stage). Returns (o [g][d], evicted pos or -1)."""
+        if self.n.value + 1 > self.K.shape[0]:
+            raise ValueError("DecodeList capacity exceeded")
+        q = _c(q, np.float32)
+        g = q.shape[0]
+        o = np.zeros((g, self.d), np.float64)
+        ev = _get().orc_decode_step(C.byref(self.n), self.d, g, _p(self.K), _p(self.V), _p(self.A), _p(self.pos),
+                                    _p(q), _p(_c(k_new, np.float32)), _p(_c(v_new, np.float32)), int(pos_new),
+                                    gamma, T, M, b, _p(o))
+        return o, int(ev)
+
+    def entries(self):
+        n = self.n.value
+        return self.K[:n].copy(), self.V[:n].copy(), self.A[:n].copy(), self.pos[:n].copy()
+
+
+def recent_count(b: int, recent_pct: int) -> int:
+    """M = floor(recent_pct * b / 100) (VoxZip: recent window = 20% of the budget)."""
+    return (recent_pct * b) // 100
+
+
+def decode_run_heads(Kc_list, Vc_list, pos_list, q, k_new, v_new, pos0, gamma, T, M, b, n_threads: int = 0):
+    """Run every head's decode steps independently (CPU baseline).
+
+    q [steps][heads][g][d]; k_new, v_new [steps][heads][d]. Returns
+    (o [steps][heads][g][d] float64, evicted [steps][heads]).
+    """
+    heads = len(Kc_list)
+    steps, _, g, d = q.shape
+    caps = [len(k) + 1 for k in Kc_list]
+    off = np.concatenate([[0], np.cumsum(caps)]).astype(np.int64)
+    Kc = np.zeros((off[-1], d), np.float32)
+    Vc = np.zeros((off[-1], d), np.float32)
+    A = np.zeros(off[-1], np.float64)
+    pos = np.zeros(off[-1], np.int64)
+    n = np.zeros(heads, np.int64)
+    for h in range(heads):
+        order = np.argsort(pos_list[h], kind="stable")
+        k = len(Kc_list[h])
+        Kc[off[h]:off[h] + k] = Kc_list[h][order]
+        Vc[off[h]:off[h] + k] = Vc_list[h][order]
+        pos[off[h]:off[h] + k] = np.asarray(pos_list[h])[order]
+        n[h] = k
+    o = np.zeros((steps, heads, g, d), np.float64)
+    ev = np.zeros((steps, heads), np.int64)
+    _get().orc_decode_run_heads(heads, _p(n), d, g, _p(Kc), _p(Vc), _p(A), _p(pos), _p(off), steps,
+                                _p(_c(q, np.float32)), _p(_c(k_new, np.float32)), _p(_c(v_new, np.float32)),
+                                _p(_c(pos0, np.int64)), gamma, T, _p(_c(M, np.int32)), _p(_c(b, np.int64)),
+                                _p(o), _p(ev), n_threads or default_threads())
+    return o, ev
+
+
+__all__ = ["build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
+           "gather", "DecodeList", "recent_count", "decode_run_heads", "default_threads"]

@@ -1,0 +1,583 @@
+/*
+ * CPU oracle for the attention-score-driven KV selection and compaction path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product library may link, load or
+ * call this file; only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark use it. It shares no code, header, table or constant with the
+ * CUDA path. It is plain, slow, double-precision C that restates each step of
+ * the method in the order and notation of the pages:
+ *
+ *   [AudioKV]  AudioKV blog post ("1. 音频语言模型中的KV缓存挑战 ..."),
+ *              §1.2 (raw importance scores), §2.2 (Spectral Score Smoothing),
+ *              §3.1 (head-aware allocation), §5.1 (deployment parameters).
+ *   [AudioKV-abs] "AudioKV: KV Cache Eviction in Efficient Large Audio
+ *              Language Models" (arxivlens abstract): SSS is an FFT low-pass.
+ *   [VoxZip]   "VoxZip: Semantic-Anchored Temporal KV Cache Compression for
+ *              Long-Context Audio Inference", 方法概述和架构, second stage
+ *              (Temporally Decayed KV Cache Eviction): the A^(t) update and the
+ *              Concat(K[:T], K[I_hist], K[-M:]) rule; 细节详述 (gamma, T, M).
+ *   [C3]       "C3: Speech-Guided KV Retrieval for Long-Context SpeechLLM
+ *              Inference": the budget bypass (audio length <= B keeps all).
+ *
+ * Readings of points the pages leave open are marked READING in the comments.
+ *
+ * Parity status: every function here is pinned by closed forms, invariants,
+ * brute force or an independent library routine in tests/test_oracle_*.py.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC -pthread
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef M_PI
+#define M_PI 3.14159265358979323846
+#endif
+
+/* ------------------------------------------------------------------------- */
+/* A tiny thread pool: run fn(i, ctx) for i in [0, n) on up to n_threads.     */
+/* ------------------------------------------------------------------------- */
+typedef void (*orc_task_fn)(int64_t i, void* ctx);
+typedef struct {
+  orc_task_fn fn;
+  void* ctx;
+  int64_t n;
+  int64_t next;
+  pthread_mutex_t mu;
+} orc_pool;
+
+static void* orc_worker(void* arg) {
+  orc_pool* p = (orc_pool*)arg;
+  for (;;) {
+    pthread_mutex_lock(&p->mu);
+    int64_t i = p->next++;
+    pthread_mutex_unlock(&p->mu);
+    if (i >= p->n) break;
+    p->fn(i, p->ctx);
+  }
+  return NULL;
+}
+
+static void orc_parallel(int64_t n, int n_threads, orc_task_fn fn, void* ctx) {
+  if (n_threads <= 1 || n <= 1) {
+    for (int64_t i = 0; i < n; ++i) fn(i, ctx);
+    return;
+  }
+  if (n_threads > n) n_threads = (int)n;
+  orc_pool p = {fn, ctx, n, 0, PTHREAD_MUTEX_INITIALIZER};
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)n_threads);
+  int started = 0;
+  for (int t = 0; t < n_threads; ++t)
+    if (pthread_create(&th[t], NULL, orc_worker, &p) == 0) ++started;
+  if (started == 0) orc_worker(&p);
+  for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+  free(th);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 1. Observation-window importance scores ([AudioKV] §1.2 names the raw */
+/* importance scores of SnapKV/AdaKV that SSS smooths).                       */
+/* s_j = sum over the R = g*w window queries r of softmax_j(q_r . K_j / sqrt d)*/
+/* READING: every one of the L audio keys is visible to every window query    */
+/* (no causal mask), no pooling, a sum (not a mean) over the group's heads.   */
+/* ------------------------------------------------------------------------- */
+void orc_score_row(const float* q, int R, const float* K, int64_t L, int d, double* s) {
+  double* x = (double*)malloc(sizeof(double) * (size_t)L);
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  for (int64_t j = 0; j < L; ++j) s[j] = 0.0;
+  for (int r = 0; r < R; ++r) {
+    const float* qr = q + (size_t)r * d;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < L; ++j) {
+      const float* kj = K + (size_t)j * d;
+      double dot = 0.0;
+      for (int c = 0; c < d; ++c) dot += (double)qr[c] * (double)kj[c];
+      x[j] = dot * inv_sqrt_d;
+      if (x[j] > m) m = x[j];
+    }
+    double Z = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+      x[j] = exp(x[j] - m);
+      Z += x[j];
+    }
+    for (int64_t j = 0; j < L; ++j) s[j] += x[j] / Z;
+  }
+  free(x);
+}
+
+typedef struct {
+  const int64_t* L;
+  const int64_t* key_off;
+  const float* qwin;
+  int R, d;
+  const float* K;
+  double* s;
+} score_ctx;
+
+static void score_task(int64_t i, void* vctx) {
+  score_ctx* c = (score_ctx*)vctx;
+  orc_score_row(c->qwin + (size_t)i * c->R * c->d, c->R, c->K + (size_t)c->key_off[i] * c->d,
+                c->L[i], c->d, c->s + c->key_off[i]);
+}
+
+/* rows: qwin [n_rows][R][d]; K concatenated [sum L][d] (row i starts at key_off[i]);
+ * s concatenated like K's rows. */
+void orc_score_rows(int64_t n_rows, const int64_t* L, const int64_t* key_off, const float* qwin, int R,
+                    int d, const float* K, double* s, int n_threads) {
+  score_ctx c = {L, key_off, qwin, R, d, K, s};
+  orc_parallel(n_rows, n_threads, score_task, &c);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 2. Spectral Score Smoothing ([AudioKV] §2.2; [AudioKV-abs]).          */
+/*   F = RFFT(s); E(k) = sum_{i<=k} |F_i|^2; k* = min{k : E(k) >= rho E(L/2)};  */
+/*   s_hat = (1 - alpha) s + alpha * IRFFT(F . lowpass(k*)).                   */
+/* READINGS: the garbled blend reads s_hat = (1-a)s + a*IRFFT(F.w); the filter */
+/* w is the brick wall 1[i <= k*]; E starts at the DC bin and uses one-sided   */
+/* bins without doubling; IRFFT has numpy irfft semantics (1/L scaling, real   */
+/* parts of bins 0 and L/2 only); L is even.                                    */
+/* ------------------------------------------------------------------------- */
+
+/* cos/sin(2 pi m / L) for m in [0, L): angles reduced exactly by index. */
+static void twiddles(int64_t L, double* c, double* sn) {
+  for (int64_t m = 0; m < L; ++m) {
+    double a = 2.0 * M_PI * (double)m / (double)L;
+    c[m] = cos(a);
+    sn[m] = sin(a);
+  }
+}
+
+/* Direct DFT, bins i = 0..L/2: F_i = sum_n s_n exp(-2 pi i i n / L). */
+void orc_rdft(const double* s, int64_t L, double* re, double* im) {
+  double* c = (double*)malloc(sizeof(double) * (size_t)L);
+  double* sn = (double*)malloc(sizeof(double) * (size_t)L);
+  twiddles(L, c, sn);
+  for (int64_t i = 0; i <= L / 2; ++i) {
+    double a = 0.0, b = 0.0;
+    int64_t m = 0; /* (i * n) mod L */
+    for (int64_t n = 0; n < L; ++n) {
+      a += s[n] * c[m];
+      b -= s[n] * sn[m];
+      m += i;
+      if (m >= L) m -= L;
+    }
+    re[i] = a;
+    im[i] = b;
+  }
+  free(c);
+  free(sn);
+}
+
+/* Energy prefix E(k), k = 0..L/2, summed in index order; returns k*. */
+int64_t orc_kstar(const double* re, const double* im, int64_t L, double rho, double* E) {
+  double acc = 0.0;
+  for (int64_t i = 0; i <= L / 2; ++i) {
+    acc += re[i] * re[i] + im[i] * im[i];
+    E[i] = acc;
+  }
+  double thr = rho * E[L / 2];
+  for (int64_t k = 0; k <= L / 2; ++k)
+    if (E[k] >= thr) return k;
+  return L / 2;
+}
+
+/* y = IRFFT(F . 1[i <= kstar], n = L), direct sum:
+ * y_n = (1/L) [ Re F_0 + 2 sum_{0<i<=k*, i<L/2} Re(F_i e^{+2 pi i i n/L})
+ *               + (k* = L/2 ? Re F_{L/2} (-1)^n : 0) ]. */
+void orc_irdft_lowpass(const double* re, const double* im, int64_t L, int64_t kstar, double* y) {
+  double* c = (double*)malloc(sizeof(double) * (size_t)L);
+  double* sn = (double*)malloc(sizeof(double) * (size_t)L);
+  twiddles(L, c, sn);
+  int64_t top = kstar < L / 2 ? kstar : L / 2 - 1;
+  for (int64_t n = 0; n < L; ++n) {
+    double acc = re[0];
+    int64_t m = 0; /* (i * n) mod L */
+    for (int64_t i = 1; i <= top; ++i) {
+      m += n;
+      if (m >= L) m -= L;
+      acc += 2.0 * (re[i] * c[m] - im[i] * sn[m]);
+    }
+    if (kstar >= L / 2) acc += (n % 2 == 0 ? re[L / 2] : -re[L / 2]);
+    y[n] = acc / (double)L;
+  }
+  free(c);
+  free(sn);
+}
+
+/* One row. kstar_force < 0: compute k*; else smooth at the given k*. */
+void orc_sss_row(const double* s, int64_t L, double alpha, double rho, int64_t kstar_force,
+                 double* s_hat, int64_t* kstar_out, double* E_out) {
+  int64_t nb = L / 2 + 1;
+  double* re = (double*)malloc(sizeof(double) * (size_t)nb);
+  double* im = (double*)malloc(sizeof(double) * (size_t)nb);
+  double* E = E_out ? E_out : (double*)malloc(sizeof(double) * (size_t)nb);
+  double* y = (double*)malloc(sizeof(double) * (size_t)L);
+  orc_rdft(s, L, re, im);
+  int64_t ks = orc_kstar(re, im, L, rho, E);
+  if (kstar_force >= 0) ks = kstar_force;
+  orc_irdft_lowpass(re, im, L, ks, y);
+  for (int64_t n = 0; n < L; ++n) s_hat[n] = (1.0 - alpha) * s[n] + alpha * y[n];
+  *kstar_out = ks;
+  free(re);
+  free(im);
+  if (!E_out) free(E);
+  free(y);
+}
+
+typedef struct {
+  const int64_t* L;
+  const int64_t* off;
+  const double* s;
+  double alpha, rho;
+  const int64_t* kstar_force;
+  double* s_hat;
+  int64_t* kstar;
+} sss_ctx;
+
+static void sss_task(int64_t i, void* vctx) {
+  sss_ctx* c = (sss_ctx*)vctx;
+  int64_t kf = c->kstar_force ? c->kstar_force[i] : -1;
+  orc_sss_row(c->s + c->off[i], c->L[i], c->alpha, c->rho, kf, c->s_hat + c->off[i], &c->kstar[i], NULL);
+}
+
+void orc_sss_rows(int64_t n_rows, const int64_t* L, const int64_t* off, const double* s, double alpha,
+                  double rho, const int64_t* kstar_force, double* s_hat, int64_t* kstar, int n_threads) {
+  sss_ctx c = {L, off, s, alpha, rho, kstar_force, s_hat, kstar};
+  orc_parallel(n_rows, n_threads, sss_task, &c);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 3. Head-aware budget allocation ([AudioKV] §3.1, §5.1).               */
+/*   b_{l,h} = w + r B_rem / H + (1 - r) B_rem S_{l,h} / sum_h S_{l,h}          */
+/* READINGS: per layer over that layer's H KV heads; budget_pct is the kept   */
+/* fraction, B = floor(pct L H / 100) in integers, B_rem = B - H w; b_h =      */
+/* floor(x_h), the remainder B - sum b_h goes +1 to the largest fractional     */
+/* parts (ties to the lower head); a head with b_h > L is capped at L and the  */
+/* others are re-allocated with what is left; sum S = 0 splits evenly.         */
+/* Evaluation order (fixed): t1 = r*B_rem; t1 = t1/H; t2 = (1-r)*B_rem;        */
+/* t2 = t2*S_h; t2 = t2/sumS; x = (w + t1) + t2, all in double, no FMA.        */
+/* Returns 0, or 3 when B_rem < 0 (budget below H*w).                          */
+/* ------------------------------------------------------------------------- */
+static int alloc_layer(int H, int64_t L, int w, int64_t B, double r, const float* S, int32_t* b) {
+  int active[1024];
+  double xs[1024];
+  int n_act = 0;
+  for (int h = 0; h < H; ++h) active[n_act++] = h;
+  int64_t B_left = B;
+  for (;;) {
+    if (n_act == 0) return 0;
+    int64_t B_rem = B_left - (int64_t)n_act * w;
+    if (B_rem < 0) return 3;
+    double sumS = 0.0;
+    for (int a = 0; a < n_act; ++a) sumS += (double)S[active[a]];
+    int64_t sum_b = 0;
+    for (int a = 0; a < n_act; ++a) {
+      int h = active[a];
+      double x;
+      if (sumS > 0.0) {
+        double t1 = r * (double)B_rem;
+        t1 = t1 / (double)n_act;
+        double t2 = (1.0 - r) * (double)B_rem;
+        t2 = t2 * (double)S[h];
+        t2 = t2 / sumS;
+        x = ((double)w + t1) + t2;
+      } else {
+        x = (double)w + (double)B_rem / (double)n_act;
+      }
+      xs[a] = x;
+      b[h] = (int32_t)floor(x);
+      sum_b += b[h];
+    }
+    int64_t rem = B_left - sum_b;
+    /* +1 to the rem largest fractional parts, ties to the lower head index */
+    char taken[1024];
+    memset(taken, 0, sizeof(taken));
+    for (int64_t k = 0; k < rem; ++k) {
+      int best = -1;
+      double bf = -1.0;
+      for (int a = 0; a < n_act; ++a) {
+        if (taken[a]) continue;
+        double f = xs[a] - floor(xs[a]);
+        if (f > bf) { bf = f; best = a; }
+      }
+      if (best < 0) break;
+      taken[best] = 1;
+      b[active[best]] += 1;
+    }
+    int capped = 0;
+    int keep[1024];
+    int n_keep = 0;
+    for (int a = 0; a < n_act; ++a) {
+      int h = active[a];
+      if (b[h] > L) {
+        b[h] = (int32_t)L;
+        B_left -= L;
+        capped = 1;
+      } else {
+        keep[n_keep++] = h;
+      }
+    }
+    if (!capped) return 0;
+    for (int a = 0; a < n_keep; ++a) active[a] = keep[a];
+    n_act = n_keep;
+  }
+}
+
+/* S [n_layers][H]; L per sequence; b [n_seq][n_layers][H]. */
+int orc_allocate(int n_seq, const int64_t* L, int n_layers, int H, int w, int budget_pct, float r,
+                 const float* S, int32_t* b) {
+  if (H > 1024) return 1;
+  for (int s = 0; s < n_seq; ++s) {
+    int64_t B = ((int64_t)budget_pct * L[s] * H) / 100;
+    for (int l = 0; l < n_layers; ++l) {
+      int st = alloc_layer(H, L[s], w, B, (double)r, S + (size_t)l * H, b + ((size_t)s * n_layers + l) * H);
+      if (st) return st;
+    }
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 4. Per-head selection ([AudioKV] §3.1 keeps a basic local context     */
+/* window; the rest goes by smoothed score).                                   */
+/* READINGS: the last w of the L positions are always kept and count toward b;*/
+/* the other b - w are the largest s_hat over [0, L - w), ties to the lower    */
+/* index (a full sort on (-s_hat, j)); b >= L keeps all ([C3] bypass);         */
+/* output ascending.                                                            */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+  double v;
+  int32_t j;
+} keyed;
+
+static int cmp_desc_then_index(const void* pa, const void* pb) {
+  const keyed* a = (const keyed*)pa;
+  const keyed* b = (const keyed*)pb;
+  if (a->v > b->v) return -1;
+  if (a->v < b->v) return 1;
+  return (a->j > b->j) - (a->j < b->j);
+}
+
+static int cmp_int32(const void* pa, const void* pb) {
+  int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+  return (a > b) - (a < b);
+}
+
+void orc_select_row(const double* s_hat, int64_t L, int w, int64_t b, int32_t* idx) {
+  if (b >= L) {
+    for (int64_t j = 0; j < L; ++j) idx[j] = (int32_t)j;
+    return;
+  }
+  int64_t n = L - w;
+  keyed* k = (keyed*)malloc(sizeof(keyed) * (size_t)(n > 0 ? n : 1));
+  for (int64_t j = 0; j < n; ++j) {
+    k[j].v = s_hat[j] == 0.0 ? 0.0 : s_hat[j]; /* -0 == +0 */
+    k[j].j = (int32_t)j;
+  }
+  qsort(k, (size_t)n, sizeof(keyed), cmp_desc_then_index);
+  int64_t top = b - w;
+  for (int64_t i = 0; i < top; ++i) idx[i] = k[i].j;
+  for (int64_t i = 0; i < w; ++i) idx[top + i] = (int32_t)(n + i);
+  qsort(idx, (size_t)b, sizeof(int32_t), cmp_int32);
+  free(k);
+}
+
+typedef struct {
+  const int64_t* L;
+  const int64_t* off;
+  const double* s_hat;
+  int w;
+  const int32_t* b;
+  const int64_t* idx_off;
+  int32_t* idx;
+} sel_ctx;
+
+static void sel_task(int64_t i, void* vctx) {
+  sel_ctx* c = (sel_ctx*)vctx;
+  orc_select_row(c->s_hat + c->off[i], c->L[i], c->w, c->b[i], c->idx + c->idx_off[i]);
+}
+
+void orc_select_rows(int64_t n_rows, const int64_t* L, const int64_t* off, const double* s_hat, int w,
+                     const int32_t* b, const int64_t* idx_off, int32_t* idx, int n_threads) {
+  sel_ctx c = {L, off, s_hat, w, b, idx_off, idx};
+  orc_parallel(n_rows, n_threads, sel_task, &c);
+}
+
+/* Gather: Kc[i] = K[idx[i]] (an index copy). */
+void orc_gather_row(const float* K, int d, const int32_t* idx, int64_t n, float* Kc) {
+  for (int64_t i = 0; i < n; ++i) memcpy(Kc + (size_t)i * d, K + (size_t)idx[i] * d, sizeof(float) * (size_t)d);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 5. One decode step of one KV head over its kept cache ([VoxZip],       */
+/* second stage):                                                               */
+/*   append (k_t, v_t);  p_g = softmax(q_{t,g} K_t^T / sqrt d) over the list;   */
+/*   o_g = p_g V_t;  A^(t) = gamma [A^(t-1), 0] + sum_g p_g;                     */
+/*   if the list holds more than b entries:                                     */
+/*     K_{t+1} = Concat(K_t[:T], K_t[I_hist], K_t[-M:]), V and A likewise,       */
+/*     I_hist = the top-N middle entries by A, N = b - T - M.                    */
+/* READINGS: A^(0) = 0 for the prefill entries; A is carried per entry and     */
+/* cropped with the same index set as K and V; the g query heads of the group  */
+/* add their softmaxes into one A; the output uses the list before eviction;   */
+/* ties in A keep the lower position (the higher one is evicted).              */
+/* The list is in position order. Arrays hold n entries on entry and the       */
+/* caller provides room for n + 1.                                              */
+/* Returns the evicted position, or -1 when nothing was evicted.                */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+  double A;
+  int64_t pos;
+  int64_t at; /* index in the middle part */
+} mid_entry;
+
+static int cmp_mid(const void* pa, const void* pb) {
+  const mid_entry* a = (const mid_entry*)pa;
+  const mid_entry* b = (const mid_entry*)pb;
+  if (a->A > b->A) return -1;
+  if (a->A < b->A) return 1;
+  return (a->pos > b->pos) - (a->pos < b->pos);
+}
+
+int64_t orc_decode_step(int64_t* n_io, int d, int g, float* Kc, float* Vc, double* A, int64_t* pos,
+                        const float* q, const float* k_new, const float* v_new, int64_t pos_new, double gamma,
+                        int T, int M, int64_t b, double* o) {
+  int64_t n = *n_io;
+  /* append */
+  memcpy(Kc + (size_t)n * d, k_new, sizeof(float) * (size_t)d);
+  memcpy(Vc + (size_t)n * d, v_new, sizeof(float) * (size_t)d);
+  A[n] = 0.0;
+  pos[n] = pos_new;
+  n += 1;
+  /* attention per query head, and the decayed score update */
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  double* x = (double*)malloc(sizeof(double) * (size_t)n);
+  double* padd = (double*)calloc((size_t)n, sizeof(double));
+  for (int gi = 0; gi < g; ++gi) {
+    const float* qg = q + (size_t)gi * d;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) {
+      double dot = 0.0;
+      for (int c = 0; c < d; ++c) dot += (double)qg[c] * (double)Kc[(size_t)j * d + c];
+      x[j] = dot * inv_sqrt_d;
+      if (x[j] > m) m = x[j];
+    }
+    double Z = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+      x[j] = exp(x[j] - m);
+      Z += x[j];
+    }
+    double* og = o + (size_t)gi * d;
+    for (int c = 0; c < d; ++c) og[c] = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+      double p = x[j] / Z;
+      padd[j] += p;
+      for (int c = 0; c < d; ++c) og[c] += p * (double)Vc[(size_t)j * d + c];
+    }
+  }
+  for (int64_t j = 0; j < n; ++j) A[j] = gamma * A[j] + padd[j];
+  free(x);
+  free(padd);
+
+  int64_t evicted = -1;
+  if (n > b) {
+    /* Concat(K[:T], K[I_hist], K[-M:]): keep the first T, the last M, and the
+     * top-N of the middle by A; the middle keeps its original order. */
+    int64_t N = b - T - M;
+    int64_t mid0 = T, mid1 = n - M; /* middle = [mid0, mid1) */
+    int64_t nm = mid1 - mid0;
+    mid_entry* me = (mid_entry*)malloc(sizeof(mid_entry) * (size_t)(nm > 0 ? nm : 1));
+    for (int64_t i = 0; i < nm; ++i) {
+      me[i].A = A[mid0 + i];
+      me[i].pos = pos[mid0 + i];
+      me[i].at = i;
+    }
+    qsort(me, (size_t)nm, sizeof(mid_entry), cmp_mid);
+    char* keep = (char*)calloc((size_t)(nm > 0 ? nm : 1), 1);
+    for (int64_t i = 0; i < N && i < nm; ++i) keep[me[i].at] = 1;
+    int64_t wr = mid0;
+    for (int64_t i = 0; i < nm; ++i) {
+      int64_t src = mid0 + i;
+      if (!keep[i]) {
+        evicted = pos[src];
+        continue;
+      }
+      if (wr != src) {
+        memmove(Kc + (size_t)wr * d, Kc + (size_t)src * d, sizeof(float) * (size_t)d);
+        memmove(Vc + (size_t)wr * d, Vc + (size_t)src * d, sizeof(float) * (size_t)d);
+        A[wr] = A[src];
+        pos[wr] = pos[src];
+      }
+      ++wr;
+    }
+    for (int64_t src = mid1; src < n; ++src, ++wr) {
+      memmove(Kc + (size_t)wr * d, Kc + (size_t)src * d, sizeof(float) * (size_t)d);
+      memmove(Vc + (size_t)wr * d, Vc + (size_t)src * d, sizeof(float) * (size_t)d);
+      A[wr] = A[src];
+      pos[wr] = pos[src];
+    }
+    n = wr;
+    free(me);
+    free(keep);
+  }
+  *n_io = n;
+  return evicted;
+}
+
+/* Many steps of one head (used to time the oracle as a CPU baseline).
+ * q [steps][g][d], k_new/v_new [steps][d], o [steps][g][d], evicted [steps].
+ * Cache arrays need room for b + 1 entries (or n + steps without eviction). */
+void orc_decode_run(int64_t* n_io, int d, int g, float* Kc, float* Vc, double* A, int64_t* pos,
+                    int64_t steps, const float* q, const float* k_new, const float* v_new, int64_t pos0,
+                    double gamma, int T, int M, int64_t b, double* o, int64_t* evicted) {
+  for (int64_t t = 0; t < steps; ++t) {
+    evicted[t] = orc_decode_step(n_io, d, g, Kc, Vc, A, pos, q + (size_t)t * g * d, k_new + (size_t)t * d,
+                                 v_new + (size_t)t * d, pos0 + t, gamma, T, M, b, o + (size_t)t * g * d);
+  }
+}
+
+/* Independent heads in parallel (CPU baseline). Per head h the arrays start at
+ * cache_off[h] * d (Kc, Vc) / cache_off[h] (A, pos); q/k/v/o/evicted are laid
+ * out [steps][heads][...]. */
+typedef struct {
+  int64_t* n;
+  int d, g;
+  float* Kc;
+  float* Vc;
+  double* A;
+  int64_t* pos;
+  const int64_t* cache_off;
+  int64_t heads, steps;
+  const float* q;
+  const float* k_new;
+  const float* v_new;
+  const int64_t* pos0;
+  double gamma;
+  int T;
+  const int32_t* M;
+  const int64_t* b;
+  double* o;
+  int64_t* evicted;
+} drun_ctx;
+
+static void drun_task(int64_t h, void* vctx) {
+  drun_ctx* c = (drun_ctx*)vctx;
+  int64_t off = c->cache_off[h];
+  for (int64_t t = 0; t < c->steps; ++t) {
+    size_t qo = ((size_t)t * c->heads + h) * c->g * c->d;
+    size_t ko = ((size_t)t * c->heads + h) * c->d;
+    c->evicted[t * c->heads + h] =
+        orc_decode_step(&c->n[h], c->d, c->g, c->Kc + (size_t)off * c->d, c->Vc + (size_t)off * c->d,
+                        c->A + off, c->pos + off, c->q + qo, c->k_new + ko, c->v_new + ko, c->pos0[h] + t,
+                        c->gamma, c->T, c->M[h], c->b[h], c->o + qo);
+  }
+}
+
+void orc_decode_run_heads(int64_t heads, int64_t* n, int d, int g, float* Kc, float* Vc, double* A, int64_t* pos,
+                          const int64_t* cache_off, int64_t steps, const float* q, const float* k_new,
+                          const float* v_new, const int64_t* pos0, double gamma, int T, const int32_t* M,
+                          const int64_t* b, double* o, int64_t* evicted, int n_threads) {
+  drun_ctx c = {n, d, g, Kc, Vc, A, pos, cache_off, heads, steps, q, k_new, v_new, pos0, gamma, T, M, b, o, evicted};
+  orc_parallel(heads, n_threads, drun_task, &c);
+}
