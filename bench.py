@@ -1,0 +1,353 @@
+#!/usr/bin/env python
+"""Benchmark of the KV selection/compaction path on B200.
+
+One step = one pass of the whole path over one batch of the workload:
+kv_allocate -> kv_score -> kv_sss -> kv_select_gather -> kv_decode_init ->
+the workload's decode steps (kv_decode_attn_update, all layers per launch).
+`value` = audio tokens of the batch processed per second of step time (for N
+ranks: N x that, each rank running its own replica; no data-path collective).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3b]
+       python bench.py --impl reference ...   (the CPU oracle as the arm)
+Multi-GPU: python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "compressed audio tokens/s (score→SSS→top-k→gather), decode µs/step; % HBM peak"
+UNIT = "audio tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def describe(cfg: synth.Config) -> str:
+    return (f"{cfg.name}: {cfg.n_seq} seq, L={list(cfg.L)}, {cfg.n_layers} layers, "
+            f"{cfg.n_kv_heads * cfg.group} q / {cfg.n_kv_heads} kv heads, d={cfg.head_dim}, {cfg.dtype}, w={cfg.w}, "
+            f"budget {cfg.budget_pct}%, alpha={cfg.alpha}, rho={cfg.rho}, r={cfg.r}, {cfg.decode_steps} decode steps "
+            f"(gamma={cfg.gamma}, T={cfg.sinks_T}, M={cfg.recent_pct}%)")
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------- clocks --
+class ClockSampler:
+    """Samples the SM clock and throttle reasons through NVML (read-only)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, torch_dev: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU baseline --
+def oracle_sample(cfg: synth.Config, bt: synth.Batch, rows, n_threads: int):
+    """Runs the oracle's whole path on `rows` of the batch; returns seconds."""
+    import oracle as orc
+
+    t0 = time.perf_counter()
+    L_rows = [int(bt.L_rows[r]) for r in rows]
+    koff = bt.key_off
+    Ks = np.concatenate([bt.K[koff[r]:koff[r + 1]] for r in rows])
+    b_all = orc.allocate(bt.S, cfg.L, cfg.w, cfg.budget_pct, cfg.r).reshape(-1)
+    s = orc.score(bt.qwin[rows], Ks, L_rows, n_threads=n_threads)
+    if bt.spikes is not None:
+        s = s * np.concatenate([np.where(bt.spikes[koff[r]:koff[r + 1]], 10.0, 1.0) for r in rows])
+    s_hat, _ = orc.sss(s, L_rows, cfg.alpha, cfg.rho, n_threads=n_threads)
+    b = [int(b_all[r]) for r in rows]
+    idx = orc.select(s_hat, L_rows, cfg.w, b, n_threads=n_threads)
+    Kc = [bt.K[koff[r] + idx[i]] for i, r in enumerate(rows)]
+    Vc = [bt.V[koff[r] + idx[i]] for i, r in enumerate(rows)]
+    M = [orc.recent_count(x, cfg.recent_pct) for x in b]
+    orc.decode_run_heads(Kc, Vc, idx, bt.q_dec[:, rows], bt.k_dec[:, rows], bt.v_dec[:, rows],
+                         np.array(L_rows, np.int64), cfg.gamma, cfg.sinks_T, M, np.array(b, np.int64),
+                         n_threads=n_threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, bt, n_rows_sample: int):
+    import oracle as orc
+
+    threads = orc.default_threads()
+    rows = list(range(min(n_rows_sample, cfg.rows)))
+    orc.build()
+    secs = oracle_sample(cfg, bt, rows, threads)
+    full = secs * cfg.rows / len(rows)  # the rows of one batch are independent
+    tokens = sum(cfg.L)
+    return {"value": tokens / full, "unit": UNIT, "cores": min(threads, len(rows)), "kind": "oracle",
+            "sample": f"{len(rows)} of {cfg.rows} rows through the whole path incl. {cfg.decode_steps} decode steps "
+                      f"({secs:.2f} s), scaled to one batch"}
+
+
+# ------------------------------------------------------------------ our arm --
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import kv_cache_compression_layer_b200 as kv
+    from kv_cache_compression_layer_b200 import Compressor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    cfg = synth.CONFIGS[args.config].with_(seed=rank)
+    bt = synth.make_batch(cfg)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    shape = kv.make_shape(cfg.n_layers, cfg.n_kv_heads, cfg.group, cfg.head_dim, cfg.w,
+                          kv.KV_BF16 if cfg.dtype == "bf16" else kv.KV_F32)
+    params = kv.make_params(cfg.budget_pct, cfg.alpha, cfg.rho, cfg.r, cfg.gamma, cfg.sinks_T, cfg.recent_pct)
+
+    def h(x, dtype):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dtype)
+
+    host = {"qwin": h(bt.qwin, dt), "K": h(bt.K, dt), "V": h(bt.V, dt), "S": h(bt.S, torch.float32),
+            "q": h(bt.q_dec, dt), "k": h(bt.k_dec, dt), "v": h(bt.v_dec, dt)}
+    if bt.spikes is not None:
+        host["spikes"] = h(np.where(bt.spikes, 10.0, 1.0), torch.float32)
+    d_in = {k: v.to(dev) for k, v in host.items()}
+    comp = Compressor(shape, cfg.L, params, device=dev)
+    D = cfg.decode_steps
+    out = torch.empty(D, cfg.rows, cfg.group, cfg.head_dim, dtype=dt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+
+    def step(x, dec_events=None):
+        comp.compress(x["qwin"], x["K"], x["V"], x["S"], spikes=x.get("spikes"), stream=stream)
+        for t in range(D):
+            if dec_events is not None:
+                dec_events[t][0].record(stream)
+            comp.decode_step(x["q"][t], x["k"][t], x["v"][t], out[t], stream=stream)
+            if dec_events is not None:
+                dec_events[t][1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        step(d_in)
+    torch.cuda.synchronize()
+    st = kv.kv_read_device_status(comp.status, stream) | kv.kv_read_device_status(comp.ws[:4].view(torch.int32),
+                                                                                  stream)
+    if st:
+        raise RuntimeError(f"device status {st:#x} after warm-up")
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    step_ev = [(E(), E(), E()) for _ in range(args.steps)]
+    dec_ev = [[(E(), E()) for _ in range(D)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            step_ev[i][0].record(stream)
+            comp.compress(d_in["qwin"], d_in["K"], d_in["V"], d_in["S"], spikes=d_in.get("spikes"), stream=stream)
+            step_ev[i][1].record(stream)
+            for t in range(D):
+                dec_ev[i][t][0].record(stream)
+                comp.decode_step(d_in["q"][t], d_in["k"][t], d_in["v"][t], out[t], stream=stream)
+                dec_ev[i][t][1].record(stream)
+            step_ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [a.elapsed_time(c) for a, _, c in step_ev]
+    comp_ms = [a.elapsed_time(b) for a, b, _ in step_ev]
+    dec_us = [1e3 * s.elapsed_time(e) for row in dec_ev for s, e in row]
+    ms = sum(step_ms) / len(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = sum(cfg.L)
+    value = world * tokens / (ms * 1e-3)
+
+    # end to end through the C ABI from pinned host buffers (copies and the
+    # read-back of the decode outputs inside the timed region)
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    out_host = torch.empty(out.shape, dtype=dt).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        a, c = E(), E()
+        a.record(stream)
+        for k, v in pinned.items():
+            d_in[k].copy_(v, non_blocking=True)
+        step(d_in)
+        out_host.copy_(out, non_blocking=True)
+        c.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(c))
+    e2e = sum(e2e_ms) / len(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+
+    # roofline of the dominant kernel (the decode step) and of the compress stage
+    b = comp.b.cpu().numpy().astype(np.int64)
+    d = cfg.head_dim
+    eb = 2 if cfg.dtype == "bf16" else 4
+    dec_bytes = int(((b + 1) * (2 * eb * d + 8) + 2 * eb * d).sum())
+    dec_avg_us = sum(dec_us) / len(dec_us)
+    L_rows = np.array([cfg.L[cfg.row_triplet(r)[0]] for r in range(cfg.rows)], np.int64)
+    comp_bytes = int((2 * eb * d * (L_rows + 3 * b)).sum())
+    comp_avg_ms = sum(comp_ms) / len(comp_ms)
+    peak, peak_kind = hbm_peak()
+    dec_gbs = dec_bytes / (dec_avg_us * 1e-6) / 1e9
+    comp_gbs = comp_bytes / (comp_avg_ms * 1e-3) / 1e9
+    launches_per_step = 2 + (3 if cfg.dtype == "bf16" else 3) + 1 + 2 + 1 + D
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic (seeded AR(1) keys, diagonal-band queries; stands in for long-audio workloads)",
+        "config": {"workload": describe(cfg), "n_seq": cfg.n_seq, "rows": cfg.rows,
+                   "l2": "256 MB write between timed steps (outside the events)",
+                   "parallelism": f"replicas x{world} (rows independent, no collective)"},
+        "stages": {"compress_ms": comp_avg_ms, "compress_tokens_per_s": world * tokens / (comp_avg_ms * 1e-3),
+                   "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
+                   "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
+                   "decode_bytes_alg": dec_bytes, "decode_steps": D},
+        "roofline": {"kernel": "decode_kernel (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": None,
+                     "peak_kind": peak_kind + " (hbm_gbs copy)"},
+        "e2e": {"value": world * tokens / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg, bt, args.cpu_rows)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ------------------------------------------------------------ reference arm --
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm, on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import oracle as orc
+
+    orc.build()
+    cfg = synth.CONFIGS[args.config]
+    rows = list(range(min(args.cpu_rows, cfg.rows)))
+    bt = synth.make_batch(cfg)
+    threads = orc.default_threads()
+    for _ in range(args.warmup):
+        oracle_sample(cfg, bt, rows[:1], threads)
+    secs = [oracle_sample(cfg, bt, rows, threads) for _ in range(args.steps)]
+    full = (sum(secs) / len(secs)) * cfg.rows / len(rows)
+    value = sum(cfg.L) / full
+    res = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": full * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded AR(1) keys, diagonal-band queries)",
+           "config": {"workload": describe(cfg), "n_seq": cfg.n_seq, "rows": cfg.rows},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, len(rows)), "kind": "oracle",
+                            "sample": f"{len(rows)} of {cfg.rows} rows per step, scaled to one batch"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="3b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

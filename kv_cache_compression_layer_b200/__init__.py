@@ -1,0 +1,200 @@
+"""Python binding of libkvcomp.so (the C ABI declared in include/kvcomp.h).
+
+Argument marshalling only: every step of the path runs in the library's
+sm_100a kernels. Functions take torch tensors (or raw device addresses as
+ints) and the current CUDA stream, and raise ``KvError`` on a non-zero
+status. The library must be built (``python -m
+kv_cache_compression_layer_b200.build``); importing the binding without it
+fails loudly, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvcomp.so")
+
+KV_OK, KV_ERR_ARG, KV_ERR_UNSUPPORTED_L, KV_ERR_BUDGET, KV_ERR_WORKSPACE, KV_ERR_CUDA, KV_ERR_TIMEOUT = range(7)
+KV_DEV_TIMEOUT, KV_DEV_BUDGET, KV_DEV_CAPACITY = 0x1, 0x2, 0x4
+KV_F32, KV_BF16 = 0, 1
+KV_MAX_SEQ = 64
+META_INTS = 8
+
+# Every symbol include/kvcomp.h declares.
+EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
+           "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
+           "kv_status_string")
+
+
+class kv_shape(C.Structure):
+    _fields_ = [("n_layers", C.c_int32), ("n_kv_heads", C.c_int32), ("group", C.c_int32), ("head_dim", C.c_int32),
+                ("w", C.c_int32), ("dtype", C.c_int32)]
+
+
+class kv_params(C.Structure):
+    _fields_ = [("budget_pct", C.c_int32), ("alpha", C.c_float), ("rho", C.c_float), ("r", C.c_float),
+                ("gamma", C.c_float), ("sinks_T", C.c_int32), ("recent_pct", C.c_int32)]
+
+
+class kv_cache(C.Structure):
+    _fields_ = [("Kc", C.c_void_p), ("Vc", C.c_void_p), ("A", C.c_void_p), ("pos", C.c_void_p),
+                ("slot_off", C.c_void_p), ("b", C.c_void_p), ("meta", C.c_void_p), ("status", C.c_void_p)]
+
+
+class KvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libkvcomp.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with python -m kv_cache_compression_layer_b200.build")
+        L = C.CDLL(LIB_PATH)
+        P, I32, SZ, I64 = C.c_void_p, C.c_int32, C.c_size_t, C.c_int64
+        Ps, Pp, Pc = C.POINTER(kv_shape), C.POINTER(kv_params), C.POINTER(kv_cache)
+        sig = {
+            "kv_rows": (I64, [Ps, I32]),
+            "kv_check_lengths": (C.c_int, [Ps, P, I32]),
+            "kv_workspace_bytes": (SZ, [Ps, P, I32]),
+            "kv_total_slots": (I64, [Ps, P, I32, Pp]),
+            "kv_score": (C.c_int, [Ps, P, I32, P, P, P, P, SZ, P]),
+            "kv_sss": (C.c_int, [Ps, P, I32, P, P, P, C.c_float, C.c_float, P]),
+            "kv_allocate": (C.c_int, [Ps, P, I32, Pp, P, P, P, P]),
+            "kv_select_gather": (C.c_int, [Ps, P, I32, P, P, P, P, P, P, P, P, P]),
+            "kv_decode_init": (C.c_int, [Ps, P, I32, Pp, Pc, P]),
+            "kv_decode_attn_update": (C.c_int, [Ps, P, I32, Pp, Pc, P, P, P, P, P]),
+            "kv_read_device_status": (C.c_int, [P, P, P]),
+            "kv_status_string": (C.c_char_p, [C.c_int]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(st: int) -> str:
+    return lib().kv_status_string(st).decode()
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _L(L: Sequence[int]):
+    arr = (C.c_int32 * len(L))(*[int(x) for x in L])
+    return arr, len(L)
+
+
+def _check(fn: str, st: int):
+    if st != KV_OK:
+        raise KvError(fn, st)
+
+
+def make_shape(n_layers: int, n_kv_heads: int, group: int, head_dim: int, w: int, dtype: int) -> kv_shape:
+    return kv_shape(n_layers, n_kv_heads, group, head_dim, w, dtype)
+
+
+def make_params(budget_pct: int, alpha: float, rho: float, r: float, gamma: float, sinks_T: int,
+                recent_pct: int) -> kv_params:
+    return kv_params(budget_pct, alpha, rho, r, gamma, sinks_T, recent_pct)
+
+
+def kv_rows(shape: kv_shape, n_seq: int) -> int:
+    return lib().kv_rows(C.byref(shape), n_seq)
+
+
+def kv_check_lengths(shape: kv_shape, L: Sequence[int]) -> int:
+    arr, n = _L(L)
+    return lib().kv_check_lengths(C.byref(shape), arr, n)
+
+
+def kv_workspace_bytes(shape: kv_shape, L: Sequence[int]) -> int:
+    arr, n = _L(L)
+    return lib().kv_workspace_bytes(C.byref(shape), arr, n)
+
+
+def kv_total_slots(shape: kv_shape, L: Sequence[int], params: kv_params) -> int:
+    arr, n = _L(L)
+    return lib().kv_total_slots(C.byref(shape), arr, n, C.byref(params))
+
+
+def kv_score(shape, L, qwin, K, s, ws, ws_bytes: Optional[int] = None, stream=None):
+    arr, n = _L(L)
+    nbytes = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+    _check("kv_score", lib().kv_score(C.byref(shape), arr, n, _ptr(qwin), _ptr(K), _ptr(s), _ptr(ws), nbytes,
+                                      _stream(stream)))
+
+
+def kv_sss(shape, L, s, s_hat, kstar, alpha: float, rho: float, stream=None):
+    arr, n = _L(L)
+    _check("kv_sss", lib().kv_sss(C.byref(shape), arr, n, _ptr(s), _ptr(s_hat), _ptr(kstar), alpha, rho,
+                                  _stream(stream)))
+
+
+def kv_allocate(shape, L, params, S, b, slot_off, stream=None):
+    arr, n = _L(L)
+    _check("kv_allocate", lib().kv_allocate(C.byref(shape), arr, n, C.byref(params), _ptr(S), _ptr(b),
+                                            _ptr(slot_off), _stream(stream)))
+
+
+def kv_select_gather(shape, L, s_hat, K, V, b, slot_off, idx, Kc, Vc, stream=None):
+    arr, n = _L(L)
+    _check("kv_select_gather", lib().kv_select_gather(C.byref(shape), arr, n, _ptr(s_hat), _ptr(K), _ptr(V),
+                                                      _ptr(b), _ptr(slot_off), _ptr(idx), _ptr(Kc), _ptr(Vc),
+                                                      _stream(stream)))
+
+
+def make_cache(Kc, Vc, A, pos, slot_off, b, meta, status) -> kv_cache:
+    return kv_cache(_ptr(Kc), _ptr(Vc), _ptr(A), _ptr(pos), _ptr(slot_off), _ptr(b), _ptr(meta), _ptr(status))
+
+
+def kv_decode_init(shape, L, params, cache: kv_cache, stream=None):
+    arr, n = _L(L)
+    _check("kv_decode_init", lib().kv_decode_init(C.byref(shape), arr, n, C.byref(params), C.byref(cache),
+                                                  _stream(stream)))
+
+
+def kv_decode_attn_update(shape, L, params, cache: kv_cache, q_t, k_t, v_t, out, stream=None):
+    arr, n = _L(L)
+    _check("kv_decode_attn_update",
+           lib().kv_decode_attn_update(C.byref(shape), arr, n, C.byref(params), C.byref(cache), _ptr(q_t),
+                                       _ptr(k_t), _ptr(v_t), _ptr(out), _stream(stream)))
+
+
+def kv_read_device_status(status_dev, stream=None) -> int:
+    host = C.c_int32(0)
+    _check("kv_read_device_status", lib().kv_read_device_status(_ptr(status_dev), C.byref(host), _stream(stream)))
+    return host.value
+
+
+from .pipeline import Compressor  # noqa: E402  (the torch-side convenience wrapper)
+
+__all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", "make_params", "make_cache",
+           "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
+           "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
+           "status_string", "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]

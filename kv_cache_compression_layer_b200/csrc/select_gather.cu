@@ -1,0 +1,192 @@
+// kv_select_gather: per-row top-k selection and compaction of the kept K/V
+// (AudioKV blog §3.1: a basic local window is always kept, the rest of the
+// row's budget goes to the highest smoothed scores; the C3 page's bypass keeps
+// every position once the budget reaches the audio length).
+//
+// select kernel (one CTA per row): smoothed scores become order-preserving
+// uint32 keys (-0 folded into +0) in shared memory; an MSB-first 8-bit radix
+// select finds the k-th largest key T and how many keys equal to T are taken;
+// a warp-ballot compaction then writes the kept indices in ascending order:
+// keys above T, the first (k - #above) keys equal to T, and the window.
+//
+// gather kernel (persistent, all SMs): warps walk the compacted slots in
+// units of 32, and copy each kept K and V row with 16-byte loads/stores.
+#include "internal.h"
+
+namespace kvc {
+namespace {
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0;  // -0 == +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_kernel(const RowMap map, int w, const float* __restrict__ s_hat, const int32_t* __restrict__ b,
+                  const int64_t* __restrict__ slot_off, int32_t* __restrict__ idx) {
+  extern __shared__ uint32_t keys[];
+  __shared__ int hist[256];
+  __shared__ int wgt[kSelWarps], weq[kSelWarps];
+  __shared__ uint32_t sh_prefix;
+  __shared__ int sh_kk;
+
+  const int row = blockIdx.x;
+  const int L = row_len(map, row);
+  const long long koff = row_key_off(map, row);
+  const int bb = b[row];
+  int32_t* out = idx + slot_off[row];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (bb >= L) {
+    for (int j = threadIdx.x; j < L; j += kSelThreads) out[j] = j;
+    return;
+  }
+  if (bb < w) return;  // not a valid budget (kv_allocate never produces one); nothing is written
+  const int n = L - w;  // candidates [0, n); the window [n, L) is always kept
+  const int k = bb - w;
+  for (int i = threadIdx.x; i < w; i += kSelThreads) out[k + i] = n + i;
+  if (k <= 0) return;
+
+  for (int j = threadIdx.x; j < n; j += kSelThreads) keys[j] = order_key(s_hat[koff + j]);
+  if (threadIdx.x == 0) {
+    sh_prefix = 0;
+    sh_kk = k;
+  }
+  __syncthreads();
+
+  // radix select of the k-th largest key, most significant byte first
+  uint32_t mask = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = sh_prefix;
+    for (int j = threadIdx.x; j < n; j += kSelThreads) {
+      const uint32_t key = keys[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int kk = sh_kk, cum = 0, dg = 0;
+      for (dg = 255; dg > 0; --dg) {
+        if (cum + hist[dg] >= kk) break;
+        cum += hist[dg];
+      }
+      sh_kk = kk - cum;
+      sh_prefix = prefix | ((uint32_t)dg << shift);
+    }
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t T = sh_prefix;
+  const int take_eq = sh_kk;  // keys equal to T to keep, lowest indices first
+
+  // per-warp counts over contiguous chunks, then ballot compaction in index order
+  const int chunk = (((n + kSelWarps - 1) / kSelWarps) + 31) & ~31;
+  const int c0 = warp * chunk, c1 = min(n, c0 + chunk);
+  int ngt = 0, neq = 0;
+  for (int j = c0 + lane; j < c1; j += 32) {
+    const uint32_t key = keys[j];
+    ngt += key > T;
+    neq += key == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+    neq += __shfl_xor_sync(0xffffffffu, neq, o);
+  }
+  if (lane == 0) {
+    wgt[warp] = ngt;
+    weq[warp] = neq;
+  }
+  __syncthreads();
+  int eq_before = 0, sel_before = 0;
+  for (int i = 0; i < warp; ++i) {
+    sel_before += wgt[i] + max(0, min(weq[i], take_eq - eq_before));
+    eq_before += weq[i];
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = c0; base < c1; base += 32) {
+    const int j = base + lane;
+    const uint32_t key = j < c1 ? keys[j] : 0u;
+    const bool eq = j < c1 && key == T;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_before + __popc(beq & lt);
+    const bool sel = j < c1 && (key > T || (eq && eq_rank < take_eq));
+    const unsigned bsel = __ballot_sync(0xffffffffu, sel);
+    const int at = sel_before + __popc(bsel & lt);
+    if (sel && at < k) out[at] = j;
+    eq_before += __popc(beq);
+    sel_before += __popc(bsel);
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    gather_kernel(const RowMap map, int row_bytes, const int64_t* __restrict__ slot_off,
+                  const int32_t* __restrict__ b, const int32_t* __restrict__ idx, const uint8_t* __restrict__ K,
+                  const uint8_t* __restrict__ V, uint8_t* __restrict__ Kc, uint8_t* __restrict__ Vc) {
+  const int n_rows = map.n_rows;
+  const long long total = slot_off[n_rows];
+  const int lane = threadIdx.x & 31;
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int chunks = row_bytes / 16;       // 16-byte pieces per K/V row
+  const int per_iter = max(1, 32 / chunks);  // rows copied per warp instruction
+  for (long long unit = gw; unit * 32 < total; unit += nw) {
+    const long long slot = unit * 32 + lane;
+    long long src = -1;
+    if (slot < total) {
+      int lo = 0, hi = n_rows - 1;  // last row with slot_off[row] <= slot
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (slot_off[mid] <= slot) lo = mid;
+        else hi = mid - 1;
+      }
+      const long long t = slot - slot_off[lo];
+      if (t < b[lo]) {
+        const int j = idx[slot];
+        if (j >= 0 && j < row_len(map, lo)) src = row_key_off(map, lo) + j;  // skips rows select left unwritten
+      }
+    }
+    for (int i0 = 0; i0 < 32; i0 += per_iter) {
+      const int i = i0 + (per_iter > 1 ? lane / chunks : 0);
+      const long long sidx = __shfl_sync(0xffffffffu, src, min(i, 31));
+      const int piece = per_iter > 1 ? lane % chunks : lane;
+      if (i < 32 && sidx >= 0) {
+        const long long dst = unit * 32 + i;
+        for (int c = piece; c < chunks; c += 32) {
+          const uint4 kv = __ldg(reinterpret_cast<const uint4*>(K + sidx * row_bytes) + c);
+          const uint4 vv = __ldg(reinterpret_cast<const uint4*>(V + sidx * row_bytes) + c);
+          reinterpret_cast<uint4*>(Kc + dst * row_bytes)[c] = kv;
+          reinterpret_cast<uint4*>(Vc + dst * row_bytes)[c] = vv;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+int launch_select_gather(const kv_shape& sh, const RowMap& m, const float* s_hat, const void* K, const void* V,
+                         const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
+                         cudaStream_t st) {
+  int maxL = 0;
+  for (int i = 0; i < m.n_seq; ++i) maxL = std::max(maxL, m.L[i]);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    attr = true;
+  }
+  select_kernel<<<m.n_rows, kSelThreads, (size_t)maxL * sizeof(uint32_t), st>>>(m, sh.w, s_hat, b, slot_off, idx);
+  const int esz = sh.dtype == KV_BF16 ? 2 : 4;
+  const int row_bytes = sh.head_dim * esz;
+  gather_kernel<<<sm_count() * 8, 256, 0, st>>>(m, row_bytes, slot_off, b, idx, static_cast<const uint8_t*>(K),
+                                               static_cast<const uint8_t*>(V), static_cast<uint8_t*>(Kc),
+                                               static_cast<uint8_t*>(Vc));
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace kvc

@@ -228,6 +228,13 @@ class DecodeList:
                                     gamma, T, M, b, _p(o))
         return o, int(ev)
 
+    def clone(self) -> "DecodeList":
+        c = DecodeList.__new__(DecodeList)
+        c.d = self.d
+        c.n = C.c_int64(self.n.value)
+        c.K, c.V, c.A, c.pos = self.K.copy(), self.V.copy(), self.A.copy(), self.pos.copy()
+        return c
+
     def entries(self):
         n = self.n.value
         return self.K[:n].copy(), self.V[:n].copy(), self.A[:n].copy(), self.pos[:n].copy()

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the
+header declares, and its host-side checks (sizes, argument errors, fault
+injection) behave as documented. No call here reaches a kernel."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import kv_cache_compression_layer_b200 as kv
+from kv_cache_compression_layer_b200 import build as kvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    kvbuild.build()
+    return kv.lib()
+
+
+def _declared():
+    hdr = open(os.path.join(ROOT, "include", "kvcomp.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(kv_\w+)\s*\(", hdr, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert "kv_score" in names and "kv_decode_attn_update" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(kv.EXPORTS) == names
+
+
+def _shape(dtype=kv.KV_BF16):
+    return kv.make_shape(36, 2, 8, 128, 32, dtype)
+
+
+def _params():
+    return kv.make_params(60, 0.5, 0.7, 0.5, 0.95, 4, 20)
+
+
+def test_rows_and_lengths(L):
+    sh = _shape()
+    assert kv.kv_rows(sh, 1) == 72
+    assert kv.kv_rows(sh, 0) == -1
+    assert kv.kv_check_lengths(sh, [6000]) == kv.KV_OK
+    assert kv.kv_check_lengths(sh, [6001]) == kv.KV_ERR_UNSUPPORTED_L  # odd
+    assert kv.kv_check_lengths(sh, [2 * 11 * 16]) == kv.KV_ERR_UNSUPPORTED_L  # factor 11
+    assert kv.kv_check_lengths(sh, [32768 * 2]) == kv.KV_ERR_UNSUPPORTED_L  # too long
+    assert kv.kv_check_lengths(sh, [30]) == kv.KV_ERR_UNSUPPORTED_L  # shorter than w
+    assert kv.kv_check_lengths(sh, [2000, 3500, 16000]) == kv.KV_OK
+    bad = kv.make_shape(1, 1, 1, 96, 32, kv.KV_BF16)
+    assert kv.kv_check_lengths(bad, [1024]) == kv.KV_ERR_ARG
+
+
+def test_total_slots_matches_budget_formula(L):
+    sh = _shape()
+    p = _params()
+    # per layer: sum_h b_h = floor(60 * 6000 * 2 / 100) = 7200, plus one spare slot per head
+    assert kv.kv_total_slots(sh, [6000], p) == 36 * (7200 + 2)
+    p2 = kv.make_params(25, 0.5, 0.7, 0.5, 0.95, 4, 20)
+    sh2 = kv.make_shape(28, 4, 7, 128, 32, kv.KV_BF16)
+    Ls = [2000, 3500]
+    assert kv.kv_total_slots(sh2, Ls, p2) == sum(28 * ((25 * l * 4) // 100 + 4) for l in Ls)
+    assert kv.kv_total_slots(sh, [6000], kv.make_params(0, .5, .7, .5, .95, 4, 20)) == -1
+
+
+def test_workspace_grows_with_tiles(L):
+    sh = _shape()
+    a = kv.kv_workspace_bytes(sh, [6000])
+    b = kv.kv_workspace_bytes(sh, [12000])
+    assert 0 < a < b
+    tiles = 72 * ((6000 + 127) // 128)
+    assert a >= tiles * 256 * 8  # (max, sum) per tile and window row
+
+
+def test_argument_errors_launch_nothing(L):
+    sh = _shape()
+    Larr = (C.c_int32 * 1)(6000)
+    st = L.kv_score(C.byref(sh), Larr, 1, None, None, None, None, 0, None)
+    assert st == kv.KV_ERR_ARG
+    st = L.kv_score(C.byref(sh), Larr, 1, 16, 16, 16, None, 0, None)
+    assert st == kv.KV_ERR_WORKSPACE
+    st = L.kv_score(C.byref(sh), Larr, 1, 17, 16, 16, 16, 1 << 30, None)  # misaligned
+    assert st == kv.KV_ERR_ARG
+    st = L.kv_sss(C.byref(sh), Larr, 1, 16, 16, 16, C.c_float(0.5), C.c_float(0.7), None)  # s aliases s_hat
+    assert st == kv.KV_ERR_ARG
+    st = L.kv_sss(C.byref(sh), Larr, 1, 16, 32, 48, C.c_float(1.5), C.c_float(0.7), None)  # alpha > 1
+    assert st == kv.KV_ERR_ARG
+    p = kv.make_params(5, 0.5, 0.7, 0.5, 0.95, 4, 20)
+    L2 = (C.c_int32 * 1)(256)  # B = 5% of 256*2 = 25 < 2*32
+    st = L.kv_allocate(C.byref(sh), L2, 1, C.byref(p), 16, 16, 16, None)
+    assert st == kv.KV_ERR_BUDGET
+    cache = kv.kv_cache()
+    st = L.kv_decode_attn_update(C.byref(sh), Larr, 1, C.byref(_params()), C.byref(cache), 16, 16, 16, 16, None)
+    assert st == kv.KV_ERR_ARG
+
+
+def test_fault_injection_env(L, monkeypatch):
+    sh = _shape()
+    Larr = (C.c_int32 * 1)(6000)
+    monkeypatch.setenv("KV_FAULT_INJECT", "kv_select_gather")
+    st = L.kv_select_gather(C.byref(sh), Larr, 1, 16, 16, 16, 16, 16, 16, 16, 16, None)
+    assert st == kv.KV_ERR_CUDA
+    monkeypatch.delenv("KV_FAULT_INJECT")
+    st = L.kv_select_gather(C.byref(sh), Larr, 1, None, 16, 16, 16, 16, 16, 16, 16, None)
+    assert st == kv.KV_ERR_ARG
+
+
+def test_status_strings(L):
+    assert kv.status_string(kv.KV_OK) == "ok"
+    assert "budget" in kv.status_string(kv.KV_ERR_BUDGET)
+    assert kv.status_string(99) == "unknown status"
