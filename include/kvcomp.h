@@ -206,6 +206,29 @@ int kv_decode_attn_update(const kv_shape* shape, const int32_t* L, int32_t n_seq
                           kv_cache* cache, const void* q_t, const void* k_t, const void* v_t, void* out,
                           void* stream);
 
+/*
+ * kv_score_noalloc — kv_score for callers that cannot allocate device memory
+ * (no counterpart in the pages: a deployment variant of the same operation).
+ * Same arguments, layout and result as kv_score, minus the workspace: the
+ * scratch is a file-scope device array of KV_NOALLOC_SCRATCH_BYTES held by
+ * every GPU that loads this library until the process exits.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Batches whose scratch (kv_workspace_bytes) exceeds the limit return
+ *     KV_ERR_WORKSPACE and launch nothing.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     the status word is cleared by each call. Calls that overlap on the GPU
+ *     (different streams, or different threads' streams) race on it: order
+ *     them on one stream or synchronise between them.
+ *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *     Device-side errors are recorded in the array's status word, which this
+ *     variant does not expose.
+ * Errors: as kv_score (KV_ERR_WORKSPACE when the batch is too large).
+ */
+#define KV_NOALLOC_SCRATCH_BYTES (8u << 20)
+int kv_score_noalloc(const kv_shape* shape, const int32_t* L, int32_t n_seq, const void* qwin, const void* K,
+                     float* s, void* stream);
+
 /* Copies the device status word to the host (synchronises `stream`);
  * returns KV_OK or KV_ERR_CUDA. */
 int kv_read_device_status(const int32_t* status_dev, int32_t* status_host, void* stream);

@@ -25,7 +25,8 @@ META_INTS = 8
 # Every symbol include/kvcomp.h declares.
 EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
-           "kv_status_string")
+           "kv_status_string", "kv_score_noalloc")
+KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class kv_shape(C.Structure):
@@ -74,6 +75,7 @@ def lib():
             "kv_decode_attn_update": (C.c_int, [Ps, P, I32, Pp, Pc, P, P, P, P, P]),
             "kv_read_device_status": (C.c_int, [P, P, P]),
             "kv_status_string": (C.c_char_p, [C.c_int]),
+            "kv_score_noalloc": (C.c_int, [Ps, P, I32, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -150,6 +152,14 @@ def kv_score(shape, L, qwin, K, s, ws, ws_bytes: Optional[int] = None, stream=No
                                       _stream(stream)))
 
 
+def kv_score_noalloc(shape, L, qwin, K, s, stream=None):
+    """kv_score without a workspace: the library's own fixed scratch array is used
+    (for callers that cannot allocate device memory; see include/kvcomp.h)."""
+    arr, n = _L(L)
+    _check("kv_score_noalloc", lib().kv_score_noalloc(C.byref(shape), arr, n, _ptr(qwin), _ptr(K), _ptr(s),
+                                                      _stream(stream)))
+
+
 def kv_sss(shape, L, s, s_hat, kstar, alpha: float, rho: float, stream=None):
     arr, n = _L(L)
     _check("kv_sss", lib().kv_sss(C.byref(shape), arr, n, _ptr(s), _ptr(s_hat), _ptr(kstar), alpha, rho,
@@ -195,6 +205,7 @@ def kv_read_device_status(status_dev, stream=None) -> int:
 from .pipeline import Compressor  # noqa: E402  (the torch-side convenience wrapper)
 
 __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", "make_params", "make_cache",
-           "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
+           "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_score_noalloc",
+           "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "status_string", "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]
