@@ -98,6 +98,7 @@ typedef struct {
   int32_t* meta;           /* [rows][8]: count, next free slot, steps done, last evicted slot,
                               prefill count, 3 reserved */
   int32_t* status;         /* device status word (KV_DEV_* bits)          */
+  int64_t total_slots;     /* host: rows of Kc/Vc (slot_off[rows]); 0 = kv_total_slots() */
 } kv_cache;
 
 /* Number of rows of a batch. Returns -1 on a bad shape. */

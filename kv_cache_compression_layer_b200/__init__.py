@@ -41,7 +41,8 @@ class kv_params(C.Structure):
 
 class kv_cache(C.Structure):
     _fields_ = [("Kc", C.c_void_p), ("Vc", C.c_void_p), ("A", C.c_void_p), ("pos", C.c_void_p),
-                ("slot_off", C.c_void_p), ("b", C.c_void_p), ("meta", C.c_void_p), ("status", C.c_void_p)]
+                ("slot_off", C.c_void_p), ("b", C.c_void_p), ("meta", C.c_void_p), ("status", C.c_void_p),
+                ("total_slots", C.c_int64)]
 
 
 class KvError(RuntimeError):
@@ -179,8 +180,11 @@ def kv_select_gather(shape, L, s_hat, K, V, b, slot_off, idx, Kc, Vc, stream=Non
                                                       _stream(stream)))
 
 
-def make_cache(Kc, Vc, A, pos, slot_off, b, meta, status) -> kv_cache:
-    return kv_cache(_ptr(Kc), _ptr(Vc), _ptr(A), _ptr(pos), _ptr(slot_off), _ptr(b), _ptr(meta), _ptr(status))
+def make_cache(Kc, Vc, A, pos, slot_off, b, meta, status, total_slots: Optional[int] = None) -> kv_cache:
+    if total_slots is None:
+        total_slots = Kc.shape[0] if hasattr(Kc, "shape") else 0
+    return kv_cache(_ptr(Kc), _ptr(Vc), _ptr(A), _ptr(pos), _ptr(slot_off), _ptr(b), _ptr(meta), _ptr(status),
+                    int(total_slots))
 
 
 def kv_decode_init(shape, L, params, cache: kv_cache, stream=None):

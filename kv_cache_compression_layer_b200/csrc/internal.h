@@ -13,6 +13,8 @@ namespace kvc {
 int make_row_map(const kv_shape& sh, const int32_t* L, int32_t n_seq, RowMap& m);
 int64_t total_keys(const RowMap& m);
 int sm_count();
+// 2-D bf16 tensor map over [rows][d] with a box of 64 x box_rows, 128-byte swizzle.
+bool encode_rows_bf16(CUtensorMap* map, const void* base, int d, long long rows, int box_rows);
 
 // Workspace layout of kv_score.
 struct ScoreWs {

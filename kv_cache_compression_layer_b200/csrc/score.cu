@@ -18,8 +18,6 @@
 //
 // fp32 path (fp32 inputs): the same three steps on CUDA cores (FFMA), since
 // a tf32 contraction would not meet the fp32 tolerance.
-#include <cudaTypedefs.h>
-
 #include <cmath>
 #include <mutex>
 
@@ -366,33 +364,6 @@ __global__ void score_f32_colsum_kernel(const RowMap map, int R, int d, float c,
     sum += ex2_approx(fmaf(x, c, -Ls[r]));
   }
   s[key0 + j] = sum;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor map over [rows][d] with a box of 64 x box_rows, 128B swizzle.
-bool encode_rows_bf16(CUtensorMap* map, const void* base, int d, long long rows, int box_rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
 }
 
 }  // namespace
