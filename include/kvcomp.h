@@ -99,6 +99,9 @@ typedef struct {
                               prefill count, 3 reserved */
   int32_t* status;         /* device status word (KV_DEV_* bits)          */
   int64_t total_slots;     /* host: rows of Kc/Vc (slot_off[rows]); 0 = kv_total_slots() */
+  void* scratch;           /* device, kv_decode_scratch_bytes() bytes: per-slot logits, per-item
+                              softmax partials, work items, row tickets (L2-resident)         */
+  size_t scratch_bytes;
 } kv_cache;
 
 /* Number of rows of a batch. Returns -1 on a bad shape. */
@@ -113,6 +116,10 @@ size_t kv_workspace_bytes(const kv_shape* shape, const int32_t* L, int32_t n_seq
 /* Total compacted-cache slots sum_i (b_i + 1) for this batch (host query;
  * sum_h b_{l,h} = floor(budget_pct * L * H / 100) per layer), or -1. */
 int64_t kv_total_slots(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params);
+
+/* Bytes of decode scratch (kv_cache.scratch) for this batch and cache size. */
+size_t kv_decode_scratch_bytes(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
+                               int64_t total_slots);
 
 /*
  * kv_score — observation-window importance scores (AudioKV blog §1.2: the raw
@@ -182,7 +189,8 @@ int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, con
  * kv_decode_init — prepares the decode state after kv_select_gather:
  *   A = 0 on every slot (VoxZip defines A by the decode recursion only),
  *   meta_i = {count = b_i, next free slot = b_i, steps = 0, last evicted = -1,
- *   prefill count = b_i}, and checks that every row has an evictable middle
+ *   prefill count = b_i}, builds the decode work items (rows cut into
+ *   256-slot chunks) in the scratch, and checks that every row has an evictable middle
  *   once a token is appended (b_i >= T + M_i) where
  *   M_i = floor(recent_pct * b_i / 100); rows without one set KV_DEV_BUDGET.
  * Errors: KV_ERR_ARG, KV_ERR_CUDA.

@@ -25,7 +25,7 @@ META_INTS = 8
 # Every symbol include/kvcomp.h declares.
 EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
-           "kv_status_string", "kv_score_noalloc")
+           "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -42,7 +42,7 @@ class kv_params(C.Structure):
 class kv_cache(C.Structure):
     _fields_ = [("Kc", C.c_void_p), ("Vc", C.c_void_p), ("A", C.c_void_p), ("pos", C.c_void_p),
                 ("slot_off", C.c_void_p), ("b", C.c_void_p), ("meta", C.c_void_p), ("status", C.c_void_p),
-                ("total_slots", C.c_int64)]
+                ("total_slots", C.c_int64), ("scratch", C.c_void_p), ("scratch_bytes", C.c_size_t)]
 
 
 class KvError(RuntimeError):
@@ -77,6 +77,7 @@ def lib():
             "kv_read_device_status": (C.c_int, [P, P, P]),
             "kv_status_string": (C.c_char_p, [C.c_int]),
             "kv_score_noalloc": (C.c_int, [Ps, P, I32, P, P, P, P]),
+            "kv_decode_scratch_bytes": (SZ, [Ps, P, I32, Pp, I64]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -180,11 +181,19 @@ def kv_select_gather(shape, L, s_hat, K, V, b, slot_off, idx, Kc, Vc, stream=Non
                                                       _stream(stream)))
 
 
-def make_cache(Kc, Vc, A, pos, slot_off, b, meta, status, total_slots: Optional[int] = None) -> kv_cache:
+def make_cache(Kc, Vc, A, pos, slot_off, b, meta, status, scratch=None, total_slots: Optional[int] = None,
+               scratch_bytes: Optional[int] = None) -> kv_cache:
     if total_slots is None:
         total_slots = Kc.shape[0] if hasattr(Kc, "shape") else 0
+    if scratch_bytes is None:
+        scratch_bytes = scratch.numel() * scratch.element_size() if scratch is not None else 0
     return kv_cache(_ptr(Kc), _ptr(Vc), _ptr(A), _ptr(pos), _ptr(slot_off), _ptr(b), _ptr(meta), _ptr(status),
-                    int(total_slots))
+                    int(total_slots), _ptr(scratch), int(scratch_bytes))
+
+
+def kv_decode_scratch_bytes(shape: kv_shape, L: Sequence[int], params: kv_params, total_slots: int) -> int:
+    arr, n = _L(L)
+    return lib().kv_decode_scratch_bytes(C.byref(shape), arr, n, C.byref(params), int(total_slots))
 
 
 def kv_decode_init(shape, L, params, cache: kv_cache, stream=None):
@@ -212,4 +221,4 @@ __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", 
            "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_score_noalloc",
            "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
-           "status_string", "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]
+           "kv_decode_scratch_bytes", "status_string", "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]

@@ -128,6 +128,16 @@ int64_t kv_total_slots(const kv_shape* shape, const int32_t* L, int32_t n_seq, c
   return total;
 }
 
+size_t kv_decode_scratch_bytes(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
+                               int64_t total_slots) {
+  if (!shape_ok(shape) || !params) return 0;
+  RowMap m;
+  if (make_row_map(*shape, L, n_seq, m) != KV_OK) return 0;
+  if (total_slots <= 0) total_slots = kv_total_slots(shape, L, n_seq, params);
+  if (total_slots <= 0) return 0;
+  return decode_scratch_bytes(*shape, m, *params, total_slots);
+}
+
 int kv_score(const kv_shape* shape, const int32_t* L, int32_t n_seq, const void* qwin, const void* K, float* s,
              void* ws, size_t ws_bytes, void* stream) {
   if (fault_injected("kv_score")) return KV_ERR_CUDA;

@@ -338,27 +338,33 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(const DecArg
 
 
 // ------------------------------------------------------------------------
-// bf16 caches: tensor-core decode.
+// bf16 caches: persistent split-K tensor-core decode, then a per-row finish.
 //
-// Per row a cluster of C CTAs; CTA c owns slots [c S, c S + S). Warp 4
-// streams the CTA's slots as 64-slot tiles (K tiles first, then V tiles)
-// through a 4-stage ring with TMA (128-byte swizzled boxes, so the
-// ldmatrix reads below are bank-conflict free). Warps 0-3 each own 16 slots
-// of a tile:
-//   phase 1  S = Q K^T with mma.sync m16n8k16 (A = the g query rows, padded
-//            to 16; B = K rows via ldmatrix), logits (log2 units) kept in
-//            shared memory, running max per query head;
-//   phase 2  CTA max per query head;
-//   phase 3  P = exp2(S - max) rebuilt as mma A fragments from shared
-//            memory, O += P V (B = V rows via ldmatrix.trans), row sums;
-// then the CTAs combine (max, sum, O) through distributed shared memory,
-// each writing a slice of the output, apply the exact probabilities to A and
-// reduce the eviction candidate. The appended token's row is patched into the
-// tile (and written to the cache) by the warp that owns its slot.
-constexpr int kTcSlots = 64;
-constexpr int kTcStages = 4;
-constexpr int kTcConsumers = 4;
-constexpr int kTcThreads = (kTcConsumers + 1) * 32;
+// decode_attn_kernel: every row is cut into work items of kCH slots; one CTA
+// per SM takes a contiguous run of items. Its producer warp streams each
+// item's 64-slot tiles of K and V, with the row's g query rows and a small
+// header (row, slot range, the row's step state), through a 5-stage TMA ring
+// (128-byte swizzled boxes, so the ldmatrix reads are free of bank
+// conflicts). Eight consumer warps in two groups take alternate tiles; in a
+// group each warp owns 16 slots of a tile and runs one pass of online
+// softmax on the tensor cores (mma.sync m16n8k16: A = the g query rows padded
+// to 16, B = K rows via ldmatrix; then A = P, B = V rows via ldmatrix.trans).
+// Every logit goes to an L2-resident scratch; when a group leaves a row it
+// combines its four warps and writes one (max, sum, O) partial stamped with
+// the step number. No CTA waits on another.
+// decode_finish_kernel (one CTA per row): combines the row's stamped
+// partials into the attention output, applies the exact probabilities to A,
+// picks the eviction and updates the row's meta data.
+constexpr int kTcSlots = 64;  // slots per TMA tile
+constexpr int kCH = 128;      // slots per work item
+constexpr int kSkStages = 6;
+constexpr int kGroups = 3;  // consumer groups of four warps; group k takes the tiles with it % 3 == k
+constexpr int kSkConsumers = 4 * kGroups;
+constexpr int kSkThreads = (kSkConsumers + 1) * 32;
+constexpr int kTcMaxG = 8;                     // query heads per KV head on the tensor-core path
+constexpr int kQBytes = kTcMaxG * 128 * 2;     // staged query rows per stage
+constexpr int kFinThreads = 256;
+constexpr int kFinSlots = 512;  // slots per finishing CTA
 
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int slot, int dcol) {
   const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
@@ -386,373 +392,616 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-struct TcDec {
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Decode scratch inside kv_cache.scratch.
+struct DecScratch {
+  int* n_items;   // [1]
+  int* item_off;  // [rows + 1] first item of each row
+  int2* items;    // [max_items] (row, chunk)
+  float* part;    // [max_items * 2][stride]: (max[G], sum[G], O[G][d], step stamp) per (item, group)
+  float* logits;  // [total_slots][G] logits in log2 units
+  int* tickets;   // [rows] finished slices of the current step, reset by the row's last slice
+  int4* bests;    // [rows][max_slices] eviction candidate per slice: (A bits, pos, slot, -)
+  int max_items, max_per_row, stride, max_slices;
+};
+
+size_t dec_scratch_layout(int rows, int G, int d, int capb, long long total_slots, char* base, DecScratch* sc) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const int per_row = (capb + kCH - 1) / kCH;
+  const int max_items = rows * per_row;
+  const int stride = 2 * G + G * d + 4;
+  size_t off = 0;
+  const size_t o_n = off;
+  off += 256;
+  const size_t o_ioff = off;
+  off += al((size_t)(rows + 1) * 4);
+  const size_t o_items = off;
+  off += al((size_t)max_items * 8);
+  const size_t o_part = off;
+  off += al((size_t)max_items * kGroups * stride * 4);
+  const size_t o_log = off;
+  off += al((size_t)total_slots * G * 4);
+  const int max_slices = (capb + kFinSlots - 1) / kFinSlots;
+  const size_t o_tk = off;
+  off += al((size_t)rows * 4);
+  const size_t o_best = off;
+  off += al((size_t)rows * max_slices * 16);
+  if (sc && base) {
+    sc->n_items = reinterpret_cast<int*>(base + o_n);
+    sc->item_off = reinterpret_cast<int*>(base + o_ioff);
+    sc->items = reinterpret_cast<int2*>(base + o_items);
+    sc->part = reinterpret_cast<float*>(base + o_part);
+    sc->logits = reinterpret_cast<float*>(base + o_log);
+    sc->tickets = reinterpret_cast<int*>(base + o_tk);
+    sc->bests = reinterpret_cast<int4*>(base + o_best);
+    sc->max_slices = max_slices;
+    sc->max_items = max_items;
+    sc->max_per_row = per_row;
+    sc->stride = stride;
+  }
+  return off;
+}
+
+struct SkArgs {
   DecArgs a;
-  int S_pad;  // row stride of the logit buffer
-  int nk;     // 64-element boxes per row (d / 64)
+  DecScratch sc;
+  int nk;  // 64-element boxes per row (d / 64)
   unsigned long long limit_ns;
 };
 
-__global__ void __launch_bounds__(kTcThreads) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                const __grid_constant__ CUtensorMap tmV,
-                                                                const TcDec P) {
+// What the producer learns about a tile and hands to the consumers.
+struct TileHdr {
+  int row, u, st0, c1, count, next, steps, cap;  // row = -1: no more tiles for this group
+  long long base;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSkThreads, 1) decode_attn_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                     const __grid_constant__ CUtensorMap tmV,
+                                                                     const SkArgs P) {
+  constexpr int NDC = D / 16;                       // 16-wide chunks of d
+  constexpr int TILE = kTcSlots * D * 2;            // bytes of one K or V tile
+  constexpr int STAGE = 2 * TILE + kQBytes;         // K tile, V tile, query rows
   const DecArgs& a = P.a;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int row = blockIdx.x / a.C;
-  const int G = a.G, d = a.d;
+  const DecScratch& sc = P.sc;
+  const int G = a.G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile_bytes = kTcSlots * d * 2;
+  const int q_bytes = G * D * 2;
 
   extern __shared__ uint8_t dsm_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  float* xs = reinterpret_cast<float*>(smem + kTcStages * tile_bytes);  // [G][S_pad] logits (log2 units)
-  float* o_s = xs + G * P.S_pad;                                        // [G][d]
-  __shared__ uint64_t full[kTcStages], empty[kTcStages];
-  __shared__ float m_s[kMaxG], l_s[kMaxG], lse_s[kMaxG], M_s[kMaxG], Li_s[kMaxG];
-  __shared__ float red_m[kTcConsumers][kMaxG];
-  __shared__ float mr_s[8][kMaxG];
-  __shared__ Best bw[kTcConsumers + 1];
-  __shared__ Best best_s;
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  float* o_s = reinterpret_cast<float*>(ring + kSkStages * STAGE);  // [groups][G][D]
+  __shared__ uint64_t full[kSkStages], empty[kSkStages];
+  __shared__ TileHdr hdr[kSkStages];
+  __shared__ float red_m[kSkConsumers][kTcMaxG], red_l[kSkConsumers][kTcMaxG];
   __shared__ int abort_s;
 
-  const int L = row_len(a.map, row);
-  const long long base = a.slot_off[row];
-  const int cap = (int)(a.slot_off[row + 1] - base);
-  const int bb = a.b[row];
-  int32_t* meta = a.meta + (long long)row * 8;
-  const int count = meta[0], next = meta[1], steps = meta[2], count0 = meta[4];
-  const int n = count + 1;
-  const int pos_new = L + steps;
-  const int M = (a.recent_pct * bb) / 100;
-  const int appended = steps + 1;
-  const bool evict = n > bb;
-  const int S = (cap + a.C - 1) / a.C;
-  const int j0 = rank * S, j1 = min(j0 + S, n);
-  const bool ok = S <= a.S_cap && count < cap && (!evict || bb >= a.T + M);
-  const int cnt = ok ? max(0, j1 - j0) : 0;
-  const int nt = (cnt + kTcSlots - 1) / kTcSlots;
-  if (!ok && rank == 0 && tid == 0) atomicOr(a.status, S > a.S_cap ? KV_DEV_CAPACITY : KV_DEV_BUDGET);
-
-  const __nv_bfloat16* qin = static_cast<const __nv_bfloat16*>(a.q) + (long long)row * G * d;
-  const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(a.k) + (long long)row * d;
-  const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(a.v) + (long long)row * d;
-  __nv_bfloat16* Kc = static_cast<__nv_bfloat16*>(a.Kc) + base * d;
-  __nv_bfloat16* Vc = static_cast<__nv_bfloat16*>(a.Vc) + base * d;
-  float* A = a.A + base;
-  int32_t* pos = a.pos + base;
-
   if (tid == 0) {
-    for (int i = 0; i < kTcStages; ++i) {
+    for (int i = 0; i < kSkStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kTcConsumers);
+      mbar_init(&empty[i], 4);
     }
     abort_s = 0;
     fence_barrier_init();
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
   }
-  for (int i = tid; i < G * d; i += kTcThreads) o_s[i] = 0.f;
-  if (tid < kMaxG) l_s[tid] = 0.f;
+  for (int i = tid; i < kGroups * G * D; i += kSkThreads) o_s[i] = 0.f;
+  pdl_wait();  // the previous step's finish has written meta and read the scratch
+  pdl_launch_dependents();
   __syncthreads();
   const Guard gd{&abort_s, a.status, P.limit_ns};
-  const int owner_tile = (next >= j0 && next < j0 + cnt) ? (next - j0) / kTcSlots : -1;
+  const int n_items = *sc.n_items;
+  const int u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
+  const int u1 = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
 
-  if (warp == kTcConsumers) {
-    // ------------------------------------------------------------ producer
+  if (warp == kSkConsumers) {
+    // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      bool issued[kTcStages] = {false, false, false, false};
-      uint32_t par[kTcStages] = {0, 0, 0, 0};
+      const uint64_t stream_policy = make_policy_evict_first();  // K/V are read once per step
+      bool issued[kSkStages] = {};
+      uint32_t par[kSkStages] = {};
       bool aborted = false;
-      for (int it = 0; it < 2 * nt; ++it) {
-        const int st = it % kTcStages;
-        if (it >= kTcStages && !wait_bounded(&empty[st], ((it / kTcStages) - 1) & 1, gd)) {
+      int it = 0;
+      int2 item = u0 < u1 ? sc.items[u0] : make_int2(0, 0);
+      int cur = -1, cap = 0, count = 0, next = 0, steps = 0;
+      long long base = 0;
+      for (int u = u0; u < u1 && !aborted; ++u) {
+        const int row = item.x, chunk = item.y;
+        if (u + 1 < u1) item = sc.items[u + 1];  // in flight while this item is issued
+        if (row != cur) {  // a row's state is fixed for the whole step: load it once
+          cur = row;
+          base = a.slot_off[row];
+          cap = (int)(a.slot_off[row + 1] - base);
+          const int* mrow = a.meta + (long long)row * 8;
+          count = mrow[0];
+          next = mrow[1];
+          steps = mrow[2];
+        }
+        const int c0 = chunk * kCH, c1 = min(c0 + kCH, cap);
+        const int nt = (c1 - c0 + kTcSlots - 1) / kTcSlots;
+        const void* qsrc = static_cast<const __nv_bfloat16*>(a.q) + (long long)row * G * D;
+        for (int t = 0; t < nt; ++t, ++it) {
+          const int st = it % kSkStages;
+          if (it >= kSkStages && !wait_bounded(&empty[st], ((it / kSkStages) - 1) & 1, gd)) {
+            aborted = true;
+            break;
+          }
+          TileHdr h;
+          h.row = row;
+          h.u = u;
+          h.st0 = c0 + t * kTcSlots;
+          h.c1 = c1;
+          h.count = count;
+          h.next = next;
+          h.steps = steps;
+          h.cap = cap;
+          h.base = base;
+          hdr[st] = h;
+          uint8_t* stage = ring + st * STAGE;
+          mbar_arrive_expect_tx(&full[st], 2 * TILE + q_bytes);
+          const int y = (int)(base + h.st0);
+#pragma unroll
+          for (int bx = 0; bx < D / 64; ++bx) {
+            tma_load_2d_hint(stage + bx * kTcSlots * 128, &tmK, &full[st], bx * 64, y, stream_policy);
+            tma_load_2d_hint(stage + TILE + bx * kTcSlots * 128, &tmV, &full[st], bx * 64, y, stream_policy);
+          }
+          bulk_load(stage + 2 * TILE, qsrc, q_bytes, &full[st]);
+          issued[st] = true;
+          par[st] = (it / kSkStages) & 1;
+        }
+      }
+      // one sentinel stage per consumer group: a header with row = -1, no data
+      for (int k = 0; k < kGroups && !aborted; ++k, ++it) {
+        const int st = it % kSkStages;
+        if (it >= kSkStages && !wait_bounded(&empty[st], ((it / kSkStages) - 1) & 1, gd)) {
           aborted = true;
           break;
         }
-        mbar_arrive_expect_tx(&full[st], tile_bytes);
-        const int t = it < nt ? it : it - nt;
-        const int y = (int)(base + j0 + t * kTcSlots);
-        for (int bx = 0; bx < P.nk; ++bx)
-          tma_load_2d(ring + st * tile_bytes + bx * kTcSlots * 128, it < nt ? &tmK : &tmV, &full[st], bx * 64, y);
-        issued[st] = true;
-        par[st] = (it / kTcStages) & 1;
+        hdr[st].row = -1;
+        mbar_arrive(&full[st]);
       }
       if (aborted || abort_s)
-        for (int st = 0; st < kTcStages; ++st)
+        for (int st = 0; st < kSkStages; ++st)
           if (issued[st]) wait_drain(&full[st], par[st], P.limit_ns);
     }
-  } else {
-    // ------------------------------------------------------------ consumers
-    const int g0 = lane >> 2, q4 = lane & 3;
-    const int ndc = d / 16;
-    uint32_t qa[8][4];
-#pragma unroll
-    for (int dc = 0; dc < 8; ++dc) {
-      if (dc < ndc) {
-        const int c = dc * 16 + q4 * 2;
-        qa[dc][0] = g0 < G ? *reinterpret_cast<const uint32_t*>(qin + g0 * d + c) : 0u;
-        qa[dc][1] = g0 + 8 < G ? *reinterpret_cast<const uint32_t*>(qin + (g0 + 8) * d + c) : 0u;
-        qa[dc][2] = g0 < G ? *reinterpret_cast<const uint32_t*>(qin + g0 * d + c + 8) : 0u;
-        qa[dc][3] = g0 + 8 < G ? *reinterpret_cast<const uint32_t*>(qin + (g0 + 8) * d + c + 8) : 0u;
-      }
-    }
-    const int m_ = lane >> 3, r_ = lane & 7;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-    bool aborted = false;
-    // phase 1: logits
-    for (int t = 0; t < nt; ++t) {
-      const int st = t % kTcStages;
-      if (!wait_bounded(&full[st], (t / kTcStages) & 1, gd)) {
-        aborted = true;
-        break;
-      }
-      const uint32_t tile = smem_u32(ring + st * tile_bytes);
-      if (t == owner_tile && (next - j0 - t * kTcSlots) / 16 == warp) {
-        const int r = next - j0 - t * kTcSlots;
-        if (lane < d / 8) {
-          const uint4 kv = *reinterpret_cast<const uint4*>(kin + lane * 8);
-          *reinterpret_cast<uint4*>(ring + (swz(tile, r, lane * 8) - smem_u32(ring))) = kv;
-          reinterpret_cast<uint4*>(Kc + (long long)next * d)[lane] = kv;
-          reinterpret_cast<uint4*>(Vc + (long long)next * d)[lane] = *reinterpret_cast<const uint4*>(vin + lane * 8);
-        }
-        if (lane == 0) pos[next] = pos_new;
-        fence_proxy_async();
-        __syncwarp();
-      }
-      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int dc = 0; dc < 8; ++dc) {
-        if (dc < ndc) {
-          uint32_t b00, b01, b10, b11;
-          ldsm_x4(swz(tile, warp * 16 + (m_ >> 1) * 8 + r_, dc * 16 + (m_ & 1) * 8), b00, b01, b10, b11);
-          mma16816(d0, qa[dc], b00, b01);
-          mma16816(d1, qa[dc], b10, b11);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int jla = t * kTcSlots + warp * 16 + q4 * 2 + e;  // n-tile 0
-        const int jlb = jla + 8;                                 // n-tile 1
-        const float xa0 = jla < cnt ? d0[e] * a.scale2 : -INFINITY;
-        const float xb0 = jlb < cnt ? d1[e] * a.scale2 : -INFINITY;
-        const float xa1 = jla < cnt ? d0[2 + e] * a.scale2 : -INFINITY;
-        const float xb1 = jlb < cnt ? d1[2 + e] * a.scale2 : -INFINITY;
-        if (g0 < G) {
-          xs[g0 * P.S_pad + jla] = xa0;
-          xs[g0 * P.S_pad + jlb] = xb0;
-          mx0 = fmaxf(mx0, fmaxf(xa0, xb0));
-        }
-        if (g0 + 8 < G) {
-          xs[(g0 + 8) * P.S_pad + jla] = xa1;
-          xs[(g0 + 8) * P.S_pad + jlb] = xb1;
-          mx1 = fmaxf(mx1, fmaxf(xa1, xb1));
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-    }
-    // phase 2: CTA max per query head
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    if (q4 == 0) {
-      if (g0 < G) red_m[warp][g0] = mx0;
-      if (g0 + 8 < G) red_m[warp][g0 + 8] = mx1;
-    }
-    named_bar_sync(1, kTcConsumers * 32);
-    if (tid < G) {
-      float v = -INFINITY;
-      for (int w = 0; w < kTcConsumers; ++w) v = fmaxf(v, red_m[w][tid]);
-      m_s[tid] = v;
-    }
-    named_bar_sync(1, kTcConsumers * 32);
-    const float m0 = g0 < G ? m_s[g0] : 0.f;
-    const float m1 = g0 + 8 < G ? m_s[g0 + 8] : 0.f;
-    // phase 3: P V
-    float o[16][4];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float l0 = 0.f, l1 = 0.f;
-    for (int t = 0; t < nt && !aborted; ++t) {
-      const int it = nt + t;
-      const int st = it % kTcStages;
-      if (!wait_bounded(&full[st], (it / kTcStages) & 1, gd)) {
-        aborted = true;
-        break;
-      }
-      const uint32_t tile = smem_u32(ring + st * tile_bytes);
-      if (t == owner_tile && (next - j0 - t * kTcSlots) / 16 == warp) {
-        const int r = next - j0 - t * kTcSlots;
-        if (lane < d / 8)
-          *reinterpret_cast<uint4*>(ring + (swz(tile, r, lane * 8) - smem_u32(ring))) =
-              *reinterpret_cast<const uint4*>(vin + lane * 8);
-        fence_proxy_async();
-        __syncwarp();
-      }
-      const int jl = t * kTcSlots + warp * 16 + q4 * 2;
-      uint32_t pa[4];
-      {
-        float p00 = 0.f, p01 = 0.f, p08 = 0.f, p09 = 0.f, p10 = 0.f, p11 = 0.f, p18 = 0.f, p19 = 0.f;
-        if (g0 < G) {
-          const float* xr = xs + g0 * P.S_pad + jl;
-          p00 = ex2_approx(xr[0] - m0);
-          p01 = ex2_approx(xr[1] - m0);
-          p08 = ex2_approx(xr[8] - m0);
-          p09 = ex2_approx(xr[9] - m0);
-          l0 += (p00 + p01) + (p08 + p09);
-        }
-        if (g0 + 8 < G) {
-          const float* xr = xs + (g0 + 8) * P.S_pad + jl;
-          p10 = ex2_approx(xr[0] - m1);
-          p11 = ex2_approx(xr[1] - m1);
-          p18 = ex2_approx(xr[8] - m1);
-          p19 = ex2_approx(xr[9] - m1);
-          l1 += (p10 + p11) + (p18 + p19);
-        }
-        pa[0] = pack_bf16(p00, p01);
-        pa[1] = pack_bf16(p10, p11);
-        pa[2] = pack_bf16(p08, p09);
-        pa[3] = pack_bf16(p18, p19);
-      }
-#pragma unroll
-      for (int dn = 0; dn < 8; ++dn) {
-        if (dn < ndc) {
-          uint32_t b0a, b1a, b0b, b1b;
-          ldsm_x4_t(swz(tile, warp * 16 + (m_ & 1) * 8 + r_, dn * 16 + (m_ >> 1) * 8), b0a, b1a, b0b, b1b);
-          mma16816(o[2 * dn], pa, b0a, b1a);
-          mma16816(o[2 * dn + 1], pa, b0b, b1b);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-    }
-    // CTA partials: O and row sums (shared-memory atomics across the 4 warps)
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i < 2 * ndc) {
-        const int col = i * 8 + q4 * 2;
-        if (g0 < G) {
-          atomicAdd(&o_s[g0 * d + col], o[i][0]);
-          atomicAdd(&o_s[g0 * d + col + 1], o[i][1]);
-        }
-        if (g0 + 8 < G) {
-          atomicAdd(&o_s[(g0 + 8) * d + col], o[i][2]);
-          atomicAdd(&o_s[(g0 + 8) * d + col + 1], o[i][3]);
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 1; off <= 2; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-    if (q4 == 0) {
-      if (g0 < G) atomicAdd(&l_s[g0], l0);
-      if (g0 + 8 < G) atomicAdd(&l_s[g0 + 8], l1);
-    }
-    if (aborted) abort_s = 1;
+    return;
   }
-  if (tid < G && cnt == 0) m_s[tid] = -INFINITY;
-  __syncwarp();
-  cluster.sync();
 
-  // ---- combine over the cluster; each CTA writes a slice of the output
-  if (tid < G * a.C) {
-    const int r = tid / G, g = tid % G;
-    mr_s[r][g] = *cluster.map_shared_rank(&m_s[g], r);
+  // ------------------------------------------------------------------ consumers
+  const int g0 = lane >> 2, q4 = lane & 3;  // this lane's query row and column pair
+  const bool g_ok = g0 < G;
+  const int m_ = lane >> 3, r_ = lane & 7;
+  const int grp = warp >> 2;          // tiles with it % kGroups == grp
+  const int wslot = (warp & 3) * 16;  // this warp's 16 slots of a tile
+  const uint64_t keep_policy = make_policy_evict_last();  // logits are read back by the finish kernel
+  float* og = o_s + grp * G * D;
+  bool aborted = false;
+  int cur_row = -1, seg_u = -1, seg_steps = 0;
+  uint32_t qa[NDC][2];  // A fragments of the query rows (rows 8..15 of the m16 tile are zero)
+  float m0 = -INFINITY, l0 = 0.f;
+  float o[2 * NDC][2];  // O[g0][8 i + 2 q4 + {0,1}]
+#pragma unroll
+  for (int i = 0; i < 2 * NDC; ++i) o[i][0] = o[i][1] = 0.f;
+
+  // walk the stages in issue order; this group takes the tiles with it % kGroups == grp
+  for (int it = grp;; it += kGroups) {
+    const int st = it % kSkStages;
+    const bool got = !aborted && wait_bounded(&full[st], (it / kSkStages) & 1, gd);
+    if (!got) aborted = true;
+    const int hrow = got ? hdr[st].row : -1;  // -1: sentinel (or abort), the CTA's tiles are done
+    if (hrow != cur_row || hrow < 0) {
+      if (cur_row >= 0) {
+        // leaving a row: this group's running (max, sum, O) becomes one partial at
+        // (first item of the segment, group), stamped with the step number
+        float ls0 = l0;
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) ls0 += __shfl_xor_sync(0xffffffffu, ls0, off);
+        if (q4 == 0 && g_ok) {
+          red_m[warp][g0] = m0;
+          red_l[warp][g0] = ls0;
+        }
+        named_bar_sync(1 + grp, 128);
+        float M0 = -INFINITY;
+        if (g_ok)
+          for (int w = 0; w < 4; ++w) M0 = fmaxf(M0, red_m[grp * 4 + w][g0]);
+        const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
+        if (g_ok) {
+#pragma unroll
+          for (int i = 0; i < 2 * NDC; ++i) {
+            const int col = i * 8 + q4 * 2;
+            atomicAdd(&og[g0 * D + col], o[i][0] * f0);
+            atomicAdd(&og[g0 * D + col + 1], o[i][1] * f0);
+          }
+        }
+        named_bar_sync(1 + grp, 128);
+        float* part = sc.part + ((long long)seg_u * kGroups + grp) * sc.stride;
+        const int gt = tid - grp * 128;  // thread index within the group
+        if (gt < G) {
+          float M = -INFINITY;
+          for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[grp * 4 + w][gt]);
+          float Ls = 0.f;
+          for (int w = 0; w < 4; ++w)
+            if (red_m[grp * 4 + w][gt] > -INFINITY)
+              Ls += red_l[grp * 4 + w][gt] * ex2_approx(red_m[grp * 4 + w][gt] - M);
+          part[gt] = M;
+          part[G + gt] = Ls;
+        }
+        for (int i = gt; i < G * D; i += 128) {
+          part[2 * G + i] = og[i];
+          og[i] = 0.f;
+        }
+        if (gt == 0) part[2 * G + G * D] = __int_as_float(seg_steps);
+        named_bar_sync(1 + grp, 128);
+        m0 = -INFINITY;
+        l0 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 2 * NDC; ++i) o[i][0] = o[i][1] = 0.f;
+      }
+      if (hrow < 0) break;
+      cur_row = hrow;
+      seg_u = hdr[st].u;
+      seg_steps = hdr[st].steps;
+      // query fragments from the staged [G][D] rows (rows >= G are zero)
+      const uint32_t qs = smem_u32(ring + st * STAGE) + 2 * TILE;
+      const int qrow = lane & 7;
+#pragma unroll
+      for (int dc = 0; dc < NDC; ++dc) {
+        uint32_t r0, r1, r2, r3;
+        const uint32_t addr = qs + (uint32_t)((qrow < G ? qrow : 0) * D + dc * 16 + (lane >> 4) * 8) * 2;
+        ldsm_x4(addr, r0, r1, r2, r3);
+        qa[dc][0] = g_ok ? r0 : 0u;
+        qa[dc][1] = g_ok ? r2 : 0u;
+      }
+    }
+    const TileHdr h = hdr[st];
+    uint8_t* stage = ring + st * STAGE;
+    const uint32_t ktile = smem_u32(stage), vtile = ktile + TILE;
+    const int n = h.count + 1;
+    const bool row_ok = h.count >= 0 && h.count < h.cap && h.next >= 0 && h.next < h.cap;
+    const int next = h.next;
+    const long long base = h.base;
+    if (row_ok && next >= h.st0 + wslot && next < h.st0 + wslot + 16 && next < h.c1) {
+      // the appended token: patch its K and V rows into the tile, write them to the cache
+      const int r = next - h.st0;
+      const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(a.k) + (long long)h.row * D;
+      const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(a.v) + (long long)h.row * D;
+      if (lane < D / 8) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(kin + lane * 8);
+        const uint4 vv = *reinterpret_cast<const uint4*>(vin + lane * 8);
+        *reinterpret_cast<uint4*>(stage + (swz(ktile, r, lane * 8) - ktile)) = kv;
+        *reinterpret_cast<uint4*>(stage + (swz(vtile, r, lane * 8) - ktile)) = vv;
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.Kc) + (base + next) * D)[lane] = kv;
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.Vc) + (base + next) * D)[lane] = vv;
+      }
+      if (lane == 0) a.pos[base + next] = row_len(a.map, h.row) + h.steps;
+      fence_proxy_async();
+      __syncwarp();
+    }
+    // logits S = Q K^T for this warp's 16 slots (even and odd d-chunks accumulate
+    // separately: four independent MMA chains)
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int dc = 0; dc < NDC; ++dc) {
+      uint32_t b00, b01, b10, b11;
+      ldsm_x4(swz(ktile, wslot + (m_ >> 1) * 8 + r_, dc * 16 + (m_ & 1) * 8), b00, b01, b10, b11);
+      const uint32_t af[4] = {qa[dc][0], 0u, qa[dc][1], 0u};
+      if (dc & 1) {
+        mma16816(t0, af, b00, b01);
+        mma16816(t1, af, b10, b11);
+      } else {
+        mma16816(s0, af, b00, b01);
+        mma16816(s1, af, b10, b11);
+      }
+    }
+    const int jb = h.st0 + wslot + q4 * 2;  // slots jb, jb+1 (n-tile 0) and jb+8, jb+9 (n-tile 1)
+    float x[4];                              // row g0 at those four slots
+    x[0] = s0[0] + t0[0];
+    x[1] = s0[1] + t0[1];
+    x[2] = s1[0] + t1[0];
+    x[3] = s1[1] + t1[1];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = jb + (e & 1) + (e >> 1) * 8;
+      const bool valid = row_ok && j < n && j < h.c1;
+      x[e] = valid ? x[e] * a.scale2 : -INFINITY;
+      if (valid && g_ok) st_f32_hint(sc.logits + (base + j) * G + g0, x[e], keep_policy);
+    }
+    // online softmax update of this warp's running (max, sum, O)
+    float tm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 2));
+    const float nm = fmaxf(m0, tm);
+    const float vm = nm == -INFINITY ? 0.f : nm;
+    if (__any_sync(0xffffffffu, nm != m0)) {  // rescale only when a running max moved
+      const float sc0 = ex2_approx(m0 - vm);
+      l0 *= sc0;
+#pragma unroll
+      for (int i = 0; i < 2 * NDC; ++i) {
+        o[i][0] *= sc0;
+        o[i][1] *= sc0;
+      }
+    }
+    m0 = nm;
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[e] = ex2_approx(x[e] - vm);
+      l0 += p[e];
+    }
+    const uint32_t pa[4] = {pack_bf16(p[0], p[1]), 0u, pack_bf16(p[2], p[3]), 0u};
+#pragma unroll
+    for (int dn = 0; dn < NDC; ++dn) {
+      uint32_t b0a, b1a, b0b, b1b;
+      ldsm_x4_t(swz(vtile, wslot + (m_ & 1) * 8 + r_, dn * 16 + (m_ >> 1) * 8), b0a, b1a, b0b, b1b);
+      float c0[4] = {o[2 * dn][0], o[2 * dn][1], 0.f, 0.f};
+      float c1[4] = {o[2 * dn + 1][0], o[2 * dn + 1][1], 0.f, 0.f};
+      mma16816(c0, pa, b0a, b1a);
+      mma16816(c1, pa, b0b, b1b);
+      o[2 * dn][0] = c0[0];
+      o[2 * dn][1] = c0[1];
+      o[2 * dn + 1][0] = c1[0];
+      o[2 * dn + 1][1] = c1[1];
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+  if (aborted) abort_s = 1;
+}
+
+// Finish of one decode step, one CTA per (row, slice of kFinSlots slots):
+// the row's log-denominators from the partials stamped with this step, this
+// slice's share of the attention output, the exact probabilities applied to
+// A on this slice's slots, and this slice's best eviction candidate. The
+// row's last slice to finish (atomic ticket, no waiting) picks the eviction
+// and updates the row's meta data.
+__global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs P) {
+  const DecArgs& a = P.a;
+  const DecScratch& sc = P.sc;
+  const int G = a.G, d = a.d, E = G * d;
+  const int row = blockIdx.x / sc.max_slices, slice = blockIdx.x % sc.max_slices;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  extern __shared__ int real[];  // partials of this step, in index order
+  __shared__ float Ms[kMaxG], Li[kMaxG], lse_s[kMaxG];
+  __shared__ Best bw[kFinThreads / 32];
+  __shared__ int n_real, last_s;
+
+  pdl_wait();  // the attention kernel's partials and logits are complete
+  pdl_launch_dependents();
+  // round 1: the row's state
+  int32_t* meta = a.meta + (long long)row * 8;
+  const int count = meta[0], next = meta[1], steps = meta[2], count0 = meta[4];
+  const long long base = a.slot_off[row];
+  const int cap = (int)(a.slot_off[row + 1] - base);
+  const int bb = a.b[row];
+  const int i0 = sc.item_off[row], nch = sc.item_off[row + 1] - i0;
+  const int n = count + 1;
+  const int nsl = (n + kFinSlots - 1) / kFinSlots;
+  if (slice >= nsl) return;  // uniform over the CTA
+  const int pos_new = row_len(a.map, row) + steps;
+  const int np = nch * kGroups;
+  const float* part0 = sc.part + (long long)i0 * kGroups * sc.stride;
+  const int Mr = (a.recent_pct * bb) / 100;
+  const int appended = steps + 1;
+  const bool evict = n > bb;
+  const bool ok = count < cap && next >= 0 && next < cap && (!evict || bb >= a.T + Mr);
+
+  // round 2: which partials belong to this step, and this thread's slots (A, pos, logits)
+  if (warp == 0) {
+    int k = 0;
+    for (int c0 = 0; c0 < np; c0 += 32) {
+      const int c = c0 + lane;
+      const bool used = c < np && __float_as_int(part0[(long long)c * sc.stride + 2 * G + E]) == steps;
+      const unsigned bal = __ballot_sync(0xffffffffu, used);
+      if (used) real[k + __popc(bal & ((1u << lane) - 1u))] = c;
+      k += __popc(bal);
+    }
+    if (lane == 0) n_real = k;
+  }
+  constexpr int U = kFinSlots / kFinThreads;
+  const int jbase = slice * kFinSlots;
+  float Av[U], lgv[U][kMaxG];
+  int pv[U];
+#pragma unroll
+  for (int k = 0; k < U; ++k) {
+    const int j = jbase + k * kFinThreads + tid;
+    Av[k] = 0.f;
+    pv[k] = 0;
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) lgv[k][g] = -INFINITY;
+    if (ok && j < n) {
+      Av[k] = a.A[base + j];
+      pv[k] = a.pos[base + j];
+      const float* lg = sc.logits + (base + j) * G;
+      if ((G & 3) == 0) {
+#pragma unroll
+        for (int g4 = 0; g4 < kMaxG; g4 += 4)
+          if (g4 < G) {
+            const float4 v = *reinterpret_cast<const float4*>(lg + g4);
+            lgv[k][g4] = v.x;
+            lgv[k][g4 + 1] = v.y;
+            lgv[k][g4 + 2] = v.z;
+            lgv[k][g4 + 3] = v.w;
+          }
+      } else {
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) lgv[k][g] = lg[g];
+      }
+    }
+  }
+  const int pos_thr = (!ok || appended >= Mr) ? pos_new - Mr + 1 : a.pos[base + max(0, count0 - (Mr - appended))];
+  __syncthreads();
+  const int nr = n_real;
+  // round 3: the row's max and denominator per query head (a warp per head)
+  for (int g = warp; g < G; g += kFinThreads / 32) {
+    float M = -INFINITY;
+    float mk = -INFINITY, lk = 0.f;
+    if (lane < nr) {  // a row rarely has more than 32 partials; the loop below covers the rest
+      mk = part0[(long long)real[lane] * sc.stride + g];
+      lk = part0[(long long)real[lane] * sc.stride + G + g];
+    }
+    M = mk;
+    for (int k = lane + 32; k < nr; k += 32) M = fmaxf(M, part0[(long long)real[k] * sc.stride + g]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float Ls = mk > -INFINITY ? lk * exp2f(mk - M) : 0.f;
+    for (int k = lane + 32; k < nr; k += 32) {
+      const float mc = part0[(long long)real[k] * sc.stride + g];
+      if (mc > -INFINITY) Ls += part0[(long long)real[k] * sc.stride + G + g] * exp2f(mc - M);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+    if (lane == 0) {
+      Ms[g] = M;
+      Li[g] = Ls > 0.f ? 1.f / Ls : 0.f;
+      lse_s[g] = M + log2f(Ls);
+    }
   }
   __syncthreads();
-  if (tid < G) {
-    float Mx = -INFINITY;
-    for (int r = 0; r < a.C; ++r) Mx = fmaxf(Mx, mr_s[r][tid]);
-    float Lsum = 0.f;
-    for (int r = 0; r < a.C; ++r)
-      if (mr_s[r][tid] > -INFINITY) Lsum += *cluster.map_shared_rank(&l_s[tid], r) * exp2f(mr_s[r][tid] - Mx);
-    M_s[tid] = Mx;
-    Li_s[tid] = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    lse_s[tid] = Mx + log2f(Lsum);
-  }
-  __syncthreads();
+  // round 4: this slice's share of the output
   {
-    const int E = G * d;
-    const int e0 = (int)((long long)E * rank / a.C), e1 = (int)((long long)E * (rank + 1) / a.C);
+    const int e0 = (int)((long long)E * slice / nsl), e1 = (int)((long long)E * (slice + 1) / nsl);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + (long long)row * E;
-    for (int i = e0 + tid; i < e1; i += kTcThreads) {
+    for (int i = e0 + tid; i < e1; i += kFinThreads) {
       const int g = i / d;
       float acc = 0.f;
-      for (int r = 0; r < a.C; ++r) {
-        const float mr = mr_s[r][g];
-        if (mr > -INFINITY) acc += *cluster.map_shared_rank(&o_s[i], r) * exp2f(mr - M_s[g]);
+#pragma unroll 4
+      for (int k = 0; k < nr; ++k) {
+        const float* pc = part0 + (long long)real[k] * sc.stride;
+        const float mc = pc[g];
+        const float w = mc > -INFINITY ? exp2f(mc - Ms[g]) : 0.f;
+        acc += w * pc[2 * G + i];
       }
-      out[i] = __float2bfloat16_rn(acc * Li_s[g]);
+      out[i] = __float2bfloat16_rn(acc * Li[g]);
     }
   }
-
-  // ---- exact probabilities into A, local eviction candidate
+  // the exact probabilities into A (data already in registers), this slice's candidate
+  const bool timed_out = (*reinterpret_cast<volatile int32_t*>(a.status) & KV_DEV_TIMEOUT) != 0;
   Best best{INFINITY, -1, -1};
-  if (ok && !abort_s) {
-    int pos_thr;
-    if (appended >= M) pos_thr = pos_new - M + 1;
-    else pos_thr = pos[max(0, count0 - (M - appended))];
-    for (int jl = tid; jl < cnt; jl += kTcThreads) {
-      const int j = j0 + jl;
-      float psum = 0.f;
-      for (int g = 0; g < G; ++g) psum += ex2_approx(xs[g * P.S_pad + jl] - lse_s[g]);
-      const float Anew = (j == next ? 0.f : a.gamma * A[j]) + psum;
-      A[j] = Anew;
-      const int pj = j == next ? pos_new : pos[j];
-      if (j >= a.T && pj < pos_thr) {
-        const Best c{Anew, pj, j};
-        if (better(c, best)) best = c;
+  if (ok && !timed_out) {
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int j = jbase + k * kFinThreads + tid;
+      if (j < n) {
+        float psum = 0.f;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) psum += ex2_approx(lgv[k][g] - lse_s[g]);
+        const float Anew = (j == next ? 0.f : a.gamma * Av[k]) + psum;
+        a.A[base + j] = Anew;
+        const int pj = j == next ? pos_new : pv[k];
+        if (j >= a.T && pj < pos_thr) {
+          const Best c{Anew, pj, j};
+          if (better(c, best)) best = c;
+        }
       }
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int off = 16; off > 0; off >>= 1) {
     Best y;
-    y.A = __shfl_xor_sync(0xffffffffu, best.A, o);
-    y.pos = __shfl_xor_sync(0xffffffffu, best.pos, o);
-    y.slot = __shfl_xor_sync(0xffffffffu, best.slot, o);
+    y.A = __shfl_xor_sync(0xffffffffu, best.A, off);
+    y.pos = __shfl_xor_sync(0xffffffffu, best.pos, off);
+    y.slot = __shfl_xor_sync(0xffffffffu, best.slot, off);
     if (better(y, best)) best = y;
   }
   if (lane == 0) bw[warp] = best;
   __syncthreads();
   if (tid == 0) {
     Best bst = bw[0];
-    for (int w = 1; w < kTcConsumers + 1; ++w)
+    for (int w = 1; w < kFinThreads / 32; ++w)
       if (better(bw[w], bst)) bst = bw[w];
-    best_s = bst;
+    sc.bests[(long long)row * sc.max_slices + slice] = make_int4(__float_as_int(bst.A), bst.pos, bst.slot, 0);
+    __threadfence();
+    last_s = atomicAdd(&sc.tickets[row], 1) == nsl - 1;
   }
-  __syncwarp();
-  cluster.sync();
+  __syncthreads();
+  if (!last_s || tid != 0) return;
+  // the row's last slice: reduce the candidates, evict, update meta
+  __threadfence();
+  Best bst{INFINITY, -1, -1};
+  for (int k = 0; k < nsl; ++k) {
+    const volatile int* v = reinterpret_cast<volatile int*>(sc.bests + (long long)row * sc.max_slices + k);
+    const Best c{__int_as_float(v[0]), v[1], v[2]};
+    if (better(c, bst)) bst = c;
+  }
+  if (!ok) {
+    atomicOr(a.status, KV_DEV_BUDGET);
+  } else if (!timed_out) {
+    if (evict && bst.slot >= 0) {
+      meta[0] = bb;
+      meta[1] = bst.slot;
+      meta[3] = bst.slot;
+    } else {
+      meta[0] = n;
+      meta[1] = n;
+      meta[3] = -1;
+    }
+    meta[2] = steps + 1;
+  }
+  sc.tickets[row] = 0;
+}
 
-  if (rank == 0 && tid == 0 && ok) {
-    Best bst = best_s;
-    bool any_abort = abort_s != 0;
-    for (int r = 1; r < a.C; ++r) {
-      const Best y = *cluster.map_shared_rank(&best_s, r);
-      if (better(y, bst)) bst = y;
-      any_abort |= *cluster.map_shared_rank(&abort_s, r) != 0;
-    }
-    if (!any_abort) {
-      if (evict && bst.slot >= 0) {
-        meta[0] = bb;
-        meta[1] = bst.slot;
-        meta[3] = bst.slot;
-      } else {
-        meta[0] = n;
-        meta[1] = n;
-        meta[3] = -1;
+// Marks every partial slot as written by no step (stamp -1).
+__global__ void decode_clear_stamps_kernel(DecScratch sc, int G, int d, int n_rows) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_rows; i += gridDim.x * blockDim.x) sc.tickets[i] = 0;
+  const long long n = (long long)sc.max_items * kGroups;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    sc.part[i * sc.stride + 2 * G + G * d] = __int_as_float(-1);
+}
+
+// Builds the work items of every row (rows cut into kCH-slot chunks) and
+// clears the row tickets; one block.
+__global__ void decode_items_kernel(int n_rows, const int64_t* __restrict__ slot_off, DecScratch sc,
+                                    int32_t* __restrict__ status) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n_rows; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    int own = 0;
+    if (i < n_rows) {
+      const long long cap = slot_off[i + 1] - slot_off[i];
+      own = (int)((cap + kCH - 1) / kCH);
+      if (own > sc.max_per_row) {
+        atomicOr(status, KV_DEV_CAPACITY);
+        own = sc.max_per_row;
       }
-      meta[2] = steps + 1;
     }
+    int v = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    int wb = 0;
+    for (int k = 0; k < warp; ++k) wb += warp_tot[k];
+    const int incl = carry + wb + v;
+    if (i < n_rows) {
+      sc.item_off[i] = incl - own;
+      for (int c = 0; c < own; ++c) sc.items[incl - own + c] = make_int2(i, c);
+    }
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = incl;
+    __syncthreads();
   }
-  __syncwarp();
-  cluster.sync();  // keep every CTA's shared memory alive until the others have read it
+  if (threadIdx.x == 0) {
+    sc.item_off[n_rows] = carry;
+    *sc.n_items = carry;
+  }
 }
 
 // One block per row: A = 0 on the row's slots, meta reset, budget check.
@@ -790,10 +1039,28 @@ int cap_bound(const kv_shape& sh, const RowMap& m, const kv_params& p) {
 
 }  // namespace
 
+int cap_bound_of(const kv_shape& sh, const RowMap& m, const kv_params& p) { return cap_bound(sh, m, p); }
+
+size_t decode_scratch_bytes(const kv_shape& sh, const RowMap& m, const kv_params& p, long long total_slots) {
+  return dec_scratch_layout(m.n_rows, sh.group, sh.head_dim, cap_bound(sh, m, p), total_slots, nullptr, nullptr);
+}
+
+static long long cache_slots(const kv_shape& sh, const RowMap& m, const kv_params& p, const kv_cache& c) {
+  return c.total_slots > 0 ? c.total_slots : kv_total_slots(&sh, m.L, m.n_seq, &p);
+}
+
 int launch_decode_init(const kv_shape& sh, const RowMap& m, const kv_params& p, const kv_cache& c,
                        cudaStream_t st) {
-  (void)sh;
   decode_init_kernel<<<m.n_rows, 256, 0, st>>>(c.slot_off, c.b, p.sinks_T, p.recent_pct, c.A, c.meta, c.status);
+  if (sh.dtype == KV_BF16 && sh.group <= kTcMaxG) {
+    const long long total = cache_slots(sh, m, p, c);
+    DecScratch sc;
+    const size_t need =
+        dec_scratch_layout(m.n_rows, sh.group, sh.head_dim, cap_bound(sh, m, p), total, (char*)c.scratch, &sc);
+    if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
+    decode_items_kernel<<<1, 1024, 0, st>>>(m.n_rows, c.slot_off, sc, c.status);
+    decode_clear_stamps_kernel<<<64, 256, 0, st>>>(sc, sh.group, sh.head_dim, m.n_rows);
+  }
   return cuda_status(cudaGetLastError());
 }
 
@@ -801,15 +1068,10 @@ int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const
                   const void* k_t, const void* v_t, void* out, cudaStream_t st) {
   if (sh.group > kMaxG) return KV_ERR_ARG;
   const int capb = cap_bound(sh, m, p);
-  int C = 8;
-  while (C > 1 && (capb + C - 1) / C < 128) C >>= 1;
-  const int S_cap = (capb + C - 1) / C;
   DecArgs a;
   a.map = m;
   a.G = sh.group;
   a.d = sh.head_dim;
-  a.C = C;
-  a.S_cap = S_cap;
   a.scale2 = (float)(1.4426950408889634 / std::sqrt((double)sh.head_dim));
   a.gamma = p.gamma;
   a.T = p.sinks_T;
@@ -826,42 +1088,74 @@ int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const
   a.b = c.b;
   a.meta = c.meta;
   a.status = c.status;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(m.n_rows * C);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   cudaError_t e;
-  if (sh.dtype == KV_BF16) {
-    TcDec P;
+  if (sh.dtype == KV_BF16 && sh.group <= kTcMaxG) {
+    const long long total = cache_slots(sh, m, p, c);
+    SkArgs P;
     P.a = a;
-    P.S_pad = ((S_cap + kTcSlots - 1) / kTcSlots) * kTcSlots + 4;
+    P.a.C = 1;
+    P.a.S_cap = 0;
+    const size_t need = dec_scratch_layout(m.n_rows, sh.group, sh.head_dim, capb, total, (char*)c.scratch, &P.sc);
+    if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
     P.nk = sh.head_dim / 64;
     P.limit_ns = kWaitLimitNs;
-    const size_t smem = 1024 + (size_t)kTcStages * kTcSlots * sh.head_dim * 2 +
-                        ((size_t)sh.group * P.S_pad + (size_t)sh.group * sh.head_dim) * sizeof(float);
-    if (smem > 220 * 1024) return KV_ERR_ARG;
-    const long long total = c.total_slots > 0 ? c.total_slots : kv_total_slots(&sh, m.L, m.n_seq, &p);
+    const int stage_bytes = 2 * kTcSlots * sh.head_dim * 2 + kQBytes;
+    const size_t smem = 1024 + (size_t)kSkStages * stage_bytes + (size_t)kGroups * sh.group * sh.head_dim * 4;
     CUtensorMap tmK, tmV;
     if (!encode_rows_bf16(&tmK, c.Kc, sh.head_dim, total, kTcSlots)) return KV_ERR_CUDA;
     if (!encode_rows_bf16(&tmV, c.Vc, sh.head_dim, total, kTcSlots)) return KV_ERR_CUDA;
-    cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = smem;
-    cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, tmK, tmV, P);
+    const size_t fsmem = (size_t)P.sc.max_per_row * kGroups * sizeof(int);
+    if (fsmem > 200 * 1024) return KV_ERR_ARG;
+    auto attn = sh.head_dim == 128 ? decode_attn_kernel<128> : decode_attn_kernel<64>;
+    if (cudaFuncSetAttribute(attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return KV_ERR_ARG;
+    cudaFuncSetAttribute(decode_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    // both launches may start while the kernel before them drains (programmatic
+    // dependent launch); each waits (griddepcontrol.wait) before touching memory
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c1 = {};
+    c1.gridDim = dim3(sm_count());
+    c1.blockDim = dim3(kSkThreads);
+    c1.dynamicSmemBytes = smem;
+    c1.stream = st;
+    c1.attrs = pdl;
+    c1.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c1, attn, tmK, tmV, P);
+    if (e != cudaSuccess) return KV_ERR_CUDA;
+    cudaLaunchConfig_t c2 = c1;
+    c2.gridDim = dim3(m.n_rows * P.sc.max_slices);
+    c2.blockDim = dim3(kFinThreads);
+    c2.dynamicSmemBytes = fsmem;
+    e = cudaLaunchKernelEx(&c2, decode_finish_kernel, P);
   } else {
-    const size_t smem = ((size_t)sh.group * S_cap + 2 * (size_t)sh.group * sh.head_dim) * sizeof(float);
+    int C = 8;
+    while (C > 1 && (capb + C - 1) / C < 128) C >>= 1;
+    a.C = C;
+    a.S_cap = (capb + C - 1) / C;
+    const size_t smem = ((size_t)sh.group * a.S_cap + 2 * (size_t)sh.group * sh.head_dim) * sizeof(float);
     if (smem > 200 * 1024) return KV_ERR_ARG;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(m.n_rows * C);
     cfg.blockDim = dim3(kDecThreads);
     cfg.dynamicSmemBytes = smem;
-    cudaFuncSetAttribute(decode_simple_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<float>, a);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (sh.dtype == KV_BF16) {
+      cudaFuncSetAttribute(decode_simple_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           200 * 1024);
+      e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<__nv_bfloat16>, a);
+    } else {
+      cudaFuncSetAttribute(decode_simple_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<float>, a);
+    }
   }
   return cuda_status(e);
 }

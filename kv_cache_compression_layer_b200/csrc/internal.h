@@ -34,6 +34,7 @@ int launch_allocate(const kv_shape& sh, const RowMap& m, const kv_params& p, con
 int launch_select_gather(const kv_shape& sh, const RowMap& m, const float* s_hat, const void* K, const void* V,
                          const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
                          cudaStream_t st);
+size_t decode_scratch_bytes(const kv_shape& sh, const RowMap& m, const kv_params& p, long long total_slots);
 int launch_decode_init(const kv_shape& sh, const RowMap& m, const kv_params& p, const kv_cache& c,
                        cudaStream_t st);
 int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const kv_cache& c, const void* q_t,

@@ -11,8 +11,9 @@ from typing import Optional, Sequence
 
 import torch
 
-from . import (KV_BF16, META_INTS, kv_allocate, kv_decode_attn_update, kv_decode_init, kv_params, kv_score,
-               kv_select_gather, kv_shape, kv_sss, kv_total_slots, kv_workspace_bytes, make_cache)
+from . import (KV_BF16, META_INTS, kv_allocate, kv_decode_attn_update, kv_decode_init, kv_decode_scratch_bytes,
+               kv_params, kv_score, kv_select_gather, kv_shape, kv_sss, kv_total_slots, kv_workspace_bytes,
+               make_cache)
 
 
 def torch_dtype(dtype_code: int):
@@ -49,7 +50,10 @@ class Compressor:
         self.A = torch.zeros(self.n_slots, dtype=f32, device=dev)
         self.meta = torch.zeros(self.rows * META_INTS, dtype=i32, device=dev)
         self.status = torch.zeros(4, dtype=i32, device=dev)
-        self.cache = make_cache(self.Kc, self.Vc, self.A, self.pos, self.slot_off, self.b, self.meta, self.status)
+        self.scratch = torch.empty(max(256, kv_decode_scratch_bytes(shape, self.L, params, self.n_slots)),
+                                   dtype=torch.uint8, device=dev)
+        self.cache = make_cache(self.Kc, self.Vc, self.A, self.pos, self.slot_off, self.b, self.meta, self.status,
+                                self.scratch)
 
     # -- prefill compression -------------------------------------------------
     def allocate(self, S: torch.Tensor, stream=None):

@@ -51,7 +51,10 @@ def _gpu_cache(cfg, bt, b, idx, count0=None):
              pos=up(pos, torch.int32), slot_off=up(off, torch.int64), b=up(b.astype(np.int32), torch.int32),
              meta=torch.zeros(rows * kv.META_INTS, dtype=torch.int32, device=dev()),
              status=torch.zeros(4, dtype=torch.int32, device=dev()))
-    cache = kv.make_cache(t["Kc"], t["Vc"], t["A"], t["pos"], t["slot_off"], t["b"], t["meta"], t["status"])
+    nbytes = kv.kv_decode_scratch_bytes(shape_of(cfg), cfg.L, params_of(cfg), total)
+    t["scratch"] = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev())
+    cache = kv.make_cache(t["Kc"], t["Vc"], t["A"], t["pos"], t["slot_off"], t["b"], t["meta"], t["status"],
+                          t["scratch"])
     kv.kv_decode_init(shape_of(cfg), cfg.L, params_of(cfg), cache)
     if count0 is not None:  # a cache that is not full yet (no eviction until it is)
         count0 = np.broadcast_to(np.asarray(count0, np.int32), (rows,))
