@@ -269,7 +269,11 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = hbm_peak()
     dec_gbs = dec_bytes / (dec_avg_us * 1e-6) / 1e9
     comp_gbs = comp_bytes / (comp_avg_ms * 1e-3) / 1e9
-    launches_per_step = 2 + (3 if cfg.dtype == "bf16" else 3) + 1 + 2 + 1 + D
+    # our kernels per step: allocate 2, score 3, SSS 1, select 1, gather 1,
+    # decode init 1 (+ the work-item builder on the tensor-core decode path),
+    # then per decode call attention + finish (tensor-core path) or one kernel
+    tc = cfg.dtype == "bf16" and cfg.group <= 8
+    launches_per_step = 2 + 3 + 1 + 1 + 1 + 1 + (1 if tc else 0) + D * (2 if tc else 1)
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -282,7 +286,8 @@ def run_ours(args, rank, world, local_rank):
                    "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
                    "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
                    "decode_bytes_alg": dec_bytes, "decode_steps": D},
-        "roofline": {"kernel": "decode_kernel (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
+        "roofline": {"kernel": "kv_decode_attn_update (decode_attn_kernel + decode_finish_kernel)" if tc
+                     else "kv_decode_attn_update (decode_simple_kernel)", "bound": "hbm", "achieved": dec_gbs,
                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},
         "e2e": {"value": world * tokens / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,

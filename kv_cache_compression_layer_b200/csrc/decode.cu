@@ -350,9 +350,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(const DecArg
 // softmax on the tensor cores (mma.sync m16n8k16: A = the g query rows padded
 // to 16, B = K rows via ldmatrix; then A = P, B = V rows via ldmatrix.trans).
 // Every logit goes to an L2-resident scratch; when a group leaves a row it
-// combines its four warps and writes one (max, sum, O) partial stamped with
-// the step number. No CTA waits on another.
-// decode_finish_kernel (one CTA per row): combines the row's stamped
+// combines its four warps, writes one (max, sum, O) partial and appends its
+// index to the row's partial list. No CTA waits on another.
+// decode_finish_kernel (CTAs per row slice): combines the row's listed
 // partials into the attention output, applies the exact probabilities to A,
 // picks the eviction and updates the row's meta data.
 constexpr int kTcSlots = 64;  // slots per TMA tile
@@ -363,8 +363,8 @@ constexpr int kSkConsumers = 4 * kGroups;
 constexpr int kSkThreads = (kSkConsumers + 1) * 32;
 constexpr int kTcMaxG = 8;                     // query heads per KV head on the tensor-core path
 constexpr int kQBytes = kTcMaxG * 128 * 2;     // staged query rows per stage
-constexpr int kFinThreads = 256;
-constexpr int kFinSlots = 512;  // slots per finishing CTA
+constexpr int kFinThreads = 1024;
+constexpr int kFinSlots = 2048;  // slots per finishing CTA
 
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int slot, int dcol) {
   const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
@@ -405,9 +405,11 @@ struct DecScratch {
   int* n_items;   // [1]
   int* item_off;  // [rows + 1] first item of each row
   int2* items;    // [max_items] (row, chunk)
-  float* part;    // [max_items * 2][stride]: (max[G], sum[G], O[G][d], step stamp) per (item, group)
+  float* part;    // [max_items * groups][stride]: (max[G], sum[G], O[G][d]) per (segment-first item, group)
   float* logits;  // [total_slots][G] logits in log2 units
   int* tickets;   // [rows] finished slices of the current step, reset by the row's last slice
+  int* plist_n;   // [rows] partials written for the row in the current step (reset by its last slice)
+  int* plist;     // [rows][max_per_row * groups] their slot indices
   int4* bests;    // [rows][max_slices] eviction candidate per slice: (A bits, pos, slot, -)
   int max_items, max_per_row, stride, max_slices;
 };
@@ -416,7 +418,7 @@ size_t dec_scratch_layout(int rows, int G, int d, int capb, long long total_slot
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int per_row = (capb + kCH - 1) / kCH;
   const int max_items = rows * per_row;
-  const int stride = 2 * G + G * d + 4;
+  const int stride = (2 * G + G * d + 3) & ~3;
   size_t off = 0;
   const size_t o_n = off;
   off += 256;
@@ -431,6 +433,10 @@ size_t dec_scratch_layout(int rows, int G, int d, int capb, long long total_slot
   const int max_slices = (capb + kFinSlots - 1) / kFinSlots;
   const size_t o_tk = off;
   off += al((size_t)rows * 4);
+  const size_t o_pn = off;
+  off += al((size_t)rows * 4);
+  const size_t o_pl = off;
+  off += al((size_t)rows * per_row * kGroups * 4);
   const size_t o_best = off;
   off += al((size_t)rows * max_slices * 16);
   if (sc && base) {
@@ -440,6 +446,8 @@ size_t dec_scratch_layout(int rows, int G, int d, int capb, long long total_slot
     sc->part = reinterpret_cast<float*>(base + o_part);
     sc->logits = reinterpret_cast<float*>(base + o_log);
     sc->tickets = reinterpret_cast<int*>(base + o_tk);
+    sc->plist_n = reinterpret_cast<int*>(base + o_pn);
+    sc->plist = reinterpret_cast<int*>(base + o_pl);
     sc->bests = reinterpret_cast<int4*>(base + o_best);
     sc->max_slices = max_slices;
     sc->max_items = max_items;
@@ -584,7 +592,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) decode_attn_kernel(const __grid
   const uint64_t keep_policy = make_policy_evict_last();  // logits are read back by the finish kernel
   float* og = o_s + grp * G * D;
   bool aborted = false;
-  int cur_row = -1, seg_u = -1, seg_steps = 0;
+  int cur_row = -1, seg_u = -1;
   uint32_t qa[NDC][2];  // A fragments of the query rows (rows 8..15 of the m16 tile are zero)
   float m0 = -INFINITY, l0 = 0.f;
   float o[2 * NDC][2];  // O[g0][8 i + 2 q4 + {0,1}]
@@ -600,7 +608,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) decode_attn_kernel(const __grid
     if (hrow != cur_row || hrow < 0) {
       if (cur_row >= 0) {
         // leaving a row: this group's running (max, sum, O) becomes one partial at
-        // (first item of the segment, group), stamped with the step number
+        // (first item of the segment, group), listed for the row's finish
         float ls0 = l0;
 #pragma unroll
         for (int off = 1; off <= 2; off <<= 1) ls0 += __shfl_xor_sync(0xffffffffu, ls0, off);
@@ -638,7 +646,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) decode_attn_kernel(const __grid
           part[2 * G + i] = og[i];
           og[i] = 0.f;
         }
-        if (gt == 0) part[2 * G + G * D] = __int_as_float(seg_steps);
+        if (gt == 0) {
+          const int k = atomicAdd(&sc.plist_n[cur_row], 1);
+          if (k < sc.max_per_row * kGroups) sc.plist[(long long)cur_row * sc.max_per_row * kGroups + k] = seg_u * kGroups + grp;
+        }
         named_bar_sync(1 + grp, 128);
         m0 = -INFINITY;
         l0 = 0.f;
@@ -648,7 +659,6 @@ __global__ void __launch_bounds__(kSkThreads, 1) decode_attn_kernel(const __grid
       if (hrow < 0) break;
       cur_row = hrow;
       seg_u = hdr[st].u;
-      seg_steps = hdr[st].steps;
       // query fragments from the staged [G][D] rows (rows >= G are zero)
       const uint32_t qs = smem_u32(ring + st * STAGE) + 2 * TILE;
       const int qrow = lane & 7;
@@ -758,116 +768,100 @@ __global__ void __launch_bounds__(kSkThreads, 1) decode_attn_kernel(const __grid
 }
 
 // Finish of one decode step, one CTA per (row, slice of kFinSlots slots):
-// the row's log-denominators from the partials stamped with this step, this
-// slice's share of the attention output, the exact probabilities applied to
-// A on this slice's slots, and this slice's best eviction candidate. The
-// row's last slice to finish (atomic ticket, no waiting) picks the eviction
-// and updates the row's meta data.
+// the row's log-denominators from the partials the attention kernel listed
+// for the row, this slice's share of the attention output, the exact
+// probabilities p = exp2(logit - lse) added into the decayed scores A of the
+// slice's slots, and the slice's best eviction candidate. The row's last
+// slice to finish (atomic ticket, no waiting) picks the eviction, updates
+// the row's meta data and clears the row's partial list.
 __global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs P) {
   const DecArgs& a = P.a;
   const DecScratch& sc = P.sc;
   const int G = a.G, d = a.d, E = G * d;
   const int row = blockIdx.x / sc.max_slices, slice = blockIdx.x % sc.max_slices;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  extern __shared__ int real[];  // partials of this step, in index order
-  __shared__ float Ms[kMaxG], Li[kMaxG], lse_s[kMaxG];
+  constexpr int kMaxParts = 32;  // partials combined per row (more are folded serially below)
+  __shared__ int plist_s[kMaxParts];
+  __shared__ float pm_s[kMaxParts][kTcMaxG], pl_s[kMaxParts][kTcMaxG];
+  __shared__ float Ms[kTcMaxG], Li[kTcMaxG], lse_s[kTcMaxG];
   __shared__ Best bw[kFinThreads / 32];
-  __shared__ int n_real, last_s;
+  __shared__ int last_s;
 
   pdl_wait();  // the attention kernel's partials and logits are complete
   pdl_launch_dependents();
-  // round 1: the row's state
+  // round 1: the row's state and its list of partials
   int32_t* meta = a.meta + (long long)row * 8;
   const int count = meta[0], next = meta[1], steps = meta[2], count0 = meta[4];
-  const long long base = a.slot_off[row];
-  const int cap = (int)(a.slot_off[row + 1] - base);
-  const int bb = a.b[row];
-  const int i0 = sc.item_off[row], nch = sc.item_off[row + 1] - i0;
+  const int nr_all = sc.plist_n[row];
   const int n = count + 1;
   const int nsl = (n + kFinSlots - 1) / kFinSlots;
   if (slice >= nsl) return;  // uniform over the CTA
+  const long long base = a.slot_off[row];
+  const int cap = (int)(a.slot_off[row + 1] - base);
+  const int bb = a.b[row];
   const int pos_new = row_len(a.map, row) + steps;
-  const int np = nch * kGroups;
-  const float* part0 = sc.part + (long long)i0 * kGroups * sc.stride;
   const int Mr = (a.recent_pct * bb) / 100;
   const int appended = steps + 1;
   const bool evict = n > bb;
   const bool ok = count < cap && next >= 0 && next < cap && (!evict || bb >= a.T + Mr);
-
-  // round 2: which partials belong to this step, and this thread's slots (A, pos, logits)
-  if (warp == 0) {
-    int k = 0;
-    for (int c0 = 0; c0 < np; c0 += 32) {
-      const int c = c0 + lane;
-      const bool used = c < np && __float_as_int(part0[(long long)c * sc.stride + 2 * G + E]) == steps;
-      const unsigned bal = __ballot_sync(0xffffffffu, used);
-      if (used) real[k + __popc(bal & ((1u << lane) - 1u))] = c;
-      k += __popc(bal);
-    }
-    if (lane == 0) n_real = k;
-  }
+  const int nr = min(nr_all, sc.max_per_row * kGroups);
+  const int* plist = sc.plist + (long long)row * sc.max_per_row * kGroups;
+  if (tid < min(nr, kMaxParts)) plist_s[tid] = plist[tid];
+  // round 2: this thread's slots (A, pos, logits) and the eviction threshold
   constexpr int U = kFinSlots / kFinThreads;
-  const int jbase = slice * kFinSlots;
-  float Av[U], lgv[U][kMaxG];
+  float Av[U], lgv[U][kTcMaxG];
   int pv[U];
 #pragma unroll
   for (int k = 0; k < U; ++k) {
-    const int j = jbase + k * kFinThreads + tid;
+    const int j = slice * kFinSlots + k * kFinThreads + tid;
     Av[k] = 0.f;
     pv[k] = 0;
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) lgv[k][g] = -INFINITY;
+    for (int g = 0; g < kTcMaxG; ++g) lgv[k][g] = -INFINITY;
     if (ok && j < n) {
       Av[k] = a.A[base + j];
       pv[k] = a.pos[base + j];
       const float* lg = sc.logits + (base + j) * G;
-      if ((G & 3) == 0) {
-#pragma unroll
-        for (int g4 = 0; g4 < kMaxG; g4 += 4)
-          if (g4 < G) {
-            const float4 v = *reinterpret_cast<const float4*>(lg + g4);
-            lgv[k][g4] = v.x;
-            lgv[k][g4 + 1] = v.y;
-            lgv[k][g4 + 2] = v.z;
-            lgv[k][g4 + 3] = v.w;
-          }
+      if (G == 8) {
+        const float4 v0 = *reinterpret_cast<const float4*>(lg);
+        const float4 v1 = *reinterpret_cast<const float4*>(lg + 4);
+        lgv[k][0] = v0.x; lgv[k][1] = v0.y; lgv[k][2] = v0.z; lgv[k][3] = v0.w;
+        lgv[k][4] = v1.x; lgv[k][5] = v1.y; lgv[k][6] = v1.z; lgv[k][7] = v1.w;
       } else {
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
+        for (int g = 0; g < kTcMaxG; ++g)
           if (g < G) lgv[k][g] = lg[g];
       }
     }
   }
   const int pos_thr = (!ok || appended >= Mr) ? pos_new - Mr + 1 : a.pos[base + max(0, count0 - (Mr - appended))];
   __syncthreads();
-  const int nr = n_real;
-  // round 3: the row's max and denominator per query head (a warp per head)
-  for (int g = warp; g < G; g += kFinThreads / 32) {
-    float M = -INFINITY;
-    float mk = -INFINITY, lk = 0.f;
-    if (lane < nr) {  // a row rarely has more than 32 partials; the loop below covers the rest
-      mk = part0[(long long)real[lane] * sc.stride + g];
-      lk = part0[(long long)real[lane] * sc.stride + G + g];
-    }
-    M = mk;
-    for (int k = lane + 32; k < nr; k += 32) M = fmaxf(M, part0[(long long)real[k] * sc.stride + g]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float Ls = mk > -INFINITY ? lk * exp2f(mk - M) : 0.f;
-    for (int k = lane + 32; k < nr; k += 32) {
-      const float mc = part0[(long long)real[k] * sc.stride + g];
-      if (mc > -INFINITY) Ls += part0[(long long)real[k] * sc.stride + G + g] * exp2f(mc - M);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
-    if (lane == 0) {
-      Ms[g] = M;
-      Li[g] = Ls > 0.f ? 1.f / Ls : 0.f;
-      lse_s[g] = M + log2f(Ls);
-    }
+  // the partials' (max, sum) per query head
+  const int nr_s = min(nr, kMaxParts);
+  if (tid < nr_s * G) {
+    const int k = tid / G, g = tid % G;
+    const float* pc = sc.part + (long long)plist_s[k] * sc.stride;
+    pm_s[k][g] = pc[g];
+    pl_s[k][g] = pc[G + g];
   }
   __syncthreads();
-  // round 4: this slice's share of the output
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int k = 0; k < nr_s; ++k) M = fmaxf(M, pm_s[k][tid]);
+    for (int k = kMaxParts; k < nr; ++k) M = fmaxf(M, sc.part[(long long)plist[k] * sc.stride + tid]);
+    float Ls = 0.f;
+    for (int k = 0; k < nr_s; ++k)
+      if (pm_s[k][tid] > -INFINITY) Ls += pl_s[k][tid] * exp2f(pm_s[k][tid] - M);
+    for (int k = kMaxParts; k < nr; ++k) {
+      const float* pc = sc.part + (long long)plist[k] * sc.stride;
+      if (pc[tid] > -INFINITY) Ls += pc[G + tid] * exp2f(pc[tid] - M);
+    }
+    Ms[tid] = M;
+    Li[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
+    lse_s[tid] = M + log2f(Ls);
+  }
+  __syncthreads();
+  // round 3: this slice's share of the attention output
   {
     const int e0 = (int)((long long)E * slice / nsl), e1 = (int)((long long)E * (slice + 1) / nsl);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + (long long)row * E;
@@ -876,10 +870,10 @@ __global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs
       float acc = 0.f;
 #pragma unroll 4
       for (int k = 0; k < nr; ++k) {
-        const float* pc = part0 + (long long)real[k] * sc.stride;
-        const float mc = pc[g];
+        const int slot = k < kMaxParts ? plist_s[k] : plist[k];
+        const float mc = k < kMaxParts ? pm_s[k][g] : sc.part[(long long)slot * sc.stride + g];
         const float w = mc > -INFINITY ? exp2f(mc - Ms[g]) : 0.f;
-        acc += w * pc[2 * G + i];
+        acc += w * sc.part[(long long)slot * sc.stride + 2 * G + i];
       }
       out[i] = __float2bfloat16_rn(acc * Li[g]);
     }
@@ -888,14 +882,17 @@ __global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs
   const bool timed_out = (*reinterpret_cast<volatile int32_t*>(a.status) & KV_DEV_TIMEOUT) != 0;
   Best best{INFINITY, -1, -1};
   if (ok && !timed_out) {
+    float lse[kTcMaxG];
+#pragma unroll
+    for (int g = 0; g < kTcMaxG; ++g) lse[g] = g < G ? lse_s[g] : 0.f;
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      const int j = jbase + k * kFinThreads + tid;
+      const int j = slice * kFinSlots + k * kFinThreads + tid;
       if (j < n) {
         float psum = 0.f;
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-          if (g < G) psum += ex2_approx(lgv[k][g] - lse_s[g]);
+        for (int g = 0; g < kTcMaxG; ++g)
+          if (g < G) psum += ex2_approx(lgv[k][g] - lse[g]);
         const float Anew = (j == next ? 0.f : a.gamma * Av[k]) + psum;
         a.A[base + j] = Anew;
         const int pj = j == next ? pos_new : pv[k];
@@ -916,17 +913,25 @@ __global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs
   }
   if (lane == 0) bw[warp] = best;
   __syncthreads();
-  if (tid == 0) {
-    Best bst = bw[0];
-    for (int w = 1; w < kFinThreads / 32; ++w)
-      if (better(bw[w], bst)) bst = bw[w];
-    sc.bests[(long long)row * sc.max_slices + slice] = make_int4(__float_as_int(bst.A), bst.pos, bst.slot, 0);
-    __threadfence();
-    last_s = atomicAdd(&sc.tickets[row], 1) == nsl - 1;
+  if (warp == 0) {
+    Best bst = lane < kFinThreads / 32 ? bw[lane] : Best{INFINITY, -1, -1};
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      Best y;
+      y.A = __shfl_xor_sync(0xffffffffu, bst.A, off);
+      y.pos = __shfl_xor_sync(0xffffffffu, bst.pos, off);
+      y.slot = __shfl_xor_sync(0xffffffffu, bst.slot, off);
+      if (better(y, bst)) bst = y;
+    }
+    if (lane == 0) {
+      sc.bests[(long long)row * sc.max_slices + slice] = make_int4(__float_as_int(bst.A), bst.pos, bst.slot, 0);
+      __threadfence();
+      last_s = atomicAdd(&sc.tickets[row], 1) == nsl - 1;
+    }
   }
   __syncthreads();
   if (!last_s || tid != 0) return;
-  // the row's last slice: reduce the candidates, evict, update meta
+  // the row's last slice: reduce the candidates, evict, update meta, clear the list
   __threadfence();
   Best bst{INFINITY, -1, -1};
   for (int k = 0; k < nsl; ++k) {
@@ -934,8 +939,8 @@ __global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs
     const Best c{__int_as_float(v[0]), v[1], v[2]};
     if (better(c, bst)) bst = c;
   }
-  if (!ok) {
-    atomicOr(a.status, KV_DEV_BUDGET);
+  if (!ok || nr_all > sc.max_per_row * kGroups) {
+    atomicOr(a.status, !ok ? KV_DEV_BUDGET : KV_DEV_CAPACITY);
   } else if (!timed_out) {
     if (evict && bst.slot >= 0) {
       meta[0] = bb;
@@ -949,18 +954,11 @@ __global__ void __launch_bounds__(kFinThreads) decode_finish_kernel(const SkArgs
     meta[2] = steps + 1;
   }
   sc.tickets[row] = 0;
-}
-
-// Marks every partial slot as written by no step (stamp -1).
-__global__ void decode_clear_stamps_kernel(DecScratch sc, int G, int d, int n_rows) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_rows; i += gridDim.x * blockDim.x) sc.tickets[i] = 0;
-  const long long n = (long long)sc.max_items * kGroups;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-    sc.part[i * sc.stride + 2 * G + G * d] = __int_as_float(-1);
+  sc.plist_n[row] = 0;
 }
 
 // Builds the work items of every row (rows cut into kCH-slot chunks) and
-// clears the row tickets; one block.
+// clears the row tickets and partial lists; one block.
 __global__ void decode_items_kernel(int n_rows, const int64_t* __restrict__ slot_off, DecScratch sc,
                                     int32_t* __restrict__ status) {
   __shared__ int warp_tot[32];
@@ -991,6 +989,8 @@ __global__ void decode_items_kernel(int n_rows, const int64_t* __restrict__ slot
     for (int k = 0; k < warp; ++k) wb += warp_tot[k];
     const int incl = carry + wb + v;
     if (i < n_rows) {
+      sc.tickets[i] = 0;
+      sc.plist_n[i] = 0;
       sc.item_off[i] = incl - own;
       for (int c = 0; c < own; ++c) sc.items[incl - own + c] = make_int2(i, c);
     }
@@ -1059,7 +1059,6 @@ int launch_decode_init(const kv_shape& sh, const RowMap& m, const kv_params& p, 
         dec_scratch_layout(m.n_rows, sh.group, sh.head_dim, cap_bound(sh, m, p), total, (char*)c.scratch, &sc);
     if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
     decode_items_kernel<<<1, 1024, 0, st>>>(m.n_rows, c.slot_off, sc, c.status);
-    decode_clear_stamps_kernel<<<64, 256, 0, st>>>(sc, sh.group, sh.head_dim, m.n_rows);
   }
   return cuda_status(cudaGetLastError());
 }
@@ -1104,12 +1103,10 @@ int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const
     CUtensorMap tmK, tmV;
     if (!encode_rows_bf16(&tmK, c.Kc, sh.head_dim, total, kTcSlots)) return KV_ERR_CUDA;
     if (!encode_rows_bf16(&tmV, c.Vc, sh.head_dim, total, kTcSlots)) return KV_ERR_CUDA;
-    const size_t fsmem = (size_t)P.sc.max_per_row * kGroups * sizeof(int);
-    if (fsmem > 200 * 1024) return KV_ERR_ARG;
+    const size_t fsmem = 0;
     auto attn = sh.head_dim == 128 ? decode_attn_kernel<128> : decode_attn_kernel<64>;
     if (cudaFuncSetAttribute(attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return KV_ERR_ARG;
-    cudaFuncSetAttribute(decode_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     // both launches may start while the kernel before them drains (programmatic
     // dependent launch); each waits (griddepcontrol.wait) before touching memory
     cudaLaunchAttribute pdl[1];
