@@ -154,14 +154,13 @@ def run_ours(args, rank, world, local_rank):
 
     import kv_cache_compression_layer_b200 as kv
     from kv_cache_compression_layer_b200 import Compressor
+    from kv_cache_compression_layer_b200.replicas import init_group, job_throughput, max_over_ranks, replica_seed
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    if world > 1:
-        from datetime import timedelta
-
-        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
-    cfg = synth.CONFIGS[args.config].with_(seed=rank)
+    init_group("nccl", world, dev)
+    cfg = synth.CONFIGS[args.config]
+    cfg = cfg.with_(seed=replica_seed(cfg.seed, rank))
     bt = synth.make_batch(cfg)
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     shape = kv.make_shape(cfg.n_layers, cfg.n_kv_heads, cfg.group, cfg.head_dim, cfg.w,
@@ -224,13 +223,9 @@ def run_ours(args, rank, world, local_rank):
     step_ms = [a.elapsed_time(c) for a, _, c in step_ev]
     comp_ms = [a.elapsed_time(b) for a, b, _ in step_ev]
     dec_us = [1e3 * s.elapsed_time(e) for row in dec_ev for s, e in row]
-    ms = sum(step_ms) / len(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world, dev)
     tokens = sum(cfg.L)
-    value = world * tokens / (ms * 1e-3)
+    value = job_throughput(tokens, world, ms)
 
     # end to end through the C ABI from pinned host buffers (copies and the
     # read-back of the decode outputs inside the timed region)
@@ -251,11 +246,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(c))
-    e2e = sum(e2e_ms) / len(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = float(t.item())
+    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world, dev)
 
     # roofline of the dominant kernel (the decode step) and of the compress stage
     b = comp.b.cpu().numpy().astype(np.int64)
@@ -290,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
                      else "kv_decode_attn_update (decode_simple_kernel)", "bound": "hbm", "achieved": dec_gbs,
                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},
-        "e2e": {"value": world * tokens / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(tokens, world, e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
