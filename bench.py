@@ -262,9 +262,9 @@ def run_ours(args, rank, world, local_rank):
     comp_gbs = comp_bytes / (comp_avg_ms * 1e-3) / 1e9
     # our kernels per step: allocate 2, score 3, SSS 1, select 1, gather 1,
     # decode init 1 (+ the work-item builder on the tensor-core decode path),
-    # then per decode call attention + finish (tensor-core path) or one kernel
+    # then one kernel per decode call
     tc = cfg.dtype == "bf16" and cfg.group <= 8
-    launches_per_step = 2 + 3 + 1 + 1 + 1 + 1 + (1 if tc else 0) + D * (2 if tc else 1)
+    launches_per_step = 2 + 3 + 1 + 1 + 1 + 1 + (1 if tc else 0) + D
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -277,7 +277,7 @@ def run_ours(args, rank, world, local_rank):
                    "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
                    "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
                    "decode_bytes_alg": dec_bytes, "decode_steps": D},
-        "roofline": {"kernel": "kv_decode_attn_update (decode_attn_kernel + decode_finish_kernel)" if tc
+        "roofline": {"kernel": "kv_decode_attn_update (decode_attn_kernel)" if tc
                      else "kv_decode_attn_update (decode_simple_kernel)", "bound": "hbm", "achieved": dec_gbs,
                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},

@@ -1,0 +1,946 @@
+// kv_decode_attn_update on bf16 caches with g <= 8 query heads per KV head:
+// one persistent launch per decode step (VoxZip, second stage:
+// A^(t) = gamma [A^(t-1), 0] + softmax(q_t K_t^T / sqrt d), then keep the T
+// sinks, the M most recent entries and the top-N of the middle by A).
+//
+// Every row's b + 1 slots are cut into work items of kCH slots; one CTA per
+// SM takes a contiguous run of items, so each CTA owns a contiguous range of
+// the slot space.
+//
+// Attention phase. Twelve warps form three groups of four. The CTA's items
+// are walked as a sequence of 64-slot tiles and group k takes the tiles with
+// index = k (mod 3). Each group feeds itself: its first thread streams its
+// tiles (K and V as 128-byte swizzled TMA boxes, the row's g query rows as a
+// bulk copy, a header with the row's step state) into the group's two
+// stages, and refills a stage as soon as the group has finished with it.
+// In a group each warp owns 16 slots of a tile and runs one pass of online
+// softmax on the tensor cores (mma.sync m16n8k16: A = the g query rows padded
+// to 16, B = K rows via ldmatrix; then A = P, B = V rows via ldmatrix.trans).
+// Every logit goes to an L2-resident scratch; when a group leaves a row it
+// combines its four warps into one (max, sum, O) partial and lists it for
+// the row. The appended token's K and V rows are patched into the tile that
+// holds its slot and written to the cache by the warp that owns that slot.
+//
+// Grid barrier (all CTAs are resident: one per SM by shared memory; the
+// wait is bounded and reports KV_DEV_TIMEOUT).
+//
+// Finish phase. (1) Output units of 256 elements of a row's g x d output,
+// spread over every warp of the grid, combine the row's partials into the
+// attention output. (2) Each CTA computes the row constants (log2 of the
+// softmax denominators per query head, eviction thresholds) of the rows in
+// its range; then every warp sweeps its share of the CTA's slots, adds the
+// exact probabilities into A and proposes its smallest middle A per row
+// piece. The piece that completes a row's slot count picks the eviction
+// from the row's proposals and writes the row's meta data for the next step.
+#include "decode_common.cuh"
+
+namespace kvc {
+namespace {
+
+constexpr int kTcSlots = 64;                    // slots per TMA tile
+constexpr int kCH = 128;                        // slots per work item
+constexpr int kGroups = 3;                      // consumer groups of four warps
+constexpr int kGStages = 2;                     // TMA stages per group
+constexpr int kStages = kGroups * kGStages;
+constexpr int kWarps = 4 * kGroups;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kQBytes = kTcMaxG * 128 * 2;      // staged query rows per stage (d <= 128)
+constexpr int kPartO = 2 * kTcMaxG;             // offset of O in a partial (16-byte aligned)
+constexpr int kOutUnit = 256;                   // output elements per output unit
+constexpr int kRowsBatch = 64;                  // row constants held at once by a CTA's finish
+
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int slot, int dcol) {
+  const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
+  return tile + box * (kTcSlots * 128) + slot * 128 + ((chunk ^ (slot & 7)) << 4);
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Scratch of the tensor-core path inside kv_cache.scratch.
+struct TcScratch {
+  int* n_items;    // [1]
+  int* item_off;   // [rows + 1] first item of each row
+  int2* items;     // [max_items] (row, chunk)
+  float* part;     // [max_items * kGroups][stride]: max[G] at 0, sum[G] at G, O[G][d] at kPartO,
+                   // per (first item of a group's segment, group)
+  float* logits;   // [total_slots][G] logits in log2 units
+  int* plist_n;    // [2][rows] partials listed for the row in steps of even / odd parity; the
+                   // row's finish clears the counter of the row's next step
+  int* plist;      // [rows][max_per_row * kGroups] their indices
+  int* done;       // [rows] slots of the row finished in the current step
+  int* best_n;     // [rows] eviction proposals of the row in the current step
+  int4* bests;     // [rows][max_bests] proposals (A bits, pos, slot, -)
+  unsigned* bar;   // [2] grid barrier: arrivals, generation
+  int max_items, max_per_row, stride, max_bests;
+};
+
+struct TcArgs {
+  DecArgs a;
+  TcScratch sc;
+  unsigned long long limit_ns;
+};
+
+// What a group's first thread learns about a tile and hands to its group.
+struct TileHdr {
+  int row, u, st0, c1, count, next, steps, cap;  // row = -1: the group's tiles are done
+  long long base;
+};
+
+size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* base, TcScratch* sc) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const int per_row = (capb + kCH - 1) / kCH;
+  const int max_items = rows * per_row;
+  const int stride = (kPartO + G * d + 3) & ~3;
+  const int max_bests = (per_row + 1) * kWarps;
+  size_t off = 0;
+  const size_t o_n = off;
+  off += 256;
+  const size_t o_ioff = off;
+  off += al((size_t)(rows + 1) * 4);
+  const size_t o_items = off;
+  off += al((size_t)max_items * 8);
+  const size_t o_part = off;
+  off += al((size_t)max_items * kGroups * stride * 4);
+  const size_t o_log = off;
+  off += al((size_t)total_slots * G * 4);
+  const size_t o_pn = off;
+  off += al((size_t)rows * 2 * 4);
+  const size_t o_pl = off;
+  off += al((size_t)rows * per_row * kGroups * 4);
+  const size_t o_done = off;
+  off += al((size_t)rows * 4);
+  const size_t o_bn = off;
+  off += al((size_t)rows * 4);
+  const size_t o_best = off;
+  off += al((size_t)rows * max_bests * 16);
+  const size_t o_bar = off;
+  off += 256;
+  if (sc && base) {
+    sc->n_items = reinterpret_cast<int*>(base + o_n);
+    sc->item_off = reinterpret_cast<int*>(base + o_ioff);
+    sc->items = reinterpret_cast<int2*>(base + o_items);
+    sc->part = reinterpret_cast<float*>(base + o_part);
+    sc->logits = reinterpret_cast<float*>(base + o_log);
+    sc->plist_n = reinterpret_cast<int*>(base + o_pn);
+    sc->plist = reinterpret_cast<int*>(base + o_pl);
+    sc->done = reinterpret_cast<int*>(base + o_done);
+    sc->best_n = reinterpret_cast<int*>(base + o_bn);
+    sc->bests = reinterpret_cast<int4*>(base + o_best);
+    sc->bar = reinterpret_cast<unsigned*>(base + o_bar);
+    sc->max_items = max_items;
+    sc->max_per_row = per_row;
+    sc->stride = stride;
+    sc->max_bests = max_bests;
+  }
+  return off;
+}
+
+// Builds the work items of every row (rows cut into kCH-slot chunks) and
+// clears the per-row step counters and the grid barrier; one block.
+__global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off, TcScratch sc,
+                                int32_t* __restrict__ status) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    sc.bar[0] = 0;
+    sc.bar[1] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < n_rows; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    int own = 0;
+    if (i < n_rows) {
+      const long long cap = slot_off[i + 1] - slot_off[i];
+      own = (int)((cap + kCH - 1) / kCH);
+      if (own > sc.max_per_row) {
+        atomicOr(status, KV_DEV_CAPACITY);
+        own = sc.max_per_row;
+      }
+    }
+    int v = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    int wb = 0;
+    for (int k = 0; k < warp; ++k) wb += warp_tot[k];
+    const int incl = carry + wb + v;
+    if (i < n_rows) {
+      sc.plist_n[i] = 0;
+      sc.plist_n[n_rows + i] = 0;
+      sc.done[i] = 0;
+      sc.best_n[i] = 0;
+      sc.item_off[i] = incl - own;
+      for (int c = 0; c < own; ++c) sc.items[incl - own + c] = make_int2(i, c);
+    }
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    sc.item_off[n_rows] = carry;
+    *sc.n_items = carry;
+  }
+}
+
+// The walk over a CTA's tiles in issue order (items u0..u1 in turn, each cut
+// into 64-slot tiles). A group's first thread keeps one; the next row's
+// state is loaded one row ahead so that a row change does not stall it.
+struct Walk {
+  int u, u1;           // current item, end of the CTA's items
+  int t, nt;           // tile within the item, tiles of the item
+  int it;              // CTA-wide index of the current tile
+  int row, chunk, nchunk, c1;
+  int cap, count, next, steps;
+  long long base;
+  long long nend;      // slot_off[row + 2]
+  int ncount, nnext, nsteps;
+};
+
+__device__ __forceinline__ void walk_prefetch(Walk& w, const DecArgs& a, int max_per_row) {
+  w.nchunk = min((w.cap + kCH - 1) / kCH, max_per_row);
+  if (w.row + 1 < a.map.n_rows) {  // next row's state, consumed at the next row change
+    w.nend = a.slot_off[w.row + 2];
+    const int32_t* m = a.meta + (long long)(w.row + 1) * 8;
+    w.ncount = m[0];
+    w.nnext = m[1];
+    w.nsteps = m[2];
+  }
+}
+
+__device__ __forceinline__ void walk_item(Walk& w) {
+  const int c0 = w.chunk * kCH;
+  w.c1 = min(c0 + kCH, w.cap);
+  w.nt = (w.c1 - c0 + kTcSlots - 1) / kTcSlots;
+  w.t = 0;
+}
+
+// Positions the walk on tile 0 of the CTA; false when the CTA has no items.
+__device__ __forceinline__ bool walk_first(Walk& w, const DecArgs& a, const TcScratch& sc, int u0, int u1) {
+  w.u = u0;
+  w.u1 = u1;
+  w.it = 0;
+  if (u0 >= u1) return false;
+  const int2 item = sc.items[u0];
+  w.row = item.x;
+  w.chunk = item.y;
+  w.base = a.slot_off[w.row];
+  w.cap = (int)(a.slot_off[w.row + 1] - w.base);
+  const int32_t* m = a.meta + (long long)w.row * 8;
+  w.count = m[0];
+  w.next = m[1];
+  w.steps = m[2];
+  walk_prefetch(w, a, sc.max_per_row);
+  walk_item(w);
+  return true;
+}
+
+// Moves to the next tile of the CTA; false past the last one.
+__device__ __forceinline__ bool walk_advance(Walk& w, const DecArgs& a, int max_per_row) {
+  ++w.it;
+  if (++w.t < w.nt) return true;
+  if (++w.u >= w.u1) return false;
+  if (++w.chunk >= w.nchunk) {  // the next row
+    w.chunk = 0;
+    w.base += w.cap;
+    w.cap = (int)(w.nend - w.base);
+    w.count = w.ncount;
+    w.next = w.nnext;
+    w.steps = w.nsteps;
+    ++w.row;
+    walk_prefetch(w, a, max_per_row);
+  }
+  walk_item(w);
+  return true;
+}
+
+// Moves to the next tile that group `grp` takes.
+__device__ __forceinline__ bool walk_next(Walk& w, int grp, const DecArgs& a, int max_per_row) {
+  for (;;) {
+    if (!walk_advance(w, a, max_per_row)) return false;
+    if (w.it % kGroups == grp) return true;
+  }
+}
+
+// Streams the walk's current tile into a stage: header, K and V boxes, query rows.
+template <int D>
+__device__ __forceinline__ void issue_tile(const Walk& w, uint8_t* stage, uint64_t* bar, TileHdr* h,
+                                           const CUtensorMap* tmK, const CUtensorMap* tmV, const DecArgs& a,
+                                           uint64_t policy) {
+  constexpr int TILE = kTcSlots * D * 2;
+  const int q_bytes = a.G * D * 2;
+  h->row = w.row;
+  h->u = w.u;
+  h->st0 = w.chunk * kCH + w.t * kTcSlots;
+  h->c1 = w.c1;
+  h->count = w.count;
+  h->next = w.next;
+  h->steps = w.steps;
+  h->cap = w.cap;
+  h->base = w.base;
+  mbar_arrive_expect_tx(bar, 2 * TILE + q_bytes);
+  const int y = (int)(w.base + h->st0);
+#pragma unroll
+  for (int bx = 0; bx < D / 64; ++bx) {
+    tma_load_2d_hint(stage + bx * kTcSlots * 128, tmK, bar, bx * 64, y, policy);
+    tma_load_2d_hint(stage + TILE + bx * kTcSlots * 128, tmV, bar, bx * 64, y, policy);
+  }
+  bulk_load(stage + 2 * TILE, static_cast<const __nv_bfloat16*>(a.q) + (long long)w.row * a.G * D, q_bytes, bar);
+}
+
+// Per-warp scratch of the finish phase (in the freed tile ring).
+struct WarpScr {
+  int pidx[32];                // the row's first 32 partial indices
+  float pm[32][kTcMaxG];       // their maxima
+  float M[kTcMaxG], Li[kTcMaxG], lse[kTcMaxG];
+};
+
+// Constants of one row for the slot sweep (in the freed tile ring).
+struct RowC {
+  float lse[kTcMaxG];
+  long long base;
+  int cap, n, next, pos_new, pos_thr, bb, steps, flags;  // flags: 1 ok, 2 evict, 4 too many partials
+};
+
+// The row's softmax statistics per query head, merged by one warp from the
+// partials listed for the row in this step: M_g, 1/L_g and lse_g = M_g +
+// log2 L_g into ws, and the first 32 partials' indices and maxima.
+__device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, int lane, WarpScr& ws, int& nr_out,
+                                          int& nr_all_out) {
+  const DecArgs& a = P.a;
+  const TcScratch& sc = P.sc;
+  const int G = a.G;
+  const int maxp = sc.max_per_row * kGroups;
+  const int nr_all = __ldcg(sc.plist_n + lbuf * a.map.n_rows + row);
+  const int nr = min(nr_all, maxp);
+  const int* plist = sc.plist + (long long)row * maxp;
+  float m[kTcMaxG], l[kTcMaxG];
+#pragma unroll
+  for (int g = 0; g < kTcMaxG; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+  }
+  for (int k = lane; k < nr; k += 32) {
+    const int pi = __ldcg(plist + k);
+    const float* pc = sc.part + (long long)pi * sc.stride;
+    if (k < 32) ws.pidx[k] = pi;
+#pragma unroll
+    for (int g = 0; g < kTcMaxG; ++g) {
+      if (g < G) {
+        const float mk = __ldcg(pc + g), lk = __ldcg(pc + G + g);
+        if (k < 32) ws.pm[k][g] = mk;
+        if (mk > -INFINITY) {
+          const float mn = fmaxf(m[g], mk);
+          l[g] = l[g] * ex2_approx(m[g] - mn) + lk * ex2_approx(mk - mn);
+          m[g] = mn;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < kTcMaxG; ++g) {
+    float M = m[g];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = m[g] > -INFINITY ? l[g] * ex2_approx(m[g] - M) : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0 && g < G) {
+      ws.M[g] = M;
+      ws.Li[g] = L > 0.f ? 1.f / L : 0.f;
+      ws.lse[g] = M + log2f(L);
+    }
+  }
+  __syncwarp();
+  nr_out = nr;
+  nr_all_out = nr_all;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                const __grid_constant__ CUtensorMap tmV,
+                                                                const __grid_constant__ TcArgs P) {
+  constexpr int NDC = D / 16;             // 16-wide chunks of d
+  constexpr int TILE = kTcSlots * D * 2;  // bytes of one K or V tile
+  constexpr int STAGE = 2 * TILE + kQBytes;
+  static_assert(kWarps * sizeof(WarpScr) + kRowsBatch * sizeof(RowC) <= kStages * STAGE, "finish scratch");
+  const DecArgs& a = P.a;
+  const TcScratch& sc = P.sc;
+  const int G = a.G;
+  const int n_rows = a.map.n_rows;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = warp >> 2, gt = tid & 127;
+
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  float* o_s = reinterpret_cast<float*>(ring + kStages * STAGE);  // [groups][G][D]
+  __shared__ uint64_t full[kStages];
+  __shared__ TileHdr hdr[kStages];
+  __shared__ float red_m[kWarps][kTcMaxG], red_l[kWarps][kTcMaxG];
+  __shared__ int abort_s, go_s;
+  __shared__ unsigned gen_s;
+  __shared__ Walk walk_s[kGroups];  // each group's tile walk (its first thread's), kept out of registers
+  __shared__ int more_s[kGroups], ended_s[kGroups], nreal_s[kGroups];
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
+    abort_s = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  for (int i = tid; i < kGroups * G * D; i += kThreads) o_s[i] = 0.f;
+  pdl_wait();  // the previous step has finished with the cache and the scratch
+  pdl_launch_dependents();
+  if (tid == 0) gen_s = *reinterpret_cast<volatile unsigned*>(sc.bar + 1);
+  __syncthreads();
+  const Guard gd{&abort_s, a.status, P.limit_ns};
+  const int lbuf = gen_s & 1;  // parity of this step: which partial counters it uses
+  const int maxp = sc.max_per_row * kGroups;
+  const int n_items = *sc.n_items;
+  const int u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
+  const int u1 = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
+
+  // ---------------------------------------------------------------- attention
+  {
+    Walk& w = walk_s[grp];
+    if (gt == 0) {
+      const uint64_t stream_policy = make_policy_evict_first();  // K and V are read once per step
+      int more = walk_first(w, a, sc, u0, u1);
+      if (more && w.it % kGroups != grp) more = walk_next(w, grp, a, sc.max_per_row);
+      int ended = 0, n_real = 0;
+      for (int s = 0; s < kGStages && !ended; ++s) {
+        const int stg = grp * kGStages + s;
+        if (more) {
+          issue_tile<D>(w, ring + stg * STAGE, &full[stg], &hdr[stg], &tmK, &tmV, a, stream_policy);
+          ++n_real;
+          more = walk_next(w, grp, a, sc.max_per_row);
+        } else {
+          hdr[stg].row = -1;
+          mbar_arrive(&full[stg]);
+          ended = 1;
+        }
+      }
+      more_s[grp] = more;
+      ended_s[grp] = ended;
+      nreal_s[grp] = n_real;
+    }
+
+    const int g0 = lane >> 2, q4 = lane & 3;  // this lane's query row and column pair
+    const bool g_ok = g0 < G;
+    const int m_ = lane >> 3, r_ = lane & 7;
+    const int wslot = (warp & 3) * 16;  // this warp's 16 slots of a tile
+    const uint64_t keep_policy = make_policy_evict_last();  // logits are read back after the barrier
+    float* og = o_s + grp * G * D;
+    bool aborted = false;
+    int cur_row = -1, seg_u = -1;
+    uint32_t qa[NDC][2];  // A fragments of the query rows (rows 8..15 of the m16 tile are zero)
+    float m0 = -INFINITY, l0 = 0.f;
+    float o[2 * NDC][2];  // O[g0][8 i + 2 q4 + {0,1}]
+#pragma unroll
+    for (int i = 0; i < 2 * NDC; ++i) o[i][0] = o[i][1] = 0.f;
+
+    int k = 0;
+    for (;; ++k) {
+      const int stg = grp * kGStages + (k & 1);
+      const bool got = !aborted && wait_bounded(&full[stg], (k >> 1) & 1, gd);
+      if (!got) aborted = true;
+      const int hrow = got ? hdr[stg].row : -1;  // -1: sentinel (or abort)
+      if (hrow != cur_row || hrow < 0) {
+        if (cur_row >= 0) {
+          // leaving a row: the group's running (max, sum, O) becomes one partial at
+          // (first item of the segment, group), listed for the row
+          float ls0 = l0;
+#pragma unroll
+          for (int off = 1; off <= 2; off <<= 1) ls0 += __shfl_xor_sync(0xffffffffu, ls0, off);
+          if (q4 == 0 && g_ok) {
+            red_m[warp][g0] = m0;
+            red_l[warp][g0] = ls0;
+          }
+          named_bar_sync(1 + grp, 128);
+          float M0 = -INFINITY;
+          if (g_ok)
+            for (int w4 = 0; w4 < 4; ++w4) M0 = fmaxf(M0, red_m[grp * 4 + w4][g0]);
+          const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
+          if (g_ok) {
+#pragma unroll
+            for (int i = 0; i < 2 * NDC; ++i) {
+              const int col = i * 8 + q4 * 2;
+              atomicAdd(&og[g0 * D + col], o[i][0] * f0);
+              atomicAdd(&og[g0 * D + col + 1], o[i][1] * f0);
+            }
+          }
+          named_bar_sync(1 + grp, 128);
+          float* part = sc.part + ((long long)seg_u * kGroups + grp) * sc.stride;
+          if (gt < G) {
+            float M = -INFINITY;
+            for (int w4 = 0; w4 < 4; ++w4) M = fmaxf(M, red_m[grp * 4 + w4][gt]);
+            float Ls = 0.f;
+            for (int w4 = 0; w4 < 4; ++w4)
+              if (red_m[grp * 4 + w4][gt] > -INFINITY)
+                Ls += red_l[grp * 4 + w4][gt] * ex2_approx(red_m[grp * 4 + w4][gt] - M);
+            part[gt] = M;
+            part[G + gt] = Ls;
+          }
+          for (int i = gt; i < G * D; i += 128) {
+            part[kPartO + i] = og[i];
+            og[i] = 0.f;
+          }
+          if (gt == 0) {
+            const int kk = atomicAdd(&sc.plist_n[lbuf * n_rows + cur_row], 1);
+            if (kk < maxp) sc.plist[(long long)cur_row * maxp + kk] = seg_u * kGroups + grp;
+          }
+          named_bar_sync(1 + grp, 128);
+          m0 = -INFINITY;
+          l0 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 2 * NDC; ++i) o[i][0] = o[i][1] = 0.f;
+        }
+        if (hrow < 0) break;
+        cur_row = hrow;
+        seg_u = hdr[stg].u;
+        // query fragments from the staged [G][D] rows (rows >= G are zero)
+        const uint32_t qs = smem_u32(ring + stg * STAGE) + 2 * TILE;
+        const int qrow = lane & 7;
+#pragma unroll
+        for (int dc = 0; dc < NDC; ++dc) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(qs + (uint32_t)((qrow < G ? qrow : 0) * D + dc * 16 + (lane >> 4) * 8) * 2, r0, r1, r2, r3);
+          qa[dc][0] = g_ok ? r0 : 0u;
+          qa[dc][1] = g_ok ? r2 : 0u;
+        }
+      }
+      const TileHdr h = hdr[stg];
+      uint8_t* stage = ring + stg * STAGE;
+      const uint32_t ktile = smem_u32(stage), vtile = ktile + TILE;
+      const int n = h.count + 1;
+      const bool row_ok = h.count >= 0 && h.count < h.cap && h.next >= 0 && h.next < h.cap;
+      const long long base = h.base;
+      if (row_ok && h.next >= h.st0 + wslot && h.next < h.st0 + wslot + 16 && h.next < h.c1) {
+        // the appended token: patch its K and V rows into the tile, write them to the cache
+        const int r = h.next - h.st0;
+        const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(a.k) + (long long)h.row * D;
+        const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(a.v) + (long long)h.row * D;
+        if (lane < D / 8) {
+          const uint4 kv = *reinterpret_cast<const uint4*>(kin + lane * 8);
+          const uint4 vv = *reinterpret_cast<const uint4*>(vin + lane * 8);
+          *reinterpret_cast<uint4*>(stage + (swz(ktile, r, lane * 8) - ktile)) = kv;
+          *reinterpret_cast<uint4*>(stage + (swz(vtile, r, lane * 8) - ktile)) = vv;
+          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.Kc) + (base + h.next) * D)[lane] = kv;
+          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.Vc) + (base + h.next) * D)[lane] = vv;
+        }
+        if (lane == 0) a.pos[base + h.next] = row_len(a.map, h.row) + h.steps;
+        fence_proxy_async();
+        __syncwarp();
+      }
+      // logits S = Q K^T for this warp's 16 slots (two n-tiles of 8 slots, even and
+      // odd d-chunks in separate accumulators)
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int dc = 0; dc < NDC; ++dc) {
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4(swz(ktile, wslot + (m_ >> 1) * 8 + r_, dc * 16 + (m_ & 1) * 8), b00, b01, b10, b11);
+        const uint32_t af[4] = {qa[dc][0], 0u, qa[dc][1], 0u};
+        if (dc & 1) {
+          mma16816(t0, af, b00, b01);
+          mma16816(t1, af, b10, b11);
+        } else {
+          mma16816(s0, af, b00, b01);
+          mma16816(s1, af, b10, b11);
+        }
+      }
+      const int jb = h.st0 + wslot + q4 * 2;  // slots jb, jb+1 (n-tile 0) and jb+8, jb+9 (n-tile 1)
+      float x[4];                              // row g0 at those four slots
+      x[0] = s0[0] + t0[0];
+      x[1] = s0[1] + t0[1];
+      x[2] = s1[0] + t1[0];
+      x[3] = s1[1] + t1[1];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = jb + (e & 1) + (e >> 1) * 8;
+        const bool valid = row_ok && j < n && j < h.c1;
+        x[e] = valid ? x[e] * a.scale2 : -INFINITY;
+        if (valid && g_ok) st_f32_hint(sc.logits + (base + j) * G + g0, x[e], keep_policy);
+      }
+      // online softmax update of this warp's running (max, sum, O)
+      float tm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
+      tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 2));
+      const float nm = fmaxf(m0, tm);
+      const float vm = nm == -INFINITY ? 0.f : nm;
+      if (__any_sync(0xffffffffu, nm != m0)) {  // rescale only when a running max moved
+        const float sc0 = ex2_approx(m0 - vm);
+        l0 *= sc0;
+#pragma unroll
+        for (int i = 0; i < 2 * NDC; ++i) {
+          o[i][0] *= sc0;
+          o[i][1] *= sc0;
+        }
+      }
+      m0 = nm;
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        p[e] = ex2_approx(x[e] - vm);
+        l0 += p[e];
+      }
+      const uint32_t pa[4] = {pack_bf16(p[0], p[1]), 0u, pack_bf16(p[2], p[3]), 0u};
+#pragma unroll
+      for (int dn = 0; dn < NDC; ++dn) {
+        uint32_t b0a, b1a, b0b, b1b;
+        ldsm_x4_t(swz(vtile, wslot + (m_ & 1) * 8 + r_, dn * 16 + (m_ >> 1) * 8), b0a, b1a, b0b, b1b);
+        float c0[4] = {o[2 * dn][0], o[2 * dn][1], 0.f, 0.f};
+        float c1[4] = {o[2 * dn + 1][0], o[2 * dn + 1][1], 0.f, 0.f};
+        mma16816(c0, pa, b0a, b1a);
+        mma16816(c1, pa, b0b, b1b);
+        o[2 * dn][0] = c0[0];
+        o[2 * dn][1] = c0[1];
+        o[2 * dn + 1][0] = c1[0];
+        o[2 * dn + 1][1] = c1[1];
+      }
+      named_bar_sync(1 + grp, 128);  // the group is done with this stage: refill it
+      if (gt == 0) {
+        if (more_s[grp]) {
+          issue_tile<D>(w, stage, &full[stg], &hdr[stg], &tmK, &tmV, a, make_policy_evict_first());
+          ++nreal_s[grp];
+          more_s[grp] = walk_next(w, grp, a, sc.max_per_row);
+        } else if (!ended_s[grp]) {
+          hdr[stg].row = -1;
+          mbar_arrive(&full[stg]);
+          ended_s[grp] = 1;
+        }
+      }
+    }
+    if (aborted) {
+      abort_s = 1;
+      if (gt == 0)  // let this group's copies in flight land before the CTA exits
+        for (int t = k; t < nreal_s[grp]; ++t) wait_drain(&full[grp * kGStages + (t & 1)], (t >> 1) & 1, P.limit_ns);
+    }
+  }
+  __syncthreads();
+
+  // ------------------------------------------------------------- grid barrier
+  // Every CTA of the grid is resident (one per SM), so each arrives; the wait
+  // is bounded. The generation counter also gives the next step its parity.
+  if (tid == 0) {
+    int ok = 1;
+    volatile unsigned* genp = sc.bar + 1;
+    __threadfence();
+    if (atomicAdd(sc.bar, 1u) == gridDim.x - 1) {
+      atomicExch(sc.bar, 0u);
+      __threadfence();
+      atomicAdd(sc.bar + 1, 1u);
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (*genp == gen_s) {
+        if (globaltimer() - t0 > P.limit_ns) {
+          atomicOr(a.status, KV_DEV_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    go_s = ok && !abort_s && (*reinterpret_cast<volatile int32_t*>(a.status) & KV_DEV_TIMEOUT) == 0;
+  }
+  __syncthreads();
+  if (!go_s) return;
+
+  // ------------------------------------------------------------------ finish
+  WarpScr& ws = reinterpret_cast<WarpScr*>(ring)[warp];
+  RowC* rc = reinterpret_cast<RowC*>(ring + kWarps * sizeof(WarpScr));
+  const int E = G * D;
+  const int nq = (E + kOutUnit - 1) / kOutUnit;
+
+  // (1) attention outputs: units of kOutUnit elements over every warp of the grid
+  for (int un = blockIdx.x * kWarps + warp; un < n_rows * nq; un += gridDim.x * kWarps) {
+    const int row = un / nq, q = un % nq;
+    int nr, nr_all;
+    row_stats(P, row, lbuf, lane, ws, nr, nr_all);
+    const int e = q * kOutUnit + lane * 8;
+    if (e < E) {
+      const int g = e / D;
+      const float Mg = ws.M[g];
+      const int* plist = sc.plist + (long long)row * maxp;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int kp = 0; kp < nr; ++kp) {
+        const int pi = kp < 32 ? ws.pidx[kp] : __ldcg(plist + kp);
+        const float* pc = sc.part + (long long)pi * sc.stride;
+        const float mk = kp < 32 ? ws.pm[kp][g] : __ldcg(pc + g);
+        const float4 v0 = __ldcg(reinterpret_cast<const float4*>(pc + kPartO + e));
+        const float4 v1 = __ldcg(reinterpret_cast<const float4*>(pc + kPartO + e) + 1);
+        const float wk = mk > -INFINITY ? ex2_approx(mk - Mg) : 0.f;
+        acc[0] += wk * v0.x;
+        acc[1] += wk * v0.y;
+        acc[2] += wk * v0.z;
+        acc[3] += wk * v0.w;
+        acc[4] += wk * v1.x;
+        acc[5] += wk * v1.y;
+        acc[6] += wk * v1.z;
+        acc[7] += wk * v1.w;
+      }
+      const float li = ws.Li[g];
+      uint4 packed;
+      packed.x = pack_bf16(acc[0] * li, acc[1] * li);
+      packed.y = pack_bf16(acc[2] * li, acc[3] * li);
+      packed.z = pack_bf16(acc[4] * li, acc[5] * li);
+      packed.w = pack_bf16(acc[6] * li, acc[7] * li);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (long long)row * E + e) = packed;
+    }
+    __syncwarp();
+  }
+
+  // (2) decayed scores and evictions of this CTA's slots, a batch of rows at a time
+  if (u0 >= u1) return;
+  const int2 it_lo = sc.items[u0], it_hi = sc.items[u1 - 1];
+  const long long S0 = a.slot_off[it_lo.x] + (long long)it_lo.y * kCH;
+  const long long hi_base = a.slot_off[it_hi.x];
+  const long long S1 = hi_base + min((long long)(it_hi.y + 1) * kCH, a.slot_off[it_hi.x + 1] - hi_base);
+  for (int rb = it_lo.x; rb <= it_hi.x; rb += kRowsBatch) {
+    const int rn = min(kRowsBatch, it_hi.x - rb + 1);
+    for (int i = warp; i < rn; i += kWarps) {  // row constants, one warp per row
+      const int row = rb + i;
+      int count = 0, next = 0, steps = 0, count0 = 0, bb = 0;
+      long long base = 0, cap = 0;
+      if (lane == 0) {
+        const int32_t* meta = a.meta + (long long)row * 8;
+        count = meta[0];
+        next = meta[1];
+        steps = meta[2];
+        count0 = meta[4];
+        base = a.slot_off[row];
+        cap = a.slot_off[row + 1] - base;
+        bb = a.b[row];
+      }
+      int nr, nr_all;
+      row_stats(P, row, lbuf, lane, ws, nr, nr_all);
+      if (lane == 0) {
+        RowC& R = rc[i];
+        const int n = count + 1;
+        const int Mr = (a.recent_pct * bb) / 100;
+        const int appended = steps + 1;
+        const bool evict = n > bb;
+        const bool ok = count < cap && next >= 0 && next < cap && (!evict || bb >= a.T + Mr);
+        const int pos_new = row_len(a.map, row) + steps;
+        int pos_thr = pos_new - Mr + 1;
+        if (ok && appended < Mr) pos_thr = __ldcg(a.pos + base + max(0, count0 - (Mr - appended)));
+#pragma unroll
+        for (int g = 0; g < kTcMaxG; ++g) R.lse[g] = g < G ? ws.lse[g] : 0.f;
+        R.base = base;
+        R.cap = (int)cap;
+        R.n = n;
+        R.next = next;
+        R.pos_new = pos_new;
+        R.pos_thr = pos_thr;
+        R.bb = bb;
+        R.steps = steps;
+        R.flags = (ok ? 1 : 0) | (evict ? 2 : 0) | (nr_all > maxp ? 4 : 0);
+      }
+      __syncwarp();
+    }
+    __syncthreads();
+    // this warp's share of the batch's slots within the CTA's range
+    const long long B0 = max(S0, rc[0].base), B1 = min(S1, rc[rn - 1].base + rc[rn - 1].cap);
+    const long long len = B1 > B0 ? B1 - B0 : 0;
+    const long long w0 = B0 + len * warp / kWarps, w1 = B0 + len * (warp + 1) / kWarps;
+    int ri = 0;
+    while (ri < rn - 1 && w0 >= rc[ri].base + rc[ri].cap) ++ri;
+    for (long long p0 = w0; p0 < w1; ++ri) {
+      const RowC& R = rc[ri];
+      const long long p1 = min(w1, R.base + R.cap);
+      const int row = rb + ri;
+      const bool ok = (R.flags & 1) != 0;
+      Best best{INFINITY, -1, -1};
+      if (ok) {
+        float lse[kTcMaxG];
+#pragma unroll
+        for (int g = 0; g < kTcMaxG; ++g) lse[g] = R.lse[g];
+        constexpr int U = 4;
+        for (long long s0 = p0; s0 < p1; s0 += 32 * U) {
+          float Av[U], ps[U];
+          int pv[U];
+#pragma unroll
+          for (int uu = 0; uu < U; ++uu) {
+            const long long s = s0 + uu * 32 + lane;
+            const int j = (int)(s - R.base);
+            Av[uu] = 0.f;
+            ps[uu] = 0.f;
+            pv[uu] = 0;
+            if (s < p1 && j < R.n) {
+              Av[uu] = __ldcg(a.A + s);
+              pv[uu] = __ldcg(a.pos + s);
+              const float* lg = sc.logits + s * G;
+              if (G == kTcMaxG) {
+                const float4 v0 = __ldcg(reinterpret_cast<const float4*>(lg));
+                const float4 v1 = __ldcg(reinterpret_cast<const float4*>(lg) + 1);
+                ps[uu] = ex2_approx(v0.x - lse[0]) + ex2_approx(v0.y - lse[1]) + ex2_approx(v0.z - lse[2]) +
+                         ex2_approx(v0.w - lse[3]) + ex2_approx(v1.x - lse[4]) + ex2_approx(v1.y - lse[5]) +
+                         ex2_approx(v1.z - lse[6]) + ex2_approx(v1.w - lse[7]);
+              } else {
+#pragma unroll
+                for (int g = 0; g < kTcMaxG; ++g)
+                  if (g < G) ps[uu] += ex2_approx(__ldcg(lg + g) - lse[g]);
+              }
+            }
+          }
+#pragma unroll
+          for (int uu = 0; uu < U; ++uu) {
+            const long long s = s0 + uu * 32 + lane;
+            const int j = (int)(s - R.base);
+            if (s < p1 && j < R.n) {
+              const float Anew = (j == R.next ? 0.f : a.gamma * Av[uu]) + ps[uu];
+              a.A[s] = Anew;
+              const int pj = j == R.next ? R.pos_new : pv[uu];
+              if (j >= a.T && pj < R.pos_thr) {
+                const Best c{Anew, pj, j};
+                if (better(c, best)) best = c;
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        Best y;
+        y.A = __shfl_xor_sync(0xffffffffu, best.A, off);
+        y.pos = __shfl_xor_sync(0xffffffffu, best.pos, off);
+        y.slot = __shfl_xor_sync(0xffffffffu, best.slot, off);
+        if (better(y, best)) best = y;
+      }
+      int last = 0;
+      if (lane == 0) {
+        if (best.slot >= 0) {
+          const int idx = atomicAdd(&sc.best_n[row], 1);
+          if (idx < sc.max_bests)
+            sc.bests[(long long)row * sc.max_bests + idx] = make_int4(__float_as_int(best.A), best.pos, best.slot, 0);
+        }
+        __threadfence();
+        const int cnt = (int)(p1 - p0);
+        last = atomicAdd(&sc.done[row], cnt) + cnt == R.cap;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {  // every slot of the row is done: pick the eviction, write the row's meta data
+        __threadfence();
+        const int nb = __ldcg(sc.best_n + row);
+        Best bst{INFINITY, -1, -1};
+        for (int kb = lane; kb < min(nb, sc.max_bests); kb += 32) {
+          const int4 v = __ldcg(sc.bests + (long long)row * sc.max_bests + kb);
+          const Best c{__int_as_float(v.x), v.y, v.z};
+          if (better(c, bst)) bst = c;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          Best y;
+          y.A = __shfl_xor_sync(0xffffffffu, bst.A, off);
+          y.pos = __shfl_xor_sync(0xffffffffu, bst.pos, off);
+          y.slot = __shfl_xor_sync(0xffffffffu, bst.slot, off);
+          if (better(y, bst)) bst = y;
+        }
+        if (lane == 0) {
+          int32_t* meta = a.meta + (long long)row * 8;
+          if (!ok) {
+            atomicOr(a.status, KV_DEV_BUDGET);
+          } else if ((R.flags & 4) || nb > sc.max_bests) {
+            atomicOr(a.status, KV_DEV_CAPACITY);
+          } else {
+            if ((R.flags & 2) && bst.slot >= 0) {
+              meta[0] = R.bb;
+              meta[1] = bst.slot;
+              meta[3] = bst.slot;
+            } else {
+              meta[0] = R.n;
+              meta[1] = R.n;
+              meta[3] = -1;
+            }
+            meta[2] = R.steps + 1;
+          }
+          sc.done[row] = 0;
+          sc.best_n[row] = 0;
+          sc.plist_n[(lbuf ^ 1) * n_rows + row] = 0;  // the row's next step lists its partials there
+        }
+      }
+      p0 = p1;
+    }
+    __syncthreads();  // the row constants are rewritten by the next batch
+  }
+}
+
+}  // namespace
+
+size_t tc_scratch_bytes(const kv_shape& sh, const RowMap& m, int capb, long long total_slots) {
+  return tc_layout(m.n_rows, sh.group, sh.head_dim, capb, total_slots, nullptr, nullptr);
+}
+
+int launch_tc_init(const kv_shape& sh, const RowMap& m, int capb, long long total_slots, const kv_cache& c,
+                   cudaStream_t st) {
+  TcScratch sc;
+  const size_t need = tc_layout(m.n_rows, sh.group, sh.head_dim, capb, total_slots, (char*)c.scratch, &sc);
+  if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
+  tc_items_kernel<<<1, 1024, 0, st>>>(m.n_rows, c.slot_off, sc, c.status);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_tc(const kv_shape& sh, const RowMap& m, int capb, long long total_slots, const DecArgs& a,
+              const kv_cache& c, cudaStream_t st) {
+  if (total_slots >= (1ll << 31)) return KV_ERR_ARG;  // slot indices are TMA coordinates (int32)
+  TcArgs P;
+  P.a = a;
+  P.limit_ns = kWaitLimitNs;
+  const size_t need = tc_layout(m.n_rows, sh.group, sh.head_dim, capb, total_slots, (char*)c.scratch, &P.sc);
+  if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
+  const int stage_bytes = 2 * kTcSlots * sh.head_dim * 2 + kQBytes;
+  const size_t smem = 1024 + (size_t)kStages * stage_bytes + (size_t)kGroups * sh.group * sh.head_dim * 4;
+  CUtensorMap tmK, tmV;
+  if (!encode_rows_bf16(&tmK, c.Kc, sh.head_dim, total_slots, kTcSlots)) return KV_ERR_CUDA;
+  if (!encode_rows_bf16(&tmV, c.Vc, sh.head_dim, total_slots, kTcSlots)) return KV_ERR_CUDA;
+  auto kern = sh.head_dim == 128 ? decode_tc_kernel<128> : decode_tc_kernel<64>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return KV_ERR_ARG;
+  // the launch may start while the previous step's kernel drains (programmatic
+  // dependent launch); it waits (griddepcontrol.wait) before touching memory
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sm_count());  // one CTA per SM (shared memory), all resident for the grid barrier
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tmK, tmV, P));
+}
+
+}  // namespace kvc
