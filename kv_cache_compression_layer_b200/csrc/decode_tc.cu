@@ -44,7 +44,7 @@ constexpr int kGStages = 2;                     // TMA stages per group
 constexpr int kStages = kGroups * kGStages;
 constexpr int kWarps = 4 * kGroups;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kQBytes = kTcMaxG * 128 * 2;      // staged query rows per stage (d <= 128)
+constexpr int kQBytes = kTcMaxG * 128 * 2;      // staged query rows per stage (d <= 128): two 8-row boxes
 constexpr int kPartO = 2 * kTcMaxG;             // offset of O in a partial (16-byte aligned)
 constexpr int kOutUnit = 256;                   // output elements per output unit
 constexpr int kRowsBatch = 64;                  // row constants held at once by a CTA's finish
@@ -52,6 +52,14 @@ constexpr int kRowsBatch = 64;                  // row constants held at once by
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int slot, int dcol) {
   const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
   return tile + box * (kTcSlots * 128) + slot * 128 + ((chunk ^ (slot & 7)) << 4);
+}
+// The staged query rows: two 64-column boxes of 8 rows, 128-byte swizzled.
+__device__ __forceinline__ uint32_t qswz(uint32_t qarea, int row, int dcol) {
+  const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
+  return qarea + box * 1024 + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -74,12 +82,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
 
 // Scratch of the tensor-core path inside kv_cache.scratch.
 struct TcScratch {
@@ -91,7 +93,7 @@ struct TcScratch {
   float* logits;   // [total_slots][G] logits in log2 units
   int* plist_n;    // [2][rows] partials listed for the row in steps of even / odd parity; the
                    // row's finish clears the counter of the row's next step
-  int* plist;      // [rows][max_per_row * kGroups] their indices
+  int* plist;      // [rows][max_per_row * kGroups] list entries (PEnt: per-head max and sum, index)
   int* done;       // [rows] slots of the row finished in the current step
   int* best_n;     // [rows] eviction proposals of the row in the current step
   int4* bests;     // [rows][max_bests] proposals (A bits, pos, slot, -)
@@ -131,7 +133,7 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
   const size_t o_pn = off;
   off += al((size_t)rows * 2 * 4);
   const size_t o_pl = off;
-  off += al((size_t)rows * per_row * kGroups * 4);
+  off += al((size_t)rows * per_row * kGroups * 80);
   const size_t o_done = off;
   off += al((size_t)rows * 4);
   const size_t o_bn = off;
@@ -295,8 +297,8 @@ __device__ __forceinline__ bool walk_next(Walk& w, int grp, const DecArgs& a, in
 // Streams the walk's current tile into a stage: header, K and V boxes, query rows.
 template <int D>
 __device__ __forceinline__ void issue_tile(const Walk& w, uint8_t* stage, uint64_t* bar, TileHdr* h,
-                                           const CUtensorMap* tmK, const CUtensorMap* tmV, const DecArgs& a,
-                                           uint64_t policy) {
+                                           const CUtensorMap* tmK, const CUtensorMap* tmV, const CUtensorMap* tmQ,
+                                           const DecArgs& a, uint64_t policy) {
   constexpr int TILE = kTcSlots * D * 2;
   const int q_bytes = a.G * D * 2;
   h->row = w.row;
@@ -315,7 +317,24 @@ __device__ __forceinline__ void issue_tile(const Walk& w, uint8_t* stage, uint64
     tma_load_2d_hint(stage + bx * kTcSlots * 128, tmK, bar, bx * 64, y, policy);
     tma_load_2d_hint(stage + TILE + bx * kTcSlots * 128, tmV, bar, bx * 64, y, policy);
   }
-  bulk_load(stage + 2 * TILE, static_cast<const __nv_bfloat16*>(a.q) + (long long)w.row * a.G * D, q_bytes, bar);
+#pragma unroll
+  for (int bx = 0; bx < D / 64; ++bx) tma_load_2d(stage + 2 * TILE + bx * 1024, tmQ, bar, bx * 64, w.row * a.G);
+}
+
+// One entry of a row's partial list: the partial's per-head (max, sum) and index.
+struct PEnt {
+  float m[kTcMaxG];
+  float l[kTcMaxG];
+  int pidx, pad0, pad1, pad2;
+};
+static_assert(sizeof(PEnt) == 80, "list entry layout");
+
+__device__ __forceinline__ void ld_pent(const PEnt* e, float (&m)[kTcMaxG], float (&l)[kTcMaxG], int& pidx) {
+  const float4* v = reinterpret_cast<const float4*>(e);
+  const float4 a0 = __ldcg(v), a1 = __ldcg(v + 1), b0 = __ldcg(v + 2), b1 = __ldcg(v + 3);
+  pidx = __ldcg(reinterpret_cast<const int*>(v + 4));
+  m[0] = a0.x; m[1] = a0.y; m[2] = a0.z; m[3] = a0.w; m[4] = a1.x; m[5] = a1.y; m[6] = a1.z; m[7] = a1.w;
+  l[0] = b0.x; l[1] = b0.y; l[2] = b0.z; l[3] = b0.w; l[4] = b1.x; l[5] = b1.y; l[6] = b1.z; l[7] = b1.w;
 }
 
 // Per-warp scratch of the finish phase (in the freed tile ring).
@@ -325,7 +344,7 @@ struct WarpScr {
   float M[kTcMaxG], Li[kTcMaxG], lse[kTcMaxG];
 };
 
-// Constants of one row for the slot sweep (in the freed tile ring).
+// Constants of one row for the slot sweep.
 struct RowC {
   float lse[kTcMaxG];
   long long base;
@@ -333,17 +352,21 @@ struct RowC {
 };
 
 // The row's softmax statistics per query head, merged by one warp from the
-// partials listed for the row in this step: M_g, 1/L_g and lse_g = M_g +
-// log2 L_g into ws, and the first 32 partials' indices and maxima.
+// list of partials of this step: M_g, 1/L_g and lse_g = M_g + log2 L_g into
+// ws, with the first 32 partials' indices and maxima. The list entries carry
+// each partial's (max, sum), so this is one round of loads.
 __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, int lane, WarpScr& ws, int& nr_out,
                                           int& nr_all_out) {
   const DecArgs& a = P.a;
   const TcScratch& sc = P.sc;
   const int G = a.G;
   const int maxp = sc.max_per_row * kGroups;
+  const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
   const int nr_all = __ldcg(sc.plist_n + lbuf * a.map.n_rows + row);
+  float em[kTcMaxG], el[kTcMaxG];
+  int ep = 0;
+  if (lane < maxp) ld_pent(lst + lane, em, el, ep);  // ahead of the count; unused past it
   const int nr = min(nr_all, maxp);
-  const int* plist = sc.plist + (long long)row * maxp;
   float m[kTcMaxG], l[kTcMaxG];
 #pragma unroll
   for (int g = 0; g < kTcMaxG; ++g) {
@@ -351,17 +374,15 @@ __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, in
     l[g] = 0.f;
   }
   for (int k = lane; k < nr; k += 32) {
-    const int pi = __ldcg(plist + k);
-    const float* pc = sc.part + (long long)pi * sc.stride;
-    if (k < 32) ws.pidx[k] = pi;
+    if (k >= 32) ld_pent(lst + k, em, el, ep);
+    if (k < 32) ws.pidx[k] = ep;
 #pragma unroll
     for (int g = 0; g < kTcMaxG; ++g) {
       if (g < G) {
-        const float mk = __ldcg(pc + g), lk = __ldcg(pc + G + g);
-        if (k < 32) ws.pm[k][g] = mk;
-        if (mk > -INFINITY) {
-          const float mn = fmaxf(m[g], mk);
-          l[g] = l[g] * ex2_approx(m[g] - mn) + lk * ex2_approx(mk - mn);
+        if (k < 32) ws.pm[k][g] = em[g];
+        if (em[g] > -INFINITY) {
+          const float mn = fmaxf(m[g], em[g]);
+          l[g] = l[g] * ex2_approx(m[g] - mn) + el[g] * ex2_approx(em[g] - mn);
           m[g] = mn;
         }
       }
@@ -386,9 +407,40 @@ __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, in
   nr_all_out = nr_all;
 }
 
+// Step constants of `row` except its log-denominators (they need the step's
+// partials): slot range, count, next free slot, the appended position, the
+// recent-window threshold, budget checks. Run by one thread.
+__device__ __forceinline__ void row_consts(const DecArgs& a, int row, RowC& R) {
+  const int32_t* meta = a.meta + (long long)row * 8;
+  const int count = meta[0], next = meta[1], steps = meta[2], count0 = meta[4];
+  const long long base = a.slot_off[row];
+  const int cap = (int)(a.slot_off[row + 1] - base);
+  const int bb = a.b[row];
+  const int n = count + 1;
+  const int Mr = (a.recent_pct * bb) / 100;
+  const int appended = steps + 1;
+  const bool evict = n > bb;
+  const bool ok = count < cap && next >= 0 && next < cap && (!evict || bb >= a.T + Mr);
+  const int pos_new = row_len(a.map, row) + steps;
+  // the M most recent positions are >= pos_thr: the appended ones and, early on,
+  // the last prefill entries (never evicted while recent, so their pos is stable)
+  int pos_thr = pos_new - Mr + 1;
+  if (ok && appended < Mr) pos_thr = a.pos[base + max(0, count0 - (Mr - appended))];
+  R.base = base;
+  R.cap = cap;
+  R.n = n;
+  R.next = next;
+  R.pos_new = pos_new;
+  R.pos_thr = pos_thr;
+  R.bb = bb;
+  R.steps = steps;
+  R.flags = (ok ? 1 : 0) | (evict ? 2 : 0);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                 const __grid_constant__ CUtensorMap tmV,
+                                                                const __grid_constant__ CUtensorMap tmQ,
                                                                 const __grid_constant__ TcArgs P) {
   constexpr int NDC = D / 16;             // 16-wide chunks of d
   constexpr int TILE = kTcSlots * D * 2;  // bytes of one K or V tile
@@ -408,7 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __shared__ TileHdr hdr[kStages];
   __shared__ float red_m[kWarps][kTcMaxG], red_l[kWarps][kTcMaxG];
   __shared__ int abort_s, go_s;
-  __shared__ unsigned gen_s;
+  __shared__ unsigned arr0_s;         // the barrier's arrival count when this step began
+  __shared__ RowC rowc[kRowsBatch];   // constants of the first rows of this CTA's finish range
+  __shared__ long long rng_s[2];      // the finish range [S0, S1) of slots
+  __shared__ int rlo_s, rhi_s;        // its first and last row
+  __shared__ int kk_s[kGroups];       // list position of a group's partial
   __shared__ Walk walk_s[kGroups];  // each group's tile walk (its first thread's), kept out of registers
   __shared__ int more_s[kGroups], ended_s[kGroups], nreal_s[kGroups];
 
@@ -418,14 +474,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     fence_barrier_init();
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    prefetch_tmap(&tmQ);
   }
   for (int i = tid; i < kGroups * G * D; i += kThreads) o_s[i] = 0.f;
   pdl_wait();  // the previous step has finished with the cache and the scratch
   pdl_launch_dependents();
-  if (tid == 0) gen_s = *reinterpret_cast<volatile unsigned*>(sc.bar + 1);
+  if (tid == 0) arr0_s = *reinterpret_cast<volatile unsigned*>(sc.bar);
   __syncthreads();
   const Guard gd{&abort_s, a.status, P.limit_ns};
-  const int lbuf = gen_s & 1;  // parity of this step: which partial counters it uses
+  const unsigned step_no = arr0_s / gridDim.x;  // steps since the decode state was built
+  const int lbuf = step_no & 1;                  // which partial counters this step uses
   const int maxp = sc.max_per_row * kGroups;
   const int n_items = *sc.n_items;
   const int u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
@@ -442,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       for (int s = 0; s < kGStages && !ended; ++s) {
         const int stg = grp * kGStages + s;
         if (more) {
-          issue_tile<D>(w, ring + stg * STAGE, &full[stg], &hdr[stg], &tmK, &tmV, a, stream_policy);
+          issue_tile<D>(w, ring + stg * STAGE, &full[stg], &hdr[stg], &tmK, &tmV, &tmQ, a, stream_policy);
           ++n_real;
           more = walk_next(w, grp, a, sc.max_per_row);
         } else {
@@ -455,6 +513,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       ended_s[grp] = ended;
       nreal_s[grp] = n_real;
     }
+    if (warp == 0 && u0 < u1) {
+      // this CTA's finish range and its rows' step constants, loaded while the
+      // first tiles are in flight
+      if (lane == 0) {
+        const int2 i0 = sc.items[u0], i1 = sc.items[u1 - 1];
+        const long long hb = a.slot_off[i1.x];
+        rng_s[0] = a.slot_off[i0.x] + (long long)i0.y * kCH;
+        rng_s[1] = hb + min((long long)(i1.y + 1) * kCH, a.slot_off[i1.x + 1] - hb);
+        rlo_s = i0.x;
+        rhi_s = i1.x;
+      }
+      __syncwarp();
+      const int rn = min(kRowsBatch, rhi_s - rlo_s + 1);
+      for (int i = lane; i < rn; i += 32) row_consts(a, rlo_s + i, rowc[i]);
+    }
 
     const int g0 = lane >> 2, q4 = lane & 3;  // this lane's query row and column pair
     const bool g_ok = g0 < G;
@@ -464,7 +537,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     float* og = o_s + grp * G * D;
     bool aborted = false;
     int cur_row = -1, seg_u = -1;
-    uint32_t qa[NDC][2];  // A fragments of the query rows (rows 8..15 of the m16 tile are zero)
     float m0 = -INFINITY, l0 = 0.f;
     float o[2 * NDC][2];  // O[g0][8 i + 2 q4 + {0,1}]
 #pragma unroll
@@ -500,8 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               atomicAdd(&og[g0 * D + col + 1], o[i][1] * f0);
             }
           }
+          if (gt == 0) kk_s[grp] = atomicAdd(&sc.plist_n[lbuf * n_rows + cur_row], 1);
           named_bar_sync(1 + grp, 128);
-          float* part = sc.part + ((long long)seg_u * kGroups + grp) * sc.stride;
+          const int pidx = seg_u * kGroups + grp;
+          float* part = sc.part + (long long)pidx * sc.stride;
+          const int kk = kk_s[grp];
+          PEnt* ent = reinterpret_cast<PEnt*>(sc.plist) + (long long)cur_row * maxp + kk;
           if (gt < G) {
             float M = -INFINITY;
             for (int w4 = 0; w4 < 4; ++w4) M = fmaxf(M, red_m[grp * 4 + w4][gt]);
@@ -511,14 +587,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 Ls += red_l[grp * 4 + w4][gt] * ex2_approx(red_m[grp * 4 + w4][gt] - M);
             part[gt] = M;
             part[G + gt] = Ls;
+            if (kk < maxp) {
+              ent->m[gt] = M;
+              ent->l[gt] = Ls;
+            }
           }
+          if (gt == 0 && kk < maxp) ent->pidx = pidx;
           for (int i = gt; i < G * D; i += 128) {
             part[kPartO + i] = og[i];
             og[i] = 0.f;
-          }
-          if (gt == 0) {
-            const int kk = atomicAdd(&sc.plist_n[lbuf * n_rows + cur_row], 1);
-            if (kk < maxp) sc.plist[(long long)cur_row * maxp + kk] = seg_u * kGroups + grp;
           }
           named_bar_sync(1 + grp, 128);
           m0 = -INFINITY;
@@ -529,16 +606,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (hrow < 0) break;
         cur_row = hrow;
         seg_u = hdr[stg].u;
-        // query fragments from the staged [G][D] rows (rows >= G are zero)
-        const uint32_t qs = smem_u32(ring + stg * STAGE) + 2 * TILE;
-        const int qrow = lane & 7;
-#pragma unroll
-        for (int dc = 0; dc < NDC; ++dc) {
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4(qs + (uint32_t)((qrow < G ? qrow : 0) * D + dc * 16 + (lane >> 4) * 8) * 2, r0, r1, r2, r3);
-          qa[dc][0] = g_ok ? r0 : 0u;
-          qa[dc][1] = g_ok ? r2 : 0u;
-        }
       }
       const TileHdr h = hdr[stg];
       uint8_t* stage = ring + stg * STAGE;
@@ -567,11 +634,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // odd d-chunks in separate accumulators)
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t qarea = ktile + 2 * TILE;
+      const int qrow = (lane & 7) < G ? (lane & 7) : 0;  // rows >= G are zeroed below
 #pragma unroll
       for (int dc = 0; dc < NDC; ++dc) {
-        uint32_t b00, b01, b10, b11;
+        uint32_t b00, b01, b10, b11, q0, q1;
+        ldsm_x2(qswz(qarea, qrow, dc * 16 + ((lane >> 3) & 1) * 8), q0, q1);
         ldsm_x4(swz(ktile, wslot + (m_ >> 1) * 8 + r_, dc * 16 + (m_ & 1) * 8), b00, b01, b10, b11);
-        const uint32_t af[4] = {qa[dc][0], 0u, qa[dc][1], 0u};
+        const uint32_t af[4] = {g_ok ? q0 : 0u, 0u, g_ok ? q1 : 0u, 0u};
         if (dc & 1) {
           mma16816(t0, af, b00, b01);
           mma16816(t1, af, b10, b11);
@@ -632,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       named_bar_sync(1 + grp, 128);  // the group is done with this stage: refill it
       if (gt == 0) {
         if (more_s[grp]) {
-          issue_tile<D>(w, stage, &full[stg], &hdr[stg], &tmK, &tmV, a, make_policy_evict_first());
+          issue_tile<D>(w, stage, &full[stg], &hdr[stg], &tmK, &tmV, &tmQ, a, make_policy_evict_first());
           ++nreal_s[grp];
           more_s[grp] = walk_next(w, grp, a, sc.max_per_row);
         } else if (!ended_s[grp]) {
@@ -652,23 +722,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   // ------------------------------------------------------------- grid barrier
   // Every CTA of the grid is resident (one per SM), so each arrives; the wait
-  // is bounded. The generation counter also gives the next step its parity.
+  // is bounded. The arrival count only grows (the decode init clears it), so
+  // it also numbers the steps.
   if (tid == 0) {
     int ok = 1;
-    volatile unsigned* genp = sc.bar + 1;
+    const unsigned target = (step_no + 1) * gridDim.x;
     __threadfence();
-    if (atomicAdd(sc.bar, 1u) == gridDim.x - 1) {
-      atomicExch(sc.bar, 0u);
-      __threadfence();
-      atomicAdd(sc.bar + 1, 1u);
-    } else {
-      const uint64_t t0 = globaltimer();
-      while (*genp == gen_s) {
-        if (globaltimer() - t0 > P.limit_ns) {
-          atomicOr(a.status, KV_DEV_TIMEOUT);
-          ok = 0;
-          break;
-        }
+    atomicAdd(sc.bar, 1u);
+    const volatile unsigned* cnt = sc.bar;
+    const uint64_t t0 = globaltimer();
+    while (*cnt < target) {
+      if (globaltimer() - t0 > P.limit_ns) {
+        atomicOr(a.status, KV_DEV_TIMEOUT);
+        ok = 0;
+        break;
       }
     }
     __threadfence();
@@ -679,12 +746,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   // ------------------------------------------------------------------ finish
   WarpScr& ws = reinterpret_cast<WarpScr*>(ring)[warp];
-  RowC* rc = reinterpret_cast<RowC*>(ring + kWarps * sizeof(WarpScr));
+  RowC* rcb = reinterpret_cast<RowC*>(ring + kWarps * sizeof(WarpScr));  // later batches of rows
   const int E = G * D;
   const int nq = (E + kOutUnit - 1) / kOutUnit;
+  const bool has_range = u0 < u1;
+  const int r_lo = has_range ? rlo_s : 0, r_hi = has_range ? rhi_s : -1;
+  const long long S0 = has_range ? rng_s[0] : 0, S1 = has_range ? rng_s[1] : 0;
 
-  // (1) attention outputs: units of kOutUnit elements over every warp of the grid
-  for (int un = blockIdx.x * kWarps + warp; un < n_rows * nq; un += gridDim.x * kWarps) {
+  // (1) log-denominators of the first batch of this CTA's rows (one warp per row)
+  const int rn0 = min(kRowsBatch, r_hi - r_lo + 1);
+  for (int i = warp; i < rn0; i += kWarps) {
+    int nr, nr_all;
+    row_stats(P, r_lo + i, lbuf, lane, ws, nr, nr_all);
+    if (lane < kTcMaxG) rowc[i].lse[lane] = lane < G ? ws.lse[lane] : 0.f;
+    if (lane == 0 && nr_all > maxp) rowc[i].flags |= 4;
+    __syncwarp();
+  }
+
+  // (2) attention outputs: units of kOutUnit elements over every warp of the grid,
+  // spread over the CTAs first and over their warps from the last one down (the
+  // first warps are busy with step (1))
+  for (int un = blockIdx.x + gridDim.x * (kWarps - 1 - warp); un < n_rows * nq; un += gridDim.x * kWarps) {
     const int row = un / nq, q = un % nq;
     int nr, nr_all;
     row_stats(P, row, lbuf, lane, ws, nr, nr_all);
@@ -692,15 +774,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     if (e < E) {
       const int g = e / D;
       const float Mg = ws.M[g];
-      const int* plist = sc.plist + (long long)row * maxp;
+      const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int kp = 0; kp < nr; ++kp) {
-        const int pi = kp < 32 ? ws.pidx[kp] : __ldcg(plist + kp);
-        const float* pc = sc.part + (long long)pi * sc.stride;
-        const float mk = kp < 32 ? ws.pm[kp][g] : __ldcg(pc + g);
-        const float4 v0 = __ldcg(reinterpret_cast<const float4*>(pc + kPartO + e));
-        const float4 v1 = __ldcg(reinterpret_cast<const float4*>(pc + kPartO + e) + 1);
+      auto add = [&](int pi, float mk) {
+        const float* pc = sc.part + (long long)pi * sc.stride + kPartO + e;
+        const float4 v0 = __ldcg(reinterpret_cast<const float4*>(pc));
+        const float4 v1 = __ldcg(reinterpret_cast<const float4*>(pc) + 1);
         const float wk = mk > -INFINITY ? ex2_approx(mk - Mg) : 0.f;
         acc[0] += wk * v0.x;
         acc[1] += wk * v0.y;
@@ -710,7 +789,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         acc[5] += wk * v1.y;
         acc[6] += wk * v1.z;
         acc[7] += wk * v1.w;
-      }
+      };
+      const int n32 = min(nr, 32);
+#pragma unroll 8
+      for (int kp = 0; kp < n32; ++kp) add(ws.pidx[kp], ws.pm[kp][g]);
+      for (int kp = 32; kp < nr; ++kp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g]));
       const float li = ws.Li[g];
       uint4 packed;
       packed.x = pack_bf16(acc[0] * li, acc[1] * li);
@@ -721,56 +804,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
     __syncwarp();
   }
+  __syncthreads();
+  if (!has_range) return;
 
-  // (2) decayed scores and evictions of this CTA's slots, a batch of rows at a time
-  if (u0 >= u1) return;
-  const int2 it_lo = sc.items[u0], it_hi = sc.items[u1 - 1];
-  const long long S0 = a.slot_off[it_lo.x] + (long long)it_lo.y * kCH;
-  const long long hi_base = a.slot_off[it_hi.x];
-  const long long S1 = hi_base + min((long long)(it_hi.y + 1) * kCH, a.slot_off[it_hi.x + 1] - hi_base);
-  for (int rb = it_lo.x; rb <= it_hi.x; rb += kRowsBatch) {
-    const int rn = min(kRowsBatch, it_hi.x - rb + 1);
-    for (int i = warp; i < rn; i += kWarps) {  // row constants, one warp per row
-      const int row = rb + i;
-      int count = 0, next = 0, steps = 0, count0 = 0, bb = 0;
-      long long base = 0, cap = 0;
-      if (lane == 0) {
-        const int32_t* meta = a.meta + (long long)row * 8;
-        count = meta[0];
-        next = meta[1];
-        steps = meta[2];
-        count0 = meta[4];
-        base = a.slot_off[row];
-        cap = a.slot_off[row + 1] - base;
-        bb = a.b[row];
+  // (3) decayed scores and evictions of this CTA's slots, a batch of rows at a time
+  for (int rb = r_lo; rb <= r_hi; rb += kRowsBatch) {
+    const int rn = min(kRowsBatch, r_hi - rb + 1);
+    RowC* rc = rowc;
+    if (rb != r_lo) {  // rows past the first batch: constants here
+      rc = rcb;
+      for (int i = warp; i < rn; i += kWarps) {
+        if (lane == 0) row_consts(a, rb + i, rc[i]);
+        int nr, nr_all;
+        row_stats(P, rb + i, lbuf, lane, ws, nr, nr_all);
+        if (lane < kTcMaxG) rc[i].lse[lane] = lane < G ? ws.lse[lane] : 0.f;
+        if (lane == 0 && nr_all > maxp) rc[i].flags |= 4;
+        __syncwarp();
       }
-      int nr, nr_all;
-      row_stats(P, row, lbuf, lane, ws, nr, nr_all);
-      if (lane == 0) {
-        RowC& R = rc[i];
-        const int n = count + 1;
-        const int Mr = (a.recent_pct * bb) / 100;
-        const int appended = steps + 1;
-        const bool evict = n > bb;
-        const bool ok = count < cap && next >= 0 && next < cap && (!evict || bb >= a.T + Mr);
-        const int pos_new = row_len(a.map, row) + steps;
-        int pos_thr = pos_new - Mr + 1;
-        if (ok && appended < Mr) pos_thr = __ldcg(a.pos + base + max(0, count0 - (Mr - appended)));
-#pragma unroll
-        for (int g = 0; g < kTcMaxG; ++g) R.lse[g] = g < G ? ws.lse[g] : 0.f;
-        R.base = base;
-        R.cap = (int)cap;
-        R.n = n;
-        R.next = next;
-        R.pos_new = pos_new;
-        R.pos_thr = pos_thr;
-        R.bb = bb;
-        R.steps = steps;
-        R.flags = (ok ? 1 : 0) | (evict ? 2 : 0) | (nr_all > maxp ? 4 : 0);
-      }
-      __syncwarp();
+      __syncthreads();
     }
-    __syncthreads();
     // this warp's share of the batch's slots within the CTA's range
     const long long B0 = max(S0, rc[0].base), B1 = min(S1, rc[rn - 1].base + rc[rn - 1].cap);
     const long long len = B1 > B0 ? B1 - B0 : 0;
@@ -784,35 +836,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const bool ok = (R.flags & 1) != 0;
       Best best{INFINITY, -1, -1};
       if (ok) {
+        const uint64_t keep = make_policy_evict_last();
         float lse[kTcMaxG];
 #pragma unroll
         for (int g = 0; g < kTcMaxG; ++g) lse[g] = R.lse[g];
-        constexpr int U = 4;
+        constexpr int U = 8;  // slots per lane in flight
         for (long long s0 = p0; s0 < p1; s0 += 32 * U) {
-          float Av[U], ps[U];
+          // every load first (addresses clamped into the piece, so they are unconditional),
+          // then the arithmetic
+          float lg[U][kTcMaxG];
+          float Av[U];
           int pv[U];
 #pragma unroll
           for (int uu = 0; uu < U; ++uu) {
-            const long long s = s0 + uu * 32 + lane;
-            const int j = (int)(s - R.base);
-            Av[uu] = 0.f;
-            ps[uu] = 0.f;
-            pv[uu] = 0;
-            if (s < p1 && j < R.n) {
-              Av[uu] = __ldcg(a.A + s);
-              pv[uu] = __ldcg(a.pos + s);
-              const float* lg = sc.logits + s * G;
-              if (G == kTcMaxG) {
-                const float4 v0 = __ldcg(reinterpret_cast<const float4*>(lg));
-                const float4 v1 = __ldcg(reinterpret_cast<const float4*>(lg) + 1);
-                ps[uu] = ex2_approx(v0.x - lse[0]) + ex2_approx(v0.y - lse[1]) + ex2_approx(v0.z - lse[2]) +
-                         ex2_approx(v0.w - lse[3]) + ex2_approx(v1.x - lse[4]) + ex2_approx(v1.y - lse[5]) +
-                         ex2_approx(v1.z - lse[6]) + ex2_approx(v1.w - lse[7]);
-              } else {
+            const long long s = min(s0 + uu * 32 + lane, p1 - 1);
+            Av[uu] = __ldcg(a.A + s);
+            pv[uu] = __ldcg(a.pos + s);
+            const float* lgp = sc.logits + s * G;
+            if (G == kTcMaxG) {
+              const float4 v0 = __ldcg(reinterpret_cast<const float4*>(lgp));
+              const float4 v1 = __ldcg(reinterpret_cast<const float4*>(lgp) + 1);
+              lg[uu][0] = v0.x; lg[uu][1] = v0.y; lg[uu][2] = v0.z; lg[uu][3] = v0.w;
+              lg[uu][4] = v1.x; lg[uu][5] = v1.y; lg[uu][6] = v1.z; lg[uu][7] = v1.w;
+            } else {
 #pragma unroll
-                for (int g = 0; g < kTcMaxG; ++g)
-                  if (g < G) ps[uu] += ex2_approx(__ldcg(lg + g) - lse[g]);
-              }
+              for (int g = 0; g < kTcMaxG; ++g) lg[uu][g] = g < G ? __ldcg(lgp + g) : -INFINITY;
             }
           }
 #pragma unroll
@@ -820,8 +868,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const long long s = s0 + uu * 32 + lane;
             const int j = (int)(s - R.base);
             if (s < p1 && j < R.n) {
-              const float Anew = (j == R.next ? 0.f : a.gamma * Av[uu]) + ps[uu];
-              a.A[s] = Anew;
+              float ps = 0.f;
+#pragma unroll
+              for (int g = 0; g < kTcMaxG; ++g) ps += ex2_approx(lg[uu][g] - lse[g]);
+              const float Anew = (j == R.next ? 0.f : a.gamma * Av[uu]) + ps;
+              st_f32_hint(a.A + s, Anew, keep);  // read again by the next step
               const int pj = j == R.next ? R.pos_new : pv[uu];
               if (j >= a.T && pj < R.pos_thr) {
                 const Best c{Anew, pj, j};
@@ -922,9 +973,10 @@ int launch_tc(const kv_shape& sh, const RowMap& m, int capb, long long total_slo
   if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
   const int stage_bytes = 2 * kTcSlots * sh.head_dim * 2 + kQBytes;
   const size_t smem = 1024 + (size_t)kStages * stage_bytes + (size_t)kGroups * sh.group * sh.head_dim * 4;
-  CUtensorMap tmK, tmV;
+  CUtensorMap tmK, tmV, tmQ;
   if (!encode_rows_bf16(&tmK, c.Kc, sh.head_dim, total_slots, kTcSlots)) return KV_ERR_CUDA;
   if (!encode_rows_bf16(&tmV, c.Vc, sh.head_dim, total_slots, kTcSlots)) return KV_ERR_CUDA;
+  if (!encode_rows_bf16(&tmQ, a.q, sh.head_dim, (long long)m.n_rows * sh.group, sh.group)) return KV_ERR_CUDA;
   auto kern = sh.head_dim == 128 ? decode_tc_kernel<128> : decode_tc_kernel<64>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return KV_ERR_ARG;
@@ -940,7 +992,7 @@ int launch_tc(const kv_shape& sh, const RowMap& m, int capb, long long total_slo
   cfg.stream = st;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tmK, tmV, P));
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tmK, tmV, tmQ, P));
 }
 
 }  // namespace kvc
