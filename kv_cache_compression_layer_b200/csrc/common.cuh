@@ -138,6 +138,12 @@ __device__ __forceinline__ uint64_t make_policy_evict_last() {
 __device__ __forceinline__ void st_f32_hint(float* addr, float v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(addr), "f"(v), "l"(policy) : "memory");
 }
+// The same store without a compiler memory clobber, so values already loaded
+// stay in registers across it: callers order it against later reads of the
+// same data with a barrier or fence.
+__device__ __forceinline__ void st_f32_hint_nc(float* addr, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(addr), "f"(v), "l"(policy));
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -91,13 +91,14 @@ struct TcScratch {
   float* part;     // [max_items * kGroups][stride]: max[G] at 0, sum[G] at G, O[G][d] at kPartO,
                    // per (first item of a group's segment, group)
   float* logits;   // [total_slots][G] logits in log2 units
-  int* plist_n;    // [2][rows] partials listed for the row in steps of even / odd parity; the
-                   // row's finish clears the counter of the row's next step
+  int* plist_n;    // [2][rows] partials listed for the row in its steps of even / odd number;
+                   // the row's finish clears the counter of the row's next step
   int* plist;      // [rows][max_per_row * kGroups] list entries (PEnt: per-head max and sum, index)
   int* done;       // [rows] slots of the row finished in the current step
   int* best_n;     // [rows] eviction proposals of the row in the current step
   int4* bests;     // [rows][max_bests] proposals (A bits, pos, slot, -)
-  unsigned* bar;   // [2] grid barrier: arrivals, generation
+  unsigned* attn_done;  // [rows] slots of the row attended so far (grows by the row's capacity
+                        // every step; the decode init clears it)
   int max_items, max_per_row, stride, max_bests;
 };
 
@@ -140,8 +141,8 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
   off += al((size_t)rows * 4);
   const size_t o_best = off;
   off += al((size_t)rows * max_bests * 16);
-  const size_t o_bar = off;
-  off += 256;
+  const size_t o_ad = off;
+  off += al((size_t)rows * 4);
   if (sc && base) {
     sc->n_items = reinterpret_cast<int*>(base + o_n);
     sc->item_off = reinterpret_cast<int*>(base + o_ioff);
@@ -153,7 +154,7 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
     sc->done = reinterpret_cast<int*>(base + o_done);
     sc->best_n = reinterpret_cast<int*>(base + o_bn);
     sc->bests = reinterpret_cast<int4*>(base + o_best);
-    sc->bar = reinterpret_cast<unsigned*>(base + o_bar);
+    sc->attn_done = reinterpret_cast<unsigned*>(base + o_ad);
     sc->max_items = max_items;
     sc->max_per_row = per_row;
     sc->stride = stride;
@@ -163,17 +164,13 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
 }
 
 // Builds the work items of every row (rows cut into kCH-slot chunks) and
-// clears the per-row step counters and the grid barrier; one block.
+// clears the per-row step counters; one block.
 __global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off, TcScratch sc,
                                 int32_t* __restrict__ status) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    carry = 0;
-    sc.bar[0] = 0;
-    sc.bar[1] = 0;
-  }
+  if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < n_rows; base += blockDim.x) {
     const int i = base + threadIdx.x;
@@ -202,6 +199,7 @@ __global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off
       sc.plist_n[n_rows + i] = 0;
       sc.done[i] = 0;
       sc.best_n[i] = 0;
+      sc.attn_done[i] = 0;
       sc.item_off[i] = incl - own;
       for (int c = 0; c < own; ++c) sc.items[incl - own + c] = make_int2(i, c);
     }
@@ -337,17 +335,18 @@ __device__ __forceinline__ void ld_pent(const PEnt* e, float (&m)[kTcMaxG], floa
   l[0] = b0.x; l[1] = b0.y; l[2] = b0.z; l[3] = b0.w; l[4] = b1.x; l[5] = b1.y; l[6] = b1.z; l[7] = b1.w;
 }
 
-// Per-warp scratch of the finish phase (in the freed tile ring).
-struct WarpScr {
+// A row's softmax statistics for the finish (in the freed tile ring).
+struct RowStat {
   int pidx[32];                // the row's first 32 partial indices
   float pm[32][kTcMaxG];       // their maxima
   float M[kTcMaxG], Li[kTcMaxG], lse[kTcMaxG];
+  int nr;                      // partials listed (capped at the list size)
 };
 
-// Constants of one row for the slot sweep.
+// Constants of one row for the finish.
 struct RowC {
-  float lse[kTcMaxG];
   long long base;
+  unsigned target;  // attended-slot count at which every CTA has finished the row's attention
   int cap, n, next, pos_new, pos_thr, bb, steps, flags;  // flags: 1 ok, 2 evict, 4 too many partials
 };
 
@@ -355,7 +354,7 @@ struct RowC {
 // list of partials of this step: M_g, 1/L_g and lse_g = M_g + log2 L_g into
 // ws, with the first 32 partials' indices and maxima. The list entries carry
 // each partial's (max, sum), so this is one round of loads.
-__device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, int lane, WarpScr& ws, int& nr_out,
+__device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, int lane, RowStat& ws, int& nr_out,
                                           int& nr_all_out) {
   const DecArgs& a = P.a;
   const TcScratch& sc = P.sc;
@@ -402,6 +401,7 @@ __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, in
       ws.lse[g] = M + log2f(L);
     }
   }
+  if (lane == 0) ws.nr = nr;
   __syncwarp();
   nr_out = nr;
   nr_all_out = nr_all;
@@ -434,6 +434,7 @@ __device__ __forceinline__ void row_consts(const DecArgs& a, int row, RowC& R) {
   R.pos_thr = pos_thr;
   R.bb = bb;
   R.steps = steps;
+  R.target = (unsigned)(steps + 1) * (unsigned)cap;
   R.flags = (ok ? 1 : 0) | (evict ? 2 : 0);
 }
 
@@ -445,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   constexpr int NDC = D / 16;             // 16-wide chunks of d
   constexpr int TILE = kTcSlots * D * 2;  // bytes of one K or V tile
   constexpr int STAGE = 2 * TILE + kQBytes;
-  static_assert(kWarps * sizeof(WarpScr) + kRowsBatch * sizeof(RowC) <= kStages * STAGE, "finish scratch");
+  static_assert(kRowsBatch * (sizeof(RowStat) + sizeof(RowC)) <= kStages * STAGE, "finish scratch");
   const DecArgs& a = P.a;
   const TcScratch& sc = P.sc;
   const int G = a.G;
@@ -459,12 +460,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __shared__ uint64_t full[kStages];
   __shared__ TileHdr hdr[kStages];
   __shared__ float red_m[kWarps][kTcMaxG], red_l[kWarps][kTcMaxG];
-  __shared__ int abort_s, go_s;
-  __shared__ unsigned arr0_s;         // the barrier's arrival count when this step began
+  __shared__ int abort_s;
   __shared__ RowC rowc[kRowsBatch];   // constants of the first rows of this CTA's finish range
   __shared__ long long rng_s[2];      // the finish range [S0, S1) of slots
   __shared__ int rlo_s, rhi_s;        // its first and last row
+  __shared__ int own_s;               // first row whose attention output this CTA writes
   __shared__ int kk_s[kGroups];       // list position of a group's partial
+  __shared__ int segc_s[kGroups], segs_s[kGroups];  // a group's segment: slots attended, row's step
   __shared__ Walk walk_s[kGroups];  // each group's tile walk (its first thread's), kept out of registers
   __shared__ int more_s[kGroups], ended_s[kGroups], nreal_s[kGroups];
 
@@ -479,11 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   for (int i = tid; i < kGroups * G * D; i += kThreads) o_s[i] = 0.f;
   pdl_wait();  // the previous step has finished with the cache and the scratch
   pdl_launch_dependents();
-  if (tid == 0) arr0_s = *reinterpret_cast<volatile unsigned*>(sc.bar);
   __syncthreads();
   const Guard gd{&abort_s, a.status, P.limit_ns};
-  const unsigned step_no = arr0_s / gridDim.x;  // steps since the decode state was built
-  const int lbuf = step_no & 1;                  // which partial counters this step uses
   const int maxp = sc.max_per_row * kGroups;
   const int n_items = *sc.n_items;
   const int u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
@@ -523,6 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         rng_s[1] = hb + min((long long)(i1.y + 1) * kCH, a.slot_off[i1.x + 1] - hb);
         rlo_s = i0.x;
         rhi_s = i1.x;
+        own_s = i0.y == 0 ? i0.x : i0.x + 1;  // rows whose first item is in this range
       }
       __syncwarp();
       const int rn = min(kRowsBatch, rhi_s - rlo_s + 1);
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               atomicAdd(&og[g0 * D + col + 1], o[i][1] * f0);
             }
           }
-          if (gt == 0) kk_s[grp] = atomicAdd(&sc.plist_n[lbuf * n_rows + cur_row], 1);
+          if (gt == 0) kk_s[grp] = atomicAdd(&sc.plist_n[(segs_s[grp] & 1) * n_rows + cur_row], 1);
           named_bar_sync(1 + grp, 128);
           const int pidx = seg_u * kGroups + grp;
           float* part = sc.part + (long long)pidx * sc.stride;
@@ -598,6 +598,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             og[i] = 0.f;
           }
           named_bar_sync(1 + grp, 128);
+          if (gt == 0) {  // the partial is published: count the slots it covers
+            __threadfence();
+            atomicAdd(&sc.attn_done[cur_row], (unsigned)segc_s[grp]);
+          }
           m0 = -INFINITY;
           l0 = 0.f;
 #pragma unroll
@@ -606,8 +610,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (hrow < 0) break;
         cur_row = hrow;
         seg_u = hdr[stg].u;
+        if (gt == 0) {
+          segs_s[grp] = hdr[stg].steps;
+          segc_s[grp] = 0;
+        }
       }
       const TileHdr h = hdr[stg];
+      if (gt == 0) segc_s[grp] += min(h.st0 + kTcSlots, h.c1) - h.st0;
       uint8_t* stage = ring + stg * STAGE;
       const uint32_t ktile = smem_u32(stage), vtile = ktile + TILE;
       const int n = h.count + 1;
@@ -720,110 +729,106 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   }
   __syncthreads();
 
-  // ------------------------------------------------------------- grid barrier
-  // Every CTA of the grid is resident (one per SM), so each arrives; the wait
-  // is bounded. The arrival count only grows (the decode init clears it), so
-  // it also numbers the steps.
-  if (tid == 0) {
-    int ok = 1;
-    const unsigned target = (step_no + 1) * gridDim.x;
-    __threadfence();
-    atomicAdd(sc.bar, 1u);
-    const volatile unsigned* cnt = sc.bar;
-    const uint64_t t0 = globaltimer();
-    while (*cnt < target) {
-      if (globaltimer() - t0 > P.limit_ns) {
-        atomicOr(a.status, KV_DEV_TIMEOUT);
-        ok = 0;
-        break;
-      }
-    }
-    __threadfence();
-    go_s = ok && !abort_s && (*reinterpret_cast<volatile int32_t*>(a.status) & KV_DEV_TIMEOUT) == 0;
-  }
-  __syncthreads();
-  if (!go_s) return;
-
   // ------------------------------------------------------------------ finish
-  WarpScr& ws = reinterpret_cast<WarpScr*>(ring)[warp];
-  RowC* rcb = reinterpret_cast<RowC*>(ring + kWarps * sizeof(WarpScr));  // later batches of rows
+  // A row is finished by the CTAs whose ranges hold its slots, once every CTA
+  // has attended its part of the row (the row's attended-slot count reaches
+  // its target; the wait is bounded). No CTA waits for rows outside its range.
+  __syncthreads();
+  if (u0 >= u1 || abort_s) return;
+  RowStat* rs = reinterpret_cast<RowStat*>(ring);  // the tile ring is free now
+  RowC* rcb = reinterpret_cast<RowC*>(ring + kRowsBatch * sizeof(RowStat));
   const int E = G * D;
   const int nq = (E + kOutUnit - 1) / kOutUnit;
-  const bool has_range = u0 < u1;
-  const int r_lo = has_range ? rlo_s : 0, r_hi = has_range ? rhi_s : -1;
-  const long long S0 = has_range ? rng_s[0] : 0, S1 = has_range ? rng_s[1] : 0;
+  const int r_lo = rlo_s, r_hi = rhi_s, own_lo = own_s;
+  const long long S0 = rng_s[0], S1 = rng_s[1];
+  for (int rb = r_lo; rb <= r_hi; rb += kRowsBatch) {
+    const int rn = min(kRowsBatch, r_hi - rb + 1);
+    RowC* rc = rb == r_lo ? rowc : rcb;
+    // (1) per row (one warp each): wait for the row's attention, then its log-denominators
+    for (int i = warp; i < rn; i += kWarps) {
+      const int row = rb + i;
+      if (rb != r_lo && lane == 0) row_consts(a, row, rc[i]);
+      __syncwarp();
+      int waited = 1;
+      if (lane == 0) {
+        const volatile unsigned* cnt = sc.attn_done + row;
+        const unsigned target = rc[i].target;
+        if ((int)(*cnt - target) < 0) {
+          const uint64_t t0 = globaltimer();
+          while ((int)(*cnt - target) < 0) {
+            if (globaltimer() - t0 > P.limit_ns) {
+              atomicOr(a.status, KV_DEV_TIMEOUT);
+              waited = 0;
+              break;
+            }
+          }
+        }
+        __threadfence();
+      }
+      waited = __shfl_sync(0xffffffffu, waited, 0);
+      if (!waited) abort_s = 1;
+      int nr, nr_all;
+      row_stats(P, row, rc[i].steps & 1, lane, rs[i], nr, nr_all);
+      if (lane == 0 && nr_all > sc.max_per_row * kGroups) rc[i].flags |= 4;
+      __syncwarp();
+    }
+    __syncthreads();
+    if (abort_s) return;
 
-  // (1) log-denominators of the first batch of this CTA's rows (one warp per row)
-  const int rn0 = min(kRowsBatch, r_hi - r_lo + 1);
-  for (int i = warp; i < rn0; i += kWarps) {
-    int nr, nr_all;
-    row_stats(P, r_lo + i, lbuf, lane, ws, nr, nr_all);
-    if (lane < kTcMaxG) rowc[i].lse[lane] = lane < G ? ws.lse[lane] : 0.f;
-    if (lane == 0 && nr_all > maxp) rowc[i].flags |= 4;
-    __syncwarp();
-  }
-
-  // (2) attention outputs: units of kOutUnit elements over every warp of the grid,
-  // spread over the CTAs first and over their warps from the last one down (the
-  // first warps are busy with step (1))
-  for (int un = blockIdx.x + gridDim.x * (kWarps - 1 - warp); un < n_rows * nq; un += gridDim.x * kWarps) {
-    const int row = un / nq, q = un % nq;
-    int nr, nr_all;
-    row_stats(P, row, lbuf, lane, ws, nr, nr_all);
-    const int e = q * kOutUnit + lane * 8;
-    if (e < E) {
-      const int g = e / D;
-      const float Mg = ws.M[g];
+    // (2) attention outputs of the rows whose first item is in this range: units of
+    // kOutUnit elements over the warps, from the last warp down
+    const int o_first = max(rb, own_lo) - rb;
+    const int n_units = max(0, rn - o_first) * nq;
+    for (int un = kWarps - 1 - warp; un < n_units; un += kWarps) {
+      const int i = o_first + un / nq, q = un % nq;
+      const int row = rb + i;
+      const RowStat& st = rs[i];
+      const int nr = st.nr;
+      // lane: elements e0..e0+3 and e0+128..e0+131 of the unit, so each of the warp's
+      // two loads per partial is 512 contiguous bytes
+      const int e0 = q * kOutUnit + lane * 4, e1 = e0 + kOutUnit / 2;
+      const bool ok0 = e0 < E, ok1 = e1 < E;
+      const int g0 = ok0 ? e0 / D : 0, g1 = ok1 ? e1 / D : 0;
+      const float M0 = st.M[g0], M1 = st.M[g1];
       const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      auto add = [&](int pi, float mk) {
-        const float* pc = sc.part + (long long)pi * sc.stride + kPartO + e;
-        const float4 v0 = __ldcg(reinterpret_cast<const float4*>(pc));
-        const float4 v1 = __ldcg(reinterpret_cast<const float4*>(pc) + 1);
-        const float wk = mk > -INFINITY ? ex2_approx(mk - Mg) : 0.f;
-        acc[0] += wk * v0.x;
-        acc[1] += wk * v0.y;
-        acc[2] += wk * v0.z;
-        acc[3] += wk * v0.w;
-        acc[4] += wk * v1.x;
-        acc[5] += wk * v1.y;
-        acc[6] += wk * v1.z;
-        acc[7] += wk * v1.w;
+      auto add = [&](int pi, float mk0, float mk1) {
+        const float* pc = sc.part + (long long)pi * sc.stride + kPartO;
+        const float4 v0 = ok0 ? __ldcg(reinterpret_cast<const float4*>(pc + e0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v1 = ok1 ? __ldcg(reinterpret_cast<const float4*>(pc + e1)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float w0 = mk0 > -INFINITY ? ex2_approx(mk0 - M0) : 0.f;
+        const float w1 = mk1 > -INFINITY ? ex2_approx(mk1 - M1) : 0.f;
+        acc[0] += w0 * v0.x;
+        acc[1] += w0 * v0.y;
+        acc[2] += w0 * v0.z;
+        acc[3] += w0 * v0.w;
+        acc[4] += w1 * v1.x;
+        acc[5] += w1 * v1.y;
+        acc[6] += w1 * v1.z;
+        acc[7] += w1 * v1.w;
       };
       const int n32 = min(nr, 32);
 #pragma unroll 8
-      for (int kp = 0; kp < n32; ++kp) add(ws.pidx[kp], ws.pm[kp][g]);
-      for (int kp = 32; kp < nr; ++kp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g]));
-      const float li = ws.Li[g];
-      uint4 packed;
-      packed.x = pack_bf16(acc[0] * li, acc[1] * li);
-      packed.y = pack_bf16(acc[2] * li, acc[3] * li);
-      packed.z = pack_bf16(acc[4] * li, acc[5] * li);
-      packed.w = pack_bf16(acc[6] * li, acc[7] * li);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (long long)row * E + e) = packed;
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  if (!has_range) return;
-
-  // (3) decayed scores and evictions of this CTA's slots, a batch of rows at a time
-  for (int rb = r_lo; rb <= r_hi; rb += kRowsBatch) {
-    const int rn = min(kRowsBatch, r_hi - rb + 1);
-    RowC* rc = rowc;
-    if (rb != r_lo) {  // rows past the first batch: constants here
-      rc = rcb;
-      for (int i = warp; i < rn; i += kWarps) {
-        if (lane == 0) row_consts(a, rb + i, rc[i]);
-        int nr, nr_all;
-        row_stats(P, rb + i, lbuf, lane, ws, nr, nr_all);
-        if (lane < kTcMaxG) rc[i].lse[lane] = lane < G ? ws.lse[lane] : 0.f;
-        if (lane == 0 && nr_all > maxp) rc[i].flags |= 4;
-        __syncwarp();
+      for (int kp = 0; kp < n32; ++kp) add(st.pidx[kp], st.pm[kp][g0], st.pm[kp][g1]);
+      for (int kp = 32; kp < nr; ++kp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g0]), __ldcg(&lst[kp].m[g1]));
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (long long)row * E;
+      if (ok0) {
+        const float li = st.Li[g0];
+        uint2 pk;
+        pk.x = pack_bf16(acc[0] * li, acc[1] * li);
+        pk.y = pack_bf16(acc[2] * li, acc[3] * li);
+        *reinterpret_cast<uint2*>(orow + e0) = pk;
       }
-      __syncthreads();
+      if (ok1) {
+        const float li = st.Li[g1];
+        uint2 pk;
+        pk.x = pack_bf16(acc[4] * li, acc[5] * li);
+        pk.y = pack_bf16(acc[6] * li, acc[7] * li);
+        *reinterpret_cast<uint2*>(orow + e1) = pk;
+      }
     }
-    // this warp's share of the batch's slots within the CTA's range
+
+    // (3) decayed scores and evictions: this warp's share of the batch's slots within the range
     const long long B0 = max(S0, rc[0].base), B1 = min(S1, rc[rn - 1].base + rc[rn - 1].cap);
     const long long len = B1 > B0 ? B1 - B0 : 0;
     const long long w0 = B0 + len * warp / kWarps, w1 = B0 + len * (warp + 1) / kWarps;
@@ -837,46 +842,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       Best best{INFINITY, -1, -1};
       if (ok) {
         const uint64_t keep = make_policy_evict_last();
+        const long long rbase = R.base;  // register copies for the sweep
+        const int rn_ = R.n, rnext = R.next, rpos_new = R.pos_new, rpos_thr = R.pos_thr;
         float lse[kTcMaxG];
 #pragma unroll
-        for (int g = 0; g < kTcMaxG; ++g) lse[g] = R.lse[g];
-        constexpr int U = 8;  // slots per lane in flight
-        for (long long s0 = p0; s0 < p1; s0 += 32 * U) {
-          // every load first (addresses clamped into the piece, so they are unconditional),
-          // then the arithmetic
-          float lg[U][kTcMaxG];
-          float Av[U];
-          int pv[U];
+        for (int g = 0; g < kTcMaxG; ++g) lse[g] = g < G ? rs[ri].lse[g] : 0.f;
+        if (G == kTcMaxG) {
+          // lane pairs share a slot: each lane loads 4 of its 8 logits, so a warp's
+          // request is 512 contiguous bytes
+          constexpr int U = 8;  // slot pairs per lane in flight
+          const int half = lane & 1, sl = lane >> 1;
+          float lh[4];
 #pragma unroll
-          for (int uu = 0; uu < U; ++uu) {
-            const long long s = min(s0 + uu * 32 + lane, p1 - 1);
-            Av[uu] = __ldcg(a.A + s);
-            pv[uu] = __ldcg(a.pos + s);
-            const float* lgp = sc.logits + s * G;
-            if (G == kTcMaxG) {
-              const float4 v0 = __ldcg(reinterpret_cast<const float4*>(lgp));
-              const float4 v1 = __ldcg(reinterpret_cast<const float4*>(lgp) + 1);
-              lg[uu][0] = v0.x; lg[uu][1] = v0.y; lg[uu][2] = v0.z; lg[uu][3] = v0.w;
-              lg[uu][4] = v1.x; lg[uu][5] = v1.y; lg[uu][6] = v1.z; lg[uu][7] = v1.w;
-            } else {
+          for (int k = 0; k < 4; ++k) lh[k] = half ? lse[4 + k] : lse[k];
+          for (long long s0 = p0; s0 < p1; s0 += 16 * U) {
+            float4 lv[U];
+            float Av[U];
+            int pv[U];
+#pragma unroll
+            for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
+              const long long s = min(s0 + uu * 16 + sl, p1 - 1);
+              lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
+              Av[uu] = __ldcg(a.A + s);
+              pv[uu] = __ldcg(a.pos + s);
+            }
+#pragma unroll
+            for (int uu = 0; uu < U; ++uu) {
+              float ps = ex2_approx(lv[uu].x - lh[0]) + ex2_approx(lv[uu].y - lh[1]) + ex2_approx(lv[uu].z - lh[2]) +
+                         ex2_approx(lv[uu].w - lh[3]);
+              ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+              const long long s = s0 + uu * 16 + sl;
+              const int j = (int)(s - rbase);
+              if (half == 0 && s < p1 && j < rn_) {
+                const float Anew = (j == rnext ? 0.f : a.gamma * Av[uu]) + ps;
+                st_f32_hint_nc(a.A + s, Anew, keep);  // read again by the next step
+                const int pj = j == rnext ? rpos_new : pv[uu];
+                if (j >= a.T && pj < rpos_thr) {
+                  const Best c{Anew, pj, j};
+                  if (better(c, best)) best = c;
+                }
+              }
+            }
+          }
+        } else {
+          constexpr int U = 4;  // slots per lane in flight
+          for (long long s0 = p0; s0 < p1; s0 += 32 * U) {
+            float lg[U][kTcMaxG];
+            float Av[U];
+            int pv[U];
+#pragma unroll
+            for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
+              const long long s = min(s0 + uu * 32 + lane, p1 - 1);
+              Av[uu] = __ldcg(a.A + s);
+              pv[uu] = __ldcg(a.pos + s);
+              const float* lgp = sc.logits + s * G;
 #pragma unroll
               for (int g = 0; g < kTcMaxG; ++g) lg[uu][g] = g < G ? __ldcg(lgp + g) : -INFINITY;
             }
-          }
 #pragma unroll
-          for (int uu = 0; uu < U; ++uu) {
-            const long long s = s0 + uu * 32 + lane;
-            const int j = (int)(s - R.base);
-            if (s < p1 && j < R.n) {
-              float ps = 0.f;
+            for (int uu = 0; uu < U; ++uu) {
+              const long long s = s0 + uu * 32 + lane;
+              const int j = (int)(s - rbase);
+              if (s < p1 && j < rn_) {
+                float ps = 0.f;
 #pragma unroll
-              for (int g = 0; g < kTcMaxG; ++g) ps += ex2_approx(lg[uu][g] - lse[g]);
-              const float Anew = (j == R.next ? 0.f : a.gamma * Av[uu]) + ps;
-              st_f32_hint(a.A + s, Anew, keep);  // read again by the next step
-              const int pj = j == R.next ? R.pos_new : pv[uu];
-              if (j >= a.T && pj < R.pos_thr) {
-                const Best c{Anew, pj, j};
-                if (better(c, best)) best = c;
+                for (int g = 0; g < kTcMaxG; ++g) ps += ex2_approx(lg[uu][g] - lse[g]);
+                const float Anew = (j == rnext ? 0.f : a.gamma * Av[uu]) + ps;
+                st_f32_hint_nc(a.A + s, Anew, keep);  // read again by the next step
+                const int pj = j == rnext ? rpos_new : pv[uu];
+                if (j >= a.T && pj < rpos_thr) {
+                  const Best c{Anew, pj, j};
+                  if (better(c, best)) best = c;
+                }
               }
             }
           }
@@ -939,12 +976,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           }
           sc.done[row] = 0;
           sc.best_n[row] = 0;
-          sc.plist_n[(lbuf ^ 1) * n_rows + row] = 0;  // the row's next step lists its partials there
+          sc.plist_n[((R.steps + 1) & 1) * n_rows + row] = 0;  // the row's next step lists its partials there
         }
       }
       p0 = p1;
     }
-    __syncthreads();  // the row constants are rewritten by the next batch
+    __syncthreads();  // the row statistics and constants are rewritten by the next batch
   }
 }
 
