@@ -53,6 +53,10 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int slot, int dcol) {
   const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
   return tile + box * (kTcSlots * 128) + slot * 128 + ((chunk ^ (slot & 7)) << 4);
 }
+// Column of (head g, column c) in a group's combine buffer: the 32 lanes of one
+// atomic (8 heads x 4 column pairs) land in 32 different banks.
+__device__ __forceinline__ int ogswz(int g, int c) { return c ^ ((g & 3) << 3) ^ (g >> 2); }
+
 // The staged query rows: two 64-column boxes of 8 rows, 128-byte swizzled.
 __device__ __forceinline__ uint32_t qswz(uint32_t qarea, int row, int dcol) {
   const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
@@ -568,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 #pragma unroll
             for (int i = 0; i < 2 * NDC; ++i) {
               const int col = i * 8 + q4 * 2;
-              atomicAdd(&og[g0 * D + col], o[i][0] * f0);
-              atomicAdd(&og[g0 * D + col + 1], o[i][1] * f0);
+              atomicAdd(&og[g0 * D + ogswz(g0, col)], o[i][0] * f0);
+              atomicAdd(&og[g0 * D + ogswz(g0, col + 1)], o[i][1] * f0);
             }
           }
           if (gt == 0) kk_s[grp] = atomicAdd(&sc.plist_n[(segs_s[grp] & 1) * n_rows + cur_row], 1);
@@ -594,8 +598,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           }
           if (gt == 0 && kk < maxp) ent->pidx = pidx;
           for (int i = gt; i < G * D; i += 128) {
-            part[kPartO + i] = og[i];
-            og[i] = 0.f;
+            const int og_i = (i / D) * D + ogswz(i / D, i % D);
+            part[kPartO + i] = og[og_i];
+            og[og_i] = 0.f;
           }
           named_bar_sync(1 + grp, 128);
           if (gt == 0) {  // the partial is published: count the slots it covers
