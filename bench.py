@@ -34,6 +34,26 @@ UNIT = "audio tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM bytes (read + write) of one decode_tc_kernel launch from an ncu capture
+# of this benchmark's workload (profiles/decode_tc_kernel_3b.md), valid while the
+# kernel source is the one captured (its SHA-256 below); otherwise null.
+NCU_TRAFFIC = {"3b": {"bytes": 139552512,
+                      "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
+                      "sha256": "2787872249ee34b5"}}
+
+
+def measured_traffic(cfg_name: str):
+    import hashlib
+    rec = NCU_TRAFFIC.get(cfg_name)
+    if not rec:
+        return None
+    try:
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return rec["bytes"] if digest.startswith(rec["sha256"]) else None
+
 
 def describe(cfg: synth.Config) -> str:
     return (f"{cfg.name}: {cfg.n_seq} seq, L={list(cfg.L)}, {cfg.n_layers} layers, "
@@ -277,9 +297,9 @@ def run_ours(args, rank, world, local_rank):
                    "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
                    "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
                    "decode_bytes_alg": dec_bytes, "decode_steps": D},
-        "roofline": {"kernel": "kv_decode_attn_update (decode_attn_kernel)" if tc
-                     else "kv_decode_attn_update (decode_simple_kernel)", "bound": "hbm", "achieved": dec_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": None,
+        "roofline": {"kernel": "decode_tc_kernel (kv_decode_attn_update)" if tc
+                     else "decode_simple_kernel (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": measured_traffic(args.config) if tc else None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},
         "e2e": {"value": job_throughput(tokens, world, e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
@@ -303,7 +323,7 @@ def run_reference(args, rank, world):
 
     orc.build()
     cfg = synth.CONFIGS[args.config]
-    rows = list(range(min(args.cpu_rows, cfg.rows)))
+    rows = list(range(min(args.ref_rows, cfg.rows)))
     bt = synth.make_batch(cfg)
     threads = orc.default_threads()
     for _ in range(args.warmup):
@@ -329,7 +349,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="3b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-rows", type=int, default=8)
+    ap.add_argument("--cpu-rows", type=int, default=64, help="rows of the oracle sample for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=8, help="rows per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
