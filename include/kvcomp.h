@@ -99,8 +99,10 @@ typedef struct {
                               prefill count, 3 reserved */
   int32_t* status;         /* device status word (KV_DEV_* bits)          */
   int64_t total_slots;     /* host: rows of Kc/Vc (slot_off[rows]); 0 = kv_total_slots() */
-  void* scratch;           /* device, kv_decode_scratch_bytes() bytes: per-slot logits, per-item
-                              softmax partials, work items, row tickets (L2-resident)         */
+  void* scratch;           /* device, kv_decode_scratch_bytes() bytes (bf16 caches with group <= 8;
+                              may be NULL otherwise): work items, per-slot logits, softmax
+                              partials and their per-row lists, per-row step counters. Owned by
+                              the caller, written by kv_decode_init, carried between steps.   */
   size_t scratch_bytes;
 } kv_cache;
 
@@ -117,7 +119,8 @@ size_t kv_workspace_bytes(const kv_shape* shape, const int32_t* L, int32_t n_seq
  * sum_h b_{l,h} = floor(budget_pct * L * H / 100) per layer), or -1. */
 int64_t kv_total_slots(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params);
 
-/* Bytes of decode scratch (kv_cache.scratch) for this batch and cache size. */
+/* Bytes of decode scratch (kv_cache.scratch) for this batch and cache size
+ * (0 when the cache is fp32 or group > 8: that path needs none). */
 size_t kv_decode_scratch_bytes(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
                                int64_t total_slots);
 
@@ -190,10 +193,10 @@ int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, con
  *   A = 0 on every slot (VoxZip defines A by the decode recursion only),
  *   meta_i = {count = b_i, next free slot = b_i, steps = 0, last evicted = -1,
  *   prefill count = b_i}, builds the decode work items (rows cut into
- *   256-slot chunks) in the scratch, and checks that every row has an evictable middle
+ *   128-slot chunks) and clears the step counters in the scratch, and checks that every row has an evictable middle
  *   once a token is appended (b_i >= T + M_i) where
  *   M_i = floor(recent_pct * b_i / 100); rows without one set KV_DEV_BUDGET.
- * Errors: KV_ERR_ARG, KV_ERR_CUDA.
+ * Errors: KV_ERR_ARG, KV_ERR_WORKSPACE (scratch missing or too small), KV_ERR_CUDA.
  */
 int kv_decode_init(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
                    kv_cache* cache, void* stream);
@@ -209,7 +212,12 @@ int kv_decode_init(const kv_shape* shape, const int32_t* L, int32_t n_seq, const
  *   evict the larger position — and its slot becomes the next free slot.
  *   q_t : device, [rows][g][d] dtype;  k_t, v_t : device, [rows][d] dtype.
  *   out : device, [rows][g][d] dtype.
- * Errors: KV_ERR_ARG, KV_ERR_CUDA.
+ * bf16 caches with g <= 8 run one persistent launch of one CTA per SM; the
+ * CTAs that share a row wait for each other (bounded: a wait that runs out
+ * sets KV_DEV_TIMEOUT, and the decode state is then undefined until
+ * kv_decode_init runs again). Steps on one stream are ordered; steps of one
+ * cache must not overlap on different streams.
+ * Errors: KV_ERR_ARG, KV_ERR_WORKSPACE, KV_ERR_CUDA.
  */
 int kv_decode_attn_update(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
                           kv_cache* cache, const void* q_t, const void* k_t, const void* v_t, void* out,
