@@ -746,6 +746,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const int nq = (E + kOutUnit - 1) / kOutUnit;
   const int r_lo = rlo_s, r_hi = rhi_s, own_lo = own_s;
   const long long S0 = rng_s[0], S1 = rng_s[1];
+  constexpr int UP = 8;  // slot pairs per lane in flight in the sweep
+  // The first round of this warp's sweep loads of logits (written by this CTA: they
+  // wait for no other CTA) goes out before the waits for the rows below.
+  float4 pf_lv[UP];
+  long long pf_s0 = -1;
+  if (G == kTcMaxG) {
+    const int rn0 = min(kRowsBatch, r_hi - r_lo + 1);
+    const long long B0 = max(S0, rowc[0].base), B1 = min(S1, rowc[rn0 - 1].base + rowc[rn0 - 1].cap);
+    const long long len = B1 > B0 ? B1 - B0 : 0;
+    const long long w0 = B0 + len * warp / kWarps, w1 = B0 + len * (warp + 1) / kWarps;
+    if (w0 < w1) {
+      int ri = 0;
+      while (ri < rn0 - 1 && w0 >= rowc[ri].base + rowc[ri].cap) ++ri;
+      const long long p1 = min(w1, rowc[ri].base + rowc[ri].cap);
+      const int half = lane & 1, sl = lane >> 1;
+#pragma unroll
+      for (int uu = 0; uu < UP; ++uu) {
+        const long long sx = min(w0 + uu * 16 + sl, p1 - 1);
+        pf_lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + sx * kTcMaxG) + half);
+      }
+      pf_s0 = w0;
+    }
+  }
   for (int rb = r_lo; rb <= r_hi; rb += kRowsBatch) {
     const int rn = min(kRowsBatch, r_hi - rb + 1);
     RowC* rc = rb == r_lo ? rowc : rcb;
@@ -855,7 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (G == kTcMaxG) {
           // lane pairs share a slot: each lane loads 4 of its 8 logits, so a warp's
           // request is 512 contiguous bytes
-          constexpr int U = 8;  // slot pairs per lane in flight
+          constexpr int U = UP;
           const int half = lane & 1, sl = lane >> 1;
           float lh[4];
 #pragma unroll
@@ -864,13 +887,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             float4 lv[U];
             float Av[U];
             int pv[U];
+            const bool pf = s0 == pf_s0;  // logits loaded ahead (same clamped addresses)
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
               const long long s = min(s0 + uu * 16 + sl, p1 - 1);
-              lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
+              lv[uu] = pf ? pf_lv[uu] : __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
               Av[uu] = __ldcg(a.A + s);
               pv[uu] = __ldcg(a.pos + s);
             }
+            if (pf) pf_s0 = -1;
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {
               float ps = ex2_approx(lv[uu].x - lh[0]) + ex2_approx(lv[uu].y - lh[1]) + ex2_approx(lv[uu].z - lh[2]) +
