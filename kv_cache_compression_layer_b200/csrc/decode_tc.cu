@@ -47,7 +47,7 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kQBytes = kTcMaxG * 128 * 2;      // staged query rows per stage (d <= 128): two 8-row boxes
 constexpr int kPartO = 2 * kTcMaxG;             // offset of O in a partial (16-byte aligned)
 constexpr int kOutUnit = 256;                   // output elements per output unit
-constexpr int kRowsBatch = 64;                  // row constants held at once by a CTA's finish
+constexpr int kRowsBatch = 32;                  // row constants held at once by a CTA's finish
 
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int slot, int dcol) {
   const int box = dcol >> 6, chunk = (dcol & 63) >> 3;
@@ -95,9 +95,8 @@ struct TcScratch {
   float* part;     // [max_items * kGroups][stride]: max[G] at 0, sum[G] at G, O[G][d] at kPartO,
                    // per (first item of a group's segment, group)
   float* logits;   // [total_slots][G] logits in log2 units
-  int* plist_n;    // [2][rows] partials listed for the row in its steps of even / odd number;
-                   // the row's finish clears the counter of the row's next step
-  int* plist;      // [rows][max_per_row * kGroups] list entries (PEnt: per-head max and sum, index)
+  int* plist;      // [rows][max_per_row * kGroups] list entries (PEnt: per-head max and sum, index,
+                   // step stamp), one place per (item that starts a group's segment, group)
   int* done;       // [rows] slots of the row finished in the current step
   int* best_n;     // [rows] eviction proposals of the row in the current step
   int4* bests;     // [rows][max_bests] proposals (A bits, pos, slot, -)
@@ -135,8 +134,6 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
   off += al((size_t)max_items * kGroups * stride * 4);
   const size_t o_log = off;
   off += al((size_t)total_slots * G * 4);
-  const size_t o_pn = off;
-  off += al((size_t)rows * 2 * 4);
   const size_t o_pl = off;
   off += al((size_t)rows * per_row * kGroups * 80);
   const size_t o_done = off;
@@ -153,7 +150,6 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
     sc->items = reinterpret_cast<int2*>(base + o_items);
     sc->part = reinterpret_cast<float*>(base + o_part);
     sc->logits = reinterpret_cast<float*>(base + o_log);
-    sc->plist_n = reinterpret_cast<int*>(base + o_pn);
     sc->plist = reinterpret_cast<int*>(base + o_pl);
     sc->done = reinterpret_cast<int*>(base + o_done);
     sc->best_n = reinterpret_cast<int*>(base + o_bn);
@@ -199,8 +195,6 @@ __global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off
     for (int k = 0; k < warp; ++k) wb += warp_tot[k];
     const int incl = carry + wb + v;
     if (i < n_rows) {
-      sc.plist_n[i] = 0;
-      sc.plist_n[n_rows + i] = 0;
       sc.done[i] = 0;
       sc.best_n[i] = 0;
       sc.attn_done[i] = 0;
@@ -327,22 +321,26 @@ __device__ __forceinline__ void issue_tile(const Walk& w, uint8_t* stage, uint64
 struct PEnt {
   float m[kTcMaxG];
   float l[kTcMaxG];
-  int pidx, pad0, pad1, pad2;
+  int pidx, stamp, pad1, pad2;  // stamp: the row's step number + 1 when written
 };
 static_assert(sizeof(PEnt) == 80, "list entry layout");
 
-__device__ __forceinline__ void ld_pent(const PEnt* e, float (&m)[kTcMaxG], float (&l)[kTcMaxG], int& pidx) {
+__device__ __forceinline__ void ld_pent(const PEnt* e, float (&m)[kTcMaxG], float (&l)[kTcMaxG], int& pidx,
+                                        int& stamp) {
   const float4* v = reinterpret_cast<const float4*>(e);
   const float4 a0 = __ldcg(v), a1 = __ldcg(v + 1), b0 = __ldcg(v + 2), b1 = __ldcg(v + 3);
-  pidx = __ldcg(reinterpret_cast<const int*>(v + 4));
+  const int2 ps = __ldcg(reinterpret_cast<const int2*>(v + 4));
+  pidx = ps.x;
+  stamp = ps.y;
   m[0] = a0.x; m[1] = a0.y; m[2] = a0.z; m[3] = a0.w; m[4] = a1.x; m[5] = a1.y; m[6] = a1.z; m[7] = a1.w;
   l[0] = b0.x; l[1] = b0.y; l[2] = b0.z; l[3] = b0.w; l[4] = b1.x; l[5] = b1.y; l[6] = b1.z; l[7] = b1.w;
 }
 
 // A row's softmax statistics for the finish (in the freed tile ring).
+constexpr int kStatParts = 64;  // partials of a row held on chip by the finish (more: read again)
 struct RowStat {
-  int pidx[32];                // the row's first 32 partial indices
-  float pm[32][kTcMaxG];       // their maxima
+  int pidx[kStatParts];              // the row's first partials' indices
+  float pm[kStatParts][kTcMaxG];     // their maxima
   float M[kTcMaxG], Li[kTcMaxG], lse[kTcMaxG];
   int nr;                      // partials listed (capped at the list size)
 };
@@ -355,38 +353,51 @@ struct RowC {
 };
 
 // The row's softmax statistics per query head, merged by one warp from the
-// list of partials of this step: M_g, 1/L_g and lse_g = M_g + log2 L_g into
-// ws, with the first 32 partials' indices and maxima. The list entries carry
-// each partial's (max, sum), so this is one round of loads.
-__device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, int lane, RowStat& ws, int& nr_out,
-                                          int& nr_all_out) {
+// partials this step listed for the row: the list has a place per (item,
+// group) of the row's ncand places, and the places written this step carry
+// the step's stamp. M_g, 1/L_g and lse_g = M_g + log2 L_g go to ws with the
+// first kStatParts partials' indices and maxima (ws.nr = all partials found).
+// The entries carry each partial's (max, sum): one round of loads.
+__device__ __forceinline__ void row_stats(const TcArgs& P, int row, int ncand, int stamp, int lane, RowStat& ws) {
   const DecArgs& a = P.a;
   const TcScratch& sc = P.sc;
   const int G = a.G;
   const int maxp = sc.max_per_row * kGroups;
   const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
-  const int nr_all = __ldcg(sc.plist_n + lbuf * a.map.n_rows + row);
-  float em[kTcMaxG], el[kTcMaxG];
-  int ep = 0;
-  if (lane < maxp) ld_pent(lst + lane, em, el, ep);  // ahead of the count; unused past it
-  const int nr = min(nr_all, maxp);
+  ncand = min(ncand, maxp);
   float m[kTcMaxG], l[kTcMaxG];
 #pragma unroll
   for (int g = 0; g < kTcMaxG; ++g) {
     m[g] = -INFINITY;
     l[g] = 0.f;
   }
-  for (int k = lane; k < nr; k += 32) {
-    if (k >= 32) ld_pent(lst + k, em, el, ep);
-    if (k < 32) ws.pidx[k] = ep;
+  int found = 0;  // partials found so far (warp-uniform)
+  for (int k0 = 0; k0 < ncand; k0 += 64) {
+    // two places per lane per round, both loads in flight together
+    float em0[kTcMaxG], el0[kTcMaxG], em1[kTcMaxG], el1[kTcMaxG];
+    int ep0 = 0, es0 = 0, ep1 = 0, es1 = 0;
+    const int k_a = k0 + lane, k_b = k0 + 32 + lane;
+    if (k_a < ncand) ld_pent(lst + k_a, em0, el0, ep0, es0);
+    if (k_b < ncand) ld_pent(lst + k_b, em1, el1, ep1, es1);
 #pragma unroll
-    for (int g = 0; g < kTcMaxG; ++g) {
-      if (g < G) {
-        if (k < 32) ws.pm[k][g] = em[g];
-        if (em[g] > -INFINITY) {
-          const float mn = fmaxf(m[g], em[g]);
-          l[g] = l[g] * ex2_approx(m[g] - mn) + el[g] * ex2_approx(em[g] - mn);
-          m[g] = mn;
+    for (int hh = 0; hh < 2; ++hh) {
+      const bool valid = (hh ? k_b : k_a) < ncand && (hh ? es1 : es0) == stamp;
+      const unsigned bal = __ballot_sync(0xffffffffu, valid);
+      const int idx = found + __popc(bal & ((1u << lane) - 1));
+      found += __popc(bal);
+      if (valid) {
+        if (idx < kStatParts) ws.pidx[idx] = hh ? ep1 : ep0;
+#pragma unroll
+        for (int g = 0; g < kTcMaxG; ++g) {
+          if (g < G) {
+            const float mk = hh ? em1[g] : em0[g], lk = hh ? el1[g] : el0[g];
+            if (idx < kStatParts) ws.pm[idx][g] = mk;
+            if (mk > -INFINITY) {
+              const float mn = fmaxf(m[g], mk);
+              l[g] = l[g] * ex2_approx(m[g] - mn) + lk * ex2_approx(mk - mn);
+              m[g] = mn;
+            }
+          }
         }
       }
     }
@@ -405,10 +416,8 @@ __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int lbuf, in
       ws.lse[g] = M + log2f(L);
     }
   }
-  if (lane == 0) ws.nr = nr;
+  if (lane == 0) ws.nr = found;
   __syncwarp();
-  nr_out = nr;
-  nr_all_out = nr_all;
 }
 
 // Step constants of `row` except its log-denominators (they need the step's
@@ -469,14 +478,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __shared__ long long rng_s[2];      // the finish range [S0, S1) of slots
   __shared__ int rlo_s, rhi_s;        // its first and last row
   __shared__ int own_s;               // first row whose attention output this CTA writes
-  __shared__ int kk_s[kGroups];       // list position of a group's partial
-  __shared__ int segc_s[kGroups], segs_s[kGroups];  // a group's segment: slots attended, row's step
+  // a group's current segment: slots attended, the row's step, the segment's first item in the row
+  __shared__ int segc_s[kGroups], segs_s[kGroups], segk_s[kGroups];
+  // a group's finished segments whose slot counts are published together at the end
+  constexpr int kDefer = 16;
+  __shared__ int dq_row[kGroups][kDefer], dq_cnt[kGroups][kDefer], dq_n[kGroups];
   __shared__ Walk walk_s[kGroups];  // each group's tile walk (its first thread's), kept out of registers
   __shared__ int more_s[kGroups], ended_s[kGroups], nreal_s[kGroups];
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
     abort_s = 0;
+    for (int g = 0; g < kGroups; ++g) dq_n[g] = 0;
     fence_barrier_init();
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -576,11 +589,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               atomicAdd(&og[g0 * D + ogswz(g0, col + 1)], o[i][1] * f0);
             }
           }
-          if (gt == 0) kk_s[grp] = atomicAdd(&sc.plist_n[(segs_s[grp] & 1) * n_rows + cur_row], 1);
           named_bar_sync(1 + grp, 128);
           const int pidx = seg_u * kGroups + grp;
           float* part = sc.part + (long long)pidx * sc.stride;
-          const int kk = kk_s[grp];
+          // the row's list place of this partial: (the segment's first item in the row, group)
+          const int kk = segk_s[grp] * kGroups + grp;
           PEnt* ent = reinterpret_cast<PEnt*>(sc.plist) + (long long)cur_row * maxp + kk;
           if (gt < G) {
             float M = -INFINITY;
@@ -596,16 +609,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               ent->l[gt] = Ls;
             }
           }
-          if (gt == 0 && kk < maxp) ent->pidx = pidx;
+          if (gt == 0 && kk < maxp) {
+            ent->pidx = pidx;
+            ent->stamp = segs_s[grp] + 1;
+          }
           for (int i = gt; i < G * D; i += 128) {
             const int og_i = (i / D) * D + ogswz(i / D, i % D);
             part[kPartO + i] = og[og_i];
             og[og_i] = 0.f;
           }
           named_bar_sync(1 + grp, 128);
-          if (gt == 0) {  // the partial is published: count the slots it covers
-            __threadfence();
-            atomicAdd(&sc.attn_done[cur_row], (unsigned)segc_s[grp]);
+          if (gt == 0) {  // count the slots the partial covers, once it is visible (at the end)
+            const int qn = dq_n[grp];
+            if (qn < kDefer) {
+              dq_row[grp][qn] = cur_row;
+              dq_cnt[grp][qn] = segc_s[grp];
+              dq_n[grp] = qn + 1;
+            } else {
+              __threadfence();
+              atomicAdd(&sc.attn_done[cur_row], (unsigned)segc_s[grp]);
+            }
           }
           m0 = -INFINITY;
           l0 = 0.f;
@@ -618,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (gt == 0) {
           segs_s[grp] = hdr[stg].steps;
           segc_s[grp] = 0;
+          segk_s[grp] = hdr[stg].st0 / kCH;
         }
       }
       const TileHdr h = hdr[stg];
@@ -726,6 +750,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
       }
     }
+    if (gt == 0 && dq_n[grp] > 0) {  // publish the group's partials, then their slot counts
+      __threadfence();
+      for (int i = 0; i < dq_n[grp]; ++i) atomicAdd(&sc.attn_done[dq_row[grp][i]], (unsigned)dq_cnt[grp][i]);
+    }
     if (aborted) {
       abort_s = 1;
       if (gt == 0)  // let this group's copies in flight land before the CTA exits
@@ -747,28 +775,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const int r_lo = rlo_s, r_hi = rhi_s, own_lo = own_s;
   const long long S0 = rng_s[0], S1 = rng_s[1];
   constexpr int UP = 8;  // slot pairs per lane in flight in the sweep
-  // The first round of this warp's sweep loads of logits (written by this CTA: they
-  // wait for no other CTA) goes out before the waits for the rows below.
-  float4 pf_lv[UP];
-  long long pf_s0 = -1;
-  if (G == kTcMaxG) {
-    const int rn0 = min(kRowsBatch, r_hi - r_lo + 1);
-    const long long B0 = max(S0, rowc[0].base), B1 = min(S1, rowc[rn0 - 1].base + rowc[rn0 - 1].cap);
-    const long long len = B1 > B0 ? B1 - B0 : 0;
-    const long long w0 = B0 + len * warp / kWarps, w1 = B0 + len * (warp + 1) / kWarps;
-    if (w0 < w1) {
-      int ri = 0;
-      while (ri < rn0 - 1 && w0 >= rowc[ri].base + rowc[ri].cap) ++ri;
-      const long long p1 = min(w1, rowc[ri].base + rowc[ri].cap);
-      const int half = lane & 1, sl = lane >> 1;
-#pragma unroll
-      for (int uu = 0; uu < UP; ++uu) {
-        const long long sx = min(w0 + uu * 16 + sl, p1 - 1);
-        pf_lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + sx * kTcMaxG) + half);
-      }
-      pf_s0 = w0;
-    }
-  }
   for (int rb = r_lo; rb <= r_hi; rb += kRowsBatch) {
     const int rn = min(kRowsBatch, r_hi - rb + 1);
     RowC* rc = rb == r_lo ? rowc : rcb;
@@ -795,10 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
       waited = __shfl_sync(0xffffffffu, waited, 0);
       if (!waited) abort_s = 1;
-      int nr, nr_all;
-      row_stats(P, row, rc[i].steps & 1, lane, rs[i], nr, nr_all);
-      if (lane == 0 && nr_all > sc.max_per_row * kGroups) rc[i].flags |= 4;
-      __syncwarp();
+      row_stats(P, row, ((rc[i].cap + kCH - 1) / kCH) * kGroups, rc[i].steps + 1, lane, rs[i]);
     }
     __syncthreads();
     if (abort_s) return;
@@ -819,6 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const int g0 = ok0 ? e0 / D : 0, g1 = ok1 ? e1 / D : 0;
       const float M0 = st.M[g0], M1 = st.M[g1];
       const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
+      const int stamp = rc[i].steps + 1, ncand = min(((rc[i].cap + kCH - 1) / kCH) * kGroups, maxp);
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       auto add = [&](int pi, float mk0, float mk1) {
         const float* pc = sc.part + (long long)pi * sc.stride + kPartO;
@@ -835,10 +839,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         acc[6] += w1 * v1.z;
         acc[7] += w1 * v1.w;
       };
-      const int n32 = min(nr, 32);
+      if (nr <= kStatParts) {
 #pragma unroll 8
-      for (int kp = 0; kp < n32; ++kp) add(st.pidx[kp], st.pm[kp][g0], st.pm[kp][g1]);
-      for (int kp = 32; kp < nr; ++kp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g0]), __ldcg(&lst[kp].m[g1]));
+        for (int kp = 0; kp < nr; ++kp) add(st.pidx[kp], st.pm[kp][g0], st.pm[kp][g1]);
+      } else {  // more partials than held on chip: read every place again
+        for (int kp = 0; kp < ncand; ++kp)
+          if (__ldcg(&lst[kp].stamp) == stamp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g0]), __ldcg(&lst[kp].m[g1]));
+      }
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (long long)row * E;
       if (ok0) {
         const float li = st.Li[g0];
@@ -887,15 +894,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             float4 lv[U];
             float Av[U];
             int pv[U];
-            const bool pf = s0 == pf_s0;  // logits loaded ahead (same clamped addresses)
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
               const long long s = min(s0 + uu * 16 + sl, p1 - 1);
-              lv[uu] = pf ? pf_lv[uu] : __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
+              lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
               Av[uu] = __ldcg(a.A + s);
               pv[uu] = __ldcg(a.pos + s);
             }
-            if (pf) pf_s0 = -1;
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {
               float ps = ex2_approx(lv[uu].x - lh[0]) + ex2_approx(lv[uu].y - lh[1]) + ex2_approx(lv[uu].z - lh[2]) +
@@ -1006,7 +1011,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           }
           sc.done[row] = 0;
           sc.best_n[row] = 0;
-          sc.plist_n[((R.steps + 1) & 1) * n_rows + row] = 0;  // the row's next step lists its partials there
         }
       }
       p0 = p1;
@@ -1026,6 +1030,9 @@ int launch_tc_init(const kv_shape& sh, const RowMap& m, int capb, long long tota
   TcScratch sc;
   const size_t need = tc_layout(m.n_rows, sh.group, sh.head_dim, capb, total_slots, (char*)c.scratch, &sc);
   if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
+  // list entries carry the step they belong to: clear the stamps of any earlier decode
+  if (cudaMemsetAsync(sc.plist, 0, (size_t)m.n_rows * sc.max_per_row * kGroups * sizeof(PEnt), st) != cudaSuccess)
+    return KV_ERR_CUDA;
   tc_items_kernel<<<1, 1024, 0, st>>>(m.n_rows, c.slot_off, sc, c.status);
   return cuda_status(cudaGetLastError());
 }
