@@ -85,6 +85,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Scratch of the tensor-core path inside kv_cache.scratch.
@@ -402,19 +409,30 @@ __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int ncand, i
       }
     }
   }
+  float M[kTcMaxG], L[kTcMaxG];
 #pragma unroll
-  for (int g = 0; g < kTcMaxG; ++g) {
-    float M = m[g];
+  for (int g = 0; g < kTcMaxG; ++g) M[g] = m[g];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = m[g] > -INFINITY ? l[g] * ex2_approx(m[g] - M) : 0.f;
+  for (int off = 16; off > 0; off >>= 1)  // all heads at once: independent shuffle chains
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    if (lane == 0 && g < G) {
-      ws.M[g] = M;
-      ws.Li[g] = L > 0.f ? 1.f / L : 0.f;
-      ws.lse[g] = M + log2f(L);
-    }
+    for (int g = 0; g < kTcMaxG; ++g) M[g] = fmaxf(M[g], __shfl_xor_sync(0xffffffffu, M[g], off));
+#pragma unroll
+  for (int g = 0; g < kTcMaxG; ++g) L[g] = m[g] > -INFINITY ? l[g] * ex2_approx(m[g] - M[g]) : 0.f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int g = 0; g < kTcMaxG; ++g) L[g] += __shfl_xor_sync(0xffffffffu, L[g], off);
+  if (lane < G) {  // lane g publishes head g
+    float Mg = M[0], Lg = L[0];
+#pragma unroll
+    for (int g = 1; g < kTcMaxG; ++g)
+      if (lane == g) {
+        Mg = M[g];
+        Lg = L[g];
+      }
+    ws.M[lane] = Mg;
+    ws.Li[lane] = Lg > 0.f ? 1.f / Lg : 0.f;
+    ws.lse[lane] = Mg + log2f(Lg);
   }
   if (lane == 0) ws.nr = found;
   __syncwarp();
@@ -775,6 +793,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const int r_lo = rlo_s, r_hi = rhi_s, own_lo = own_s;
   const long long S0 = rng_s[0], S1 = rng_s[1];
   constexpr int UP = 8;  // slot pairs per lane in flight in the sweep
+  // The first batch's slot data (logits written by this CTA, A, positions: none of it
+  // waits for another CTA) is copied into the rest of the freed ring now, without
+  // waiting; the sweep reads it from there.
+  constexpr size_t kStgOff = (size_t)kRowsBatch * (sizeof(RowStat) + sizeof(RowC));
+  constexpr int kStgSlots = (int)(((size_t)kStages * STAGE - kStgOff) / 40);
+  static_assert(kStgOff % 16 == 0, "staging alignment");
+  float* st_lg = reinterpret_cast<float*>(ring + kStgOff);  // [kStgSlots][8]
+  float* st_A = st_lg + (size_t)kStgSlots * kTcMaxG;        // [kStgSlots]
+  int* st_pos = reinterpret_cast<int*>(st_A + kStgSlots);    // [kStgSlots]
+  long long stg0 = 0;
+  int nst = 0;
+  if (G == kTcMaxG) {
+    const int rn0 = min(kRowsBatch, r_hi - r_lo + 1);
+    stg0 = max(S0, rowc[0].base);
+    const long long stg1 = min(S1, rowc[rn0 - 1].base + rowc[rn0 - 1].cap);
+    nst = (int)max(0ll, min(stg1 - stg0, (long long)kStgSlots));
+    const float* lsrc = sc.logits + stg0 * kTcMaxG;
+    for (int i = tid; i < nst * 2; i += kThreads) cp_async16(st_lg + i * 4, lsrc + i * 4);
+    for (int i = tid; i < nst; i += kThreads) {
+      cp_async4(st_A + i, a.A + stg0 + i);
+      cp_async4(st_pos + i, a.pos + stg0 + i);
+    }
+  }
   for (int rb = r_lo; rb <= r_hi; rb += kRowsBatch) {
     const int rn = min(kRowsBatch, r_hi - rb + 1);
     RowC* rc = rb == r_lo ? rowc : rcb;
@@ -803,67 +844,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (!waited) abort_s = 1;
       row_stats(P, row, ((rc[i].cap + kCH - 1) / kCH) * kGroups, rc[i].steps + 1, lane, rs[i]);
     }
-    __syncthreads();
+    cp_async_wait_all();  // this thread's copies into the staging area
+    __syncthreads();      // ... and everyone else's
     if (abort_s) return;
 
-    // (2) attention outputs of the rows whose first item is in this range: units of
-    // kOutUnit elements over the warps, from the last warp down
-    const int o_first = max(rb, own_lo) - rb;
-    const int n_units = max(0, rn - o_first) * nq;
-    for (int un = kWarps - 1 - warp; un < n_units; un += kWarps) {
-      const int i = o_first + un / nq, q = un % nq;
-      const int row = rb + i;
-      const RowStat& st = rs[i];
-      const int nr = st.nr;
-      // lane: elements e0..e0+3 and e0+128..e0+131 of the unit, so each of the warp's
-      // two loads per partial is 512 contiguous bytes
-      const int e0 = q * kOutUnit + lane * 4, e1 = e0 + kOutUnit / 2;
-      const bool ok0 = e0 < E, ok1 = e1 < E;
-      const int g0 = ok0 ? e0 / D : 0, g1 = ok1 ? e1 / D : 0;
-      const float M0 = st.M[g0], M1 = st.M[g1];
-      const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
-      const int stamp = rc[i].steps + 1, ncand = min(((rc[i].cap + kCH - 1) / kCH) * kGroups, maxp);
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      auto add = [&](int pi, float mk0, float mk1) {
-        const float* pc = sc.part + (long long)pi * sc.stride + kPartO;
-        const float4 v0 = ok0 ? __ldcg(reinterpret_cast<const float4*>(pc + e0)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 v1 = ok1 ? __ldcg(reinterpret_cast<const float4*>(pc + e1)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float w0 = mk0 > -INFINITY ? ex2_approx(mk0 - M0) : 0.f;
-        const float w1 = mk1 > -INFINITY ? ex2_approx(mk1 - M1) : 0.f;
-        acc[0] += w0 * v0.x;
-        acc[1] += w0 * v0.y;
-        acc[2] += w0 * v0.z;
-        acc[3] += w0 * v0.w;
-        acc[4] += w1 * v1.x;
-        acc[5] += w1 * v1.y;
-        acc[6] += w1 * v1.z;
-        acc[7] += w1 * v1.w;
-      };
-      if (nr <= kStatParts) {
-#pragma unroll 8
-        for (int kp = 0; kp < nr; ++kp) add(st.pidx[kp], st.pm[kp][g0], st.pm[kp][g1]);
-      } else {  // more partials than held on chip: read every place again
-        for (int kp = 0; kp < ncand; ++kp)
-          if (__ldcg(&lst[kp].stamp) == stamp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g0]), __ldcg(&lst[kp].m[g1]));
-      }
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (long long)row * E;
-      if (ok0) {
-        const float li = st.Li[g0];
-        uint2 pk;
-        pk.x = pack_bf16(acc[0] * li, acc[1] * li);
-        pk.y = pack_bf16(acc[2] * li, acc[3] * li);
-        *reinterpret_cast<uint2*>(orow + e0) = pk;
-      }
-      if (ok1) {
-        const float li = st.Li[g1];
-        uint2 pk;
-        pk.x = pack_bf16(acc[4] * li, acc[5] * li);
-        pk.y = pack_bf16(acc[6] * li, acc[7] * li);
-        *reinterpret_cast<uint2*>(orow + e1) = pk;
-      }
-    }
-
-    // (3) decayed scores and evictions: this warp's share of the batch's slots within the range
+    // (2) decayed scores and evictions first: this warp's share of the batch's slots within the range
     const long long B0 = max(S0, rc[0].base), B1 = min(S1, rc[rn - 1].base + rc[rn - 1].cap);
     const long long len = B1 > B0 ? B1 - B0 : 0;
     const long long w0 = B0 + len * warp / kWarps, w1 = B0 + len * (warp + 1) / kWarps;
@@ -894,12 +879,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             float4 lv[U];
             float Av[U];
             int pv[U];
+            if (s0 >= stg0 && min(s0 + 16 * U, p1) <= stg0 + nst) {  // staged in shared memory
 #pragma unroll
-            for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
-              const long long s = min(s0 + uu * 16 + sl, p1 - 1);
-              lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
-              Av[uu] = __ldcg(a.A + s);
-              pv[uu] = __ldcg(a.pos + s);
+              for (int uu = 0; uu < U; ++uu) {
+                const int k = (int)(min(s0 + uu * 16 + sl, p1 - 1) - stg0);
+                lv[uu] = *reinterpret_cast<const float4*>(st_lg + k * kTcMaxG + half * 4);
+                Av[uu] = st_A[k];
+                pv[uu] = st_pos[k];
+              }
+            } else {
+#pragma unroll
+              for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
+                const long long s = min(s0 + uu * 16 + sl, p1 - 1);
+                lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
+                Av[uu] = __ldcg(a.A + s);
+                pv[uu] = __ldcg(a.pos + s);
+              }
             }
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {
@@ -1015,6 +1010,64 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
       p0 = p1;
     }
+    // (3) attention outputs of the rows whose first item is in this range: units of
+    // kOutUnit elements over the warps, from the last warp down (after the sweep: the
+    // next step waits for the evictions, not for the outputs)
+    const int o_first = max(rb, own_lo) - rb;
+    const int n_units = max(0, rn - o_first) * nq;
+    for (int un = kWarps - 1 - warp; un < n_units; un += kWarps) {
+      const int i = o_first + un / nq, q = un % nq;
+      const int row = rb + i;
+      const RowStat& st = rs[i];
+      const int nr = st.nr;
+      // lane: elements e0..e0+3 and e0+128..e0+131 of the unit, so each of the warp's
+      // two loads per partial is 512 contiguous bytes
+      const int e0 = q * kOutUnit + lane * 4, e1 = e0 + kOutUnit / 2;
+      const bool ok0 = e0 < E, ok1 = e1 < E;
+      const int g0 = ok0 ? e0 / D : 0, g1 = ok1 ? e1 / D : 0;
+      const float M0 = st.M[g0], M1 = st.M[g1];
+      const PEnt* lst = reinterpret_cast<const PEnt*>(sc.plist) + (long long)row * maxp;
+      const int stamp = rc[i].steps + 1, ncand = min(((rc[i].cap + kCH - 1) / kCH) * kGroups, maxp);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      auto add = [&](int pi, float mk0, float mk1) {
+        const float* pc = sc.part + (long long)pi * sc.stride + kPartO;
+        const float4 v0 = ok0 ? __ldcg(reinterpret_cast<const float4*>(pc + e0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v1 = ok1 ? __ldcg(reinterpret_cast<const float4*>(pc + e1)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float w0 = mk0 > -INFINITY ? ex2_approx(mk0 - M0) : 0.f;
+        const float w1 = mk1 > -INFINITY ? ex2_approx(mk1 - M1) : 0.f;
+        acc[0] += w0 * v0.x;
+        acc[1] += w0 * v0.y;
+        acc[2] += w0 * v0.z;
+        acc[3] += w0 * v0.w;
+        acc[4] += w1 * v1.x;
+        acc[5] += w1 * v1.y;
+        acc[6] += w1 * v1.z;
+        acc[7] += w1 * v1.w;
+      };
+      if (nr <= kStatParts) {
+#pragma unroll 8
+        for (int kp = 0; kp < nr; ++kp) add(st.pidx[kp], st.pm[kp][g0], st.pm[kp][g1]);
+      } else {  // more partials than held on chip: read every place again
+        for (int kp = 0; kp < ncand; ++kp)
+          if (__ldcg(&lst[kp].stamp) == stamp) add(__ldcg(&lst[kp].pidx), __ldcg(&lst[kp].m[g0]), __ldcg(&lst[kp].m[g1]));
+      }
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (long long)row * E;
+      if (ok0) {
+        const float li = st.Li[g0];
+        uint2 pk;
+        pk.x = pack_bf16(acc[0] * li, acc[1] * li);
+        pk.y = pack_bf16(acc[2] * li, acc[3] * li);
+        *reinterpret_cast<uint2*>(orow + e0) = pk;
+      }
+      if (ok1) {
+        const float li = st.Li[g1];
+        uint2 pk;
+        pk.x = pack_bf16(acc[4] * li, acc[5] * li);
+        pk.y = pack_bf16(acc[6] * li, acc[7] * li);
+        *reinterpret_cast<uint2*>(orow + e1) = pk;
+      }
+    }
+
     __syncthreads();  // the row statistics and constants are rewritten by the next batch
   }
 }
