@@ -379,25 +379,29 @@ __device__ __forceinline__ void row_stats(const TcArgs& P, int row, int ncand, i
     l[g] = 0.f;
   }
   int found = 0;  // partials found so far (warp-uniform)
-  for (int k0 = 0; k0 < ncand; k0 += 64) {
-    // two places per lane per round, both loads in flight together
-    float em0[kTcMaxG], el0[kTcMaxG], em1[kTcMaxG], el1[kTcMaxG];
-    int ep0 = 0, es0 = 0, ep1 = 0, es1 = 0;
-    const int k_a = k0 + lane, k_b = k0 + 32 + lane;
-    if (k_a < ncand) ld_pent(lst + k_a, em0, el0, ep0, es0);
-    if (k_b < ncand) ld_pent(lst + k_b, em1, el1, ep1, es1);
+  constexpr int kPer = 3;  // places per lane per round, all loads in flight together
+  for (int k0 = 0; k0 < ncand; k0 += 32 * kPer) {
+    float em[kPer][kTcMaxG], el[kPer][kTcMaxG];
+    int ep[kPer], es[kPer];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const bool valid = (hh ? k_b : k_a) < ncand && (hh ? es1 : es0) == stamp;
+    for (int h = 0; h < kPer; ++h) {
+      es[h] = 0;
+      ep[h] = 0;
+      const int k = k0 + h * 32 + lane;
+      if (k < ncand) ld_pent(lst + k, em[h], el[h], ep[h], es[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < kPer; ++h) {
+      const bool valid = k0 + h * 32 + lane < ncand && es[h] == stamp;
       const unsigned bal = __ballot_sync(0xffffffffu, valid);
       const int idx = found + __popc(bal & ((1u << lane) - 1));
       found += __popc(bal);
       if (valid) {
-        if (idx < kStatParts) ws.pidx[idx] = hh ? ep1 : ep0;
+        if (idx < kStatParts) ws.pidx[idx] = ep[h];
 #pragma unroll
         for (int g = 0; g < kTcMaxG; ++g) {
           if (g < G) {
-            const float mk = hh ? em1[g] : em0[g], lk = hh ? el1[g] : el0[g];
+            const float mk = em[h][g], lk = el[h][g];
             if (idx < kStatParts) ws.pm[idx][g] = mk;
             if (mk > -INFINITY) {
               const float mn = fmaxf(m[g], mk);
