@@ -37,9 +37,9 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one decode_tc_kernel launch from an ncu capture
 # of this benchmark's workload (profiles/decode_tc_kernel_3b.md), valid while the
 # kernel source is the one captured (its SHA-256 below); otherwise null.
-NCU_TRAFFIC = {"3b": {"bytes": 139552512,
+NCU_TRAFFIC = {"3b": {"bytes": 139687936,
                       "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
-                      "sha256": "2787872249ee34b5"}}
+                      "sha256": "be8e7848ab7534c7"}}
 
 
 def measured_traffic(cfg_name: str):
@@ -349,7 +349,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="3b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-rows", type=int, default=64, help="rows of the oracle sample for cpu_baseline")
+    ap.add_argument("--cpu-rows", type=int, default=1 << 20,
+                    help="rows of the oracle sample for cpu_baseline (default: the whole batch)")
     ap.add_argument("--ref-rows", type=int, default=8, help="rows per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
