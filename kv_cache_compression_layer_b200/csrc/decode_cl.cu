@@ -31,7 +31,8 @@ struct ClArgs {
   DecArgs a;
   int C;         // CTAs per row (cluster size)
   int S;         // slots per CTA (a multiple of 64)
-  int ncols;     // tensor-memory columns per CTA (power of two >= 4 S / 64)
+  int cpg;       // tensor-memory columns per group (a multiple of 32): 4 per tile of the group
+  int ncols;     // tensor-memory columns per CTA (a power of two >= 3 cpg)
   unsigned long long limit_ns;
 };
 
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cl_kernel(const __grid_con
       const bool valid = row_ok && j < n && j < hi;
       x[e] = valid ? x[e] * a.scale2 : -INFINITY;
     }
-    // the logits stay on chip: this thread's lane, columns 4 t .. 4 t + 3
-    tmem_st4(tmem + ((uint32_t)(wq * 32) << 16) + 4 * t, x[0], x[1], x[2], x[3]);
+    // the logits stay on chip: this thread's lane, the group's columns 4 k .. 4 k + 3
+    tmem_st4(tmem + ((uint32_t)(wq * 32) << 16) + grp * P.cpg + 4 * k, x[0], x[1], x[2], x[3]);
     // online softmax update of this warp's running (max, sum, O)
     float tm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
@@ -396,15 +397,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cl_kernel(const __grid_con
   {
     const float lse_g = g_ok ? flse[g0] : 0.f;
     const bool upd = !skip && row_ok;
-    for (int kk = 0;; ++kk) {
-      const int t = grp + kGroups * kk;
-      if (t >= ntiles) break;
-      float xv[4];
-      tmem_ld4(tmem + ((uint32_t)(wq * 32) << 16) + 4 * t, xv);
+    const int nk = ntiles > grp ? (ntiles - grp + kGroups - 1) / kGroups : 0;  // this group's tiles
+    for (int k0 = 0; k0 < nk; k0 += 8) {
+      float xs[32];  // eight tiles' logits in one load
+      tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + grp * P.cpg + 4 * k0, xs);
       tc_wait_ld();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+      if (k0 + kk >= nk) break;
+      const int t = grp + kGroups * (k0 + kk);
       float ps[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) ps[e] = g_ok ? ex2_approx(xv[e] - lse_g) : 0.f;
+      for (int e = 0; e < 4; ++e) ps[e] = g_ok ? ex2_approx(xs[4 * kk + e] - lse_g) : 0.f;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1)  // sum over the query heads (lanes with the same q4)
 #pragma unroll
@@ -424,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cl_kernel(const __grid_con
             }
           }
         }
+      }
       }
     }
   }
@@ -487,7 +492,8 @@ int cl_cluster_size(const kv_shape& sh, const RowMap& m, int capb) {
     const long long ctas = (long long)m.n_rows * C;
     if (ctas > sms || ctas * 8 < (long long)sms * 7) continue;
     const int S = ((capb + C - 1) / C + kTcSlots - 1) / kTcSlots * kTcSlots;
-    if (4 * (S / kTcSlots) > 512) return 0;
+    const int cpg = (4 * ((S / kTcSlots + kGroups - 1) / kGroups) + 31) / 32 * 32;
+    if (kGroups * cpg > 512) return 0;
     // shared memory of the finish: O, A and positions of S slots, the CTAs' weights
     const size_t fin = (size_t)kTcMaxG * sh.head_dim * 4 + (size_t)S * 8 + 8 * kTcMaxG * 4;
     const size_t ring = (size_t)kStages * (2 * kTcSlots * sh.head_dim * 2 + kQBytes);
@@ -504,8 +510,9 @@ int launch_cl(const kv_shape& sh, const RowMap& m, int capb, int C, long long to
   P.a = a;
   P.C = C;
   P.S = ((capb + C - 1) / C + kTcSlots - 1) / kTcSlots * kTcSlots;
+  P.cpg = (4 * ((P.S / kTcSlots + kGroups - 1) / kGroups) + 31) / 32 * 32;
   int cols = 32;
-  while (cols < 4 * (P.S / kTcSlots)) cols <<= 1;
+  while (cols < kGroups * P.cpg) cols <<= 1;
   P.ncols = cols;
   P.limit_ns = kWaitLimitNs;
   const int stage_bytes = 2 * kTcSlots * sh.head_dim * 2 + kQBytes;
