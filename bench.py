@@ -34,12 +34,23 @@ UNIT = "audio tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes (read + write) of one decode_tc_kernel launch from an ncu capture
-# of this benchmark's workload (profiles/decode_tc_kernel_3b.md), valid while the
+# DRAM bytes (read + write) of one decode kernel launch from an ncu capture of
+# this benchmark's workload (profiles/decode_cl_kernel_3b.md), valid while the
 # kernel source is the one captured (its SHA-256 below); otherwise null.
-NCU_TRAFFIC = {"3b": {"bytes": 139687936,
-                      "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
-                      "sha256": "be8e7848ab7534c7"}}
+NCU_TRAFFIC = {"3b": {"bytes": 139348224,
+                      "source": "kv_cache_compression_layer_b200/csrc/decode_cl.cu",
+                      "sha256": "78b5b0da77529123"}}
+
+
+def decode_kernel(cfg: synth.Config, sms: int) -> str:
+    """The decode kernel kv_decode_attn_update launches for this workload (the library's rule)."""
+    if cfg.dtype != "bf16" or cfg.group > 8:
+        return "decode_simple_kernel"
+    for C in (8, 4, 2, 1):
+        ctas = cfg.rows * C
+        if ctas <= sms and ctas * 8 >= sms * 7:
+            return "decode_cl_kernel"
+    return "decode_tc_kernel"
 
 
 def measured_traffic(cfg_name: str):
@@ -52,7 +63,7 @@ def measured_traffic(cfg_name: str):
             digest = hashlib.sha256(f.read()).hexdigest()
     except OSError:
         return None
-    return rec["bytes"] if digest.startswith(rec["sha256"]) else None
+    return rec["bytes"] if rec["bytes"] and digest.startswith(rec["sha256"]) else None
 
 
 def describe(cfg: synth.Config) -> str:
@@ -297,8 +308,8 @@ def run_ours(args, rank, world, local_rank):
                    "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
                    "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
                    "decode_bytes_alg": dec_bytes, "decode_steps": D},
-        "roofline": {"kernel": "decode_tc_kernel (kv_decode_attn_update)" if tc
-                     else "decode_simple_kernel (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
+        "roofline": {"kernel": decode_kernel(cfg, torch.cuda.get_device_properties(dev).multi_processor_count)
+                     + " (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": measured_traffic(args.config) if tc else None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},
         "e2e": {"value": job_throughput(tokens, world, e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
