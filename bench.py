@@ -35,8 +35,8 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (read + write) of one decode kernel launch from an ncu capture of
-# this benchmark's workload (profiles/decode_cl_kernel_3b.md), valid while the
-# kernel source is the one captured (its SHA-256 below); otherwise null.
+# this benchmark's workload (its summary is kept under profiles/), valid while
+# the kernel source is the one captured (its SHA-256 below); otherwise null.
 NCU_TRAFFIC = {"3b": {"bytes": 139348224,
                       "source": "kv_cache_compression_layer_b200/csrc/decode_cl.cu",
                       "sha256": "78b5b0da77529123"}}
