@@ -61,6 +61,9 @@ def _get():
             lib.orc_allocate.argtypes = [I32, P, I32, I32, I32, I32, C.c_float, P, P]
             lib.orc_allocate.restype = I32
             lib.orc_select_rows.argtypes = [I64, P, P, P, I32, P, P, P, I32]
+            lib.orc_select_rows_seg.argtypes = [I64, P, P, P, I32, P, I32, P, P, I32]
+            lib.orc_allocate_global.argtypes = [I32, P, I32, I32, I32, I32, C.c_float, P, P]
+            lib.orc_allocate_global.restype = I32
             lib.orc_decode_step.argtypes = [P, I32, I32, P, P, P, P, P, P, P, I64, D, I32, I32, I64, P]
             lib.orc_decode_step.restype = I64
             lib.orc_decode_run_heads.argtypes = [I64, P, I32, I32, P, P, P, P, P, I64, P, P, P, P, D, I32, P, P,
@@ -166,6 +169,21 @@ def allocate(S: np.ndarray, L_seq: Sequence[int], w: int, budget_pct: int, r: fl
     return b
 
 
+def allocate_global(S: np.ndarray, L_seq: Sequence[int], w: int, budget_pct: int, r: float) -> np.ndarray:
+    """Budgets b [n_seq][layers][H] from one allocation over all (layer, head) of a sequence
+    (variant of step 3: the same total, formula and rounding over n_layers * H heads)."""
+    S = _c(S, np.float32)
+    n_layers, H = S.shape
+    L = _c(L_seq, np.int64)
+    b = np.zeros((len(L), n_layers, H), np.int32)
+    st = _get().orc_allocate_global(len(L), _p(L), n_layers, H, w, budget_pct, C.c_float(r), _p(S), _p(b))
+    if st == 3:
+        raise BudgetError("budget below n_layers*H*w")
+    if st:
+        raise ValueError(f"allocate_global failed ({st})")
+    return b
+
+
 # ---------------------------------------------------------------- step 4 ----
 def select(s_hat: np.ndarray, L_rows: Sequence[int], w: int, b_rows: Sequence[int],
            n_threads: int = 0) -> list:
@@ -179,6 +197,22 @@ def select(s_hat: np.ndarray, L_rows: Sequence[int], w: int, b_rows: Sequence[in
     idx = np.zeros(max(1, ioff[-1]), np.int32)
     _get().orc_select_rows(len(L), _p(L), _p(off), _p(s_hat), w, _p(b), _p(ioff), _p(idx),
                            n_threads or default_threads())
+    return [idx[ioff[i]:ioff[i + 1]].copy() for i in range(len(L))]
+
+
+def select_segmented(s_hat: np.ndarray, L_rows: Sequence[int], w: int, b_rows: Sequence[int], nseg: int,
+                     n_threads: int = 0) -> list:
+    """Kept positions per row, ascending: last w + per-segment top-q_i of s_hat over [0, L-w)
+    (variant of step 4: nseg equal segments, quotas by largest remainder)."""
+    s_hat = _c(s_hat, np.float64)
+    L = _c(L_rows, np.int64)
+    off = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+    b = _c(b_rows, np.int32)
+    keep = np.minimum(b.astype(np.int64), L)
+    ioff = np.concatenate([[0], np.cumsum(keep)]).astype(np.int64)
+    idx = np.zeros(max(1, ioff[-1]), np.int32)
+    _get().orc_select_rows_seg(len(L), _p(L), _p(off), _p(s_hat), w, _p(b), int(nseg), _p(ioff), _p(idx),
+                               n_threads or default_threads())
     return [idx[ioff[i]:ioff[i + 1]].copy() for i in range(len(L))]
 
 

@@ -339,6 +339,25 @@ int orc_allocate(int n_seq, const int64_t* L, int n_layers, int H, int w, int bu
   return 0;
 }
 
+/* Variant of step 3: one allocation over every (layer, head) of a sequence   */
+/* ([AudioKV] §2.1: the audio-critical heads concentrate in some layers, so a */
+/* budget shared across layers can follow them).                               */
+/* READINGS: the same total as the per-layer allocation,                        */
+/* B = n_layers * floor(pct L H / 100), split by the same formula, rounding,    */
+/* remainder and capping rule over the n_layers * H heads in (layer, head)      */
+/* order (H in the formula becomes n_layers * H).                               */
+int orc_allocate_global(int n_seq, const int64_t* L, int n_layers, int H, int w, int budget_pct, float r,
+                        const float* S, int32_t* b) {
+  const int Hg = n_layers * H;
+  if (Hg > 1024) return 1;
+  for (int s = 0; s < n_seq; ++s) {
+    int64_t B = (int64_t)n_layers * (((int64_t)budget_pct * L[s] * H) / 100);
+    int st = alloc_layer(Hg, L[s], w, B, (double)r, S, b + (size_t)s * Hg);
+    if (st) return st;
+  }
+  return 0;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Step 4. Per-head selection ([AudioKV] §3.1 keeps a basic local context     */
 /* window; the rest goes by smoothed score).                                   */
@@ -384,6 +403,57 @@ void orc_select_row(const double* s_hat, int64_t L, int w, int64_t b, int32_t* i
   free(k);
 }
 
+/* Variant of step 4: segment-wise selection ([WnW] fixed heads keep a static */
+/* subset chosen per segment rather than by one top-k over the whole row, so   */
+/* that no stretch of a long recording is left without cache).                 */
+/* READINGS: the candidates [0, L - w) are cut into nseg segments with bounds  */
+/* e_i = floor(i (L - w) / nseg); segment i keeps q_i of the b - w positions,   */
+/* q_i = floor(k len_i / (L - w)) plus one for the (k - sum q) segments with    */
+/* the largest remainders (k len_i mod (L - w)), ties to the lower segment; in  */
+/* each segment the top-q_i by s_hat (ties to the lower index, a full sort);   */
+/* the window and the b >= L bypass are as in step 4. Output ascending.        */
+void orc_select_row_seg(const double* s_hat, int64_t L, int w, int64_t b, int nseg, int32_t* idx) {
+  if (b >= L) {
+    for (int64_t j = 0; j < L; ++j) idx[j] = (int32_t)j;
+    return;
+  }
+  const int64_t n = L - w, k = b - w;
+  int64_t* q = (int64_t*)malloc(sizeof(int64_t) * (size_t)nseg);
+  int64_t* fr = (int64_t*)malloc(sizeof(int64_t) * (size_t)nseg);
+  char* got = (char*)calloc((size_t)nseg, 1);
+  int64_t sum_q = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int64_t len = (int64_t)(i + 1) * n / nseg - (int64_t)i * n / nseg;
+    q[i] = k * len / n;
+    fr[i] = k * len % n;
+    sum_q += q[i];
+  }
+  for (int64_t t = 0; t < k - sum_q; ++t) { /* the largest remainders, lower segment first */
+    int best = -1;
+    for (int i = 0; i < nseg; ++i)
+      if (!got[i] && (best < 0 || fr[i] > fr[best])) best = i;
+    got[best] = 1;
+    q[best] += 1;
+  }
+  keyed* kk = (keyed*)malloc(sizeof(keyed) * (size_t)(n > 0 ? n : 1));
+  int64_t at = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int64_t lo = (int64_t)i * n / nseg, hi = (int64_t)(i + 1) * n / nseg;
+    for (int64_t j = lo; j < hi; ++j) {
+      kk[j - lo].v = s_hat[j] == 0.0 ? 0.0 : s_hat[j]; /* -0 == +0 */
+      kk[j - lo].j = (int32_t)j;
+    }
+    qsort(kk, (size_t)(hi - lo), sizeof(keyed), cmp_desc_then_index);
+    for (int64_t t = 0; t < q[i]; ++t) idx[at++] = kk[t].j;
+  }
+  for (int64_t i = 0; i < w; ++i) idx[at++] = (int32_t)(n + i);
+  qsort(idx, (size_t)b, sizeof(int32_t), cmp_int32);
+  free(kk);
+  free(got);
+  free(fr);
+  free(q);
+}
+
 typedef struct {
   const int64_t* L;
   const int64_t* off;
@@ -392,16 +462,26 @@ typedef struct {
   const int32_t* b;
   const int64_t* idx_off;
   int32_t* idx;
+  int nseg; /* 0: one top-k over the row (step 4); > 0: segment-wise */
 } sel_ctx;
 
 static void sel_task(int64_t i, void* vctx) {
   sel_ctx* c = (sel_ctx*)vctx;
-  orc_select_row(c->s_hat + c->off[i], c->L[i], c->w, c->b[i], c->idx + c->idx_off[i]);
+  if (c->nseg > 0)
+    orc_select_row_seg(c->s_hat + c->off[i], c->L[i], c->w, c->b[i], c->nseg, c->idx + c->idx_off[i]);
+  else
+    orc_select_row(c->s_hat + c->off[i], c->L[i], c->w, c->b[i], c->idx + c->idx_off[i]);
 }
 
 void orc_select_rows(int64_t n_rows, const int64_t* L, const int64_t* off, const double* s_hat, int w,
                      const int32_t* b, const int64_t* idx_off, int32_t* idx, int n_threads) {
-  sel_ctx c = {L, off, s_hat, w, b, idx_off, idx};
+  sel_ctx c = {L, off, s_hat, w, b, idx_off, idx, 0};
+  orc_parallel(n_rows, n_threads, sel_task, &c);
+}
+
+void orc_select_rows_seg(int64_t n_rows, const int64_t* L, const int64_t* off, const double* s_hat, int w,
+                         const int32_t* b, int nseg, const int64_t* idx_off, int32_t* idx, int n_threads) {
+  sel_ctx c = {L, off, s_hat, w, b, idx_off, idx, nseg};
   orc_parallel(n_rows, n_threads, sel_task, &c);
 }
 
