@@ -7,6 +7,8 @@
  *   kv_sss    -> Spectral Score Smoothing s_hat, k*    (AudioKV blog §2.2)
  *   kv_allocate -> head-aware per-row budgets b        (AudioKV blog §3.1, §5.1)
  *   kv_select_gather -> kept indices + compacted K/V   (AudioKV blog §3.1)
+ *   variants: kv_allocate_global (budgets pooled over a sequence's layers,
+ *   AudioKV blog §2.1), kv_select_gather_segmented (WnW segment-wise subset)
  *   kv_decode_attn_update -> one decode step with the temporally decayed
  *        score update and sink/recent/top-N eviction   (VoxZip, second stage)
  *
@@ -170,6 +172,20 @@ int kv_allocate(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv
                 int32_t* b, int64_t* slot_off, void* stream);
 
 /*
+ * kv_allocate_global — the same allocation over every (layer, head) of a
+ * sequence at once (AudioKV blog §2.1: the audio-critical heads concentrate
+ * in some layers, so a budget shared across layers can follow them): the
+ * n_layers * H heads share B = n_layers * floor(budget_pct * L * H / 100),
+ * with the formula, rounding, remainder (ties to the lower (layer, head)) and
+ * capping of kv_allocate over n_layers * H heads. The total per sequence, and
+ * so kv_total_slots, is kv_allocate's.
+ *   Arguments and outputs as kv_allocate; n_layers * n_kv_heads <= 1024.
+ * Errors: KV_ERR_ARG, KV_ERR_BUDGET, KV_ERR_CUDA.
+ */
+int kv_allocate_global(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
+                       const float* S, int32_t* b, int64_t* slot_off, void* stream);
+
+/*
  * kv_select_gather — per-row selection and compaction (AudioKV blog §3.1
  * keeps the local window; the C3 page's bypass keeps all when b >= L):
  *   keep the last w positions and the top-(b - w) positions of s_hat over
@@ -187,6 +203,24 @@ int kv_allocate(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv
 int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat, const void* K,
                      const void* V, const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
                      void* stream);
+
+/*
+ * kv_select_gather_segmented — kv_select_gather with WnW's segment-wise
+ * static subset (WnW digest: fixed heads keep positions chosen per segment,
+ * not by one top-k over the whole recording, so no stretch is left without
+ * cache): the candidates [0, L - w) are cut into n_segments segments
+ * [floor(i (L - w) / n), floor((i + 1) (L - w) / n)); segment i keeps
+ * q_i = floor(k len_i / (L - w)) of the k = b - w kept candidates, plus one
+ * for the (k - sum q) segments with the largest remainders k len_i mod (L - w)
+ * (ties to the lower segment), choosing its top-q_i by s_hat (ties to the
+ * lower index). The window, the b >= L bypass, the outputs and the gather
+ * are those of kv_select_gather. 1 <= n_segments <= 4096; n_segments = 1 is
+ * kv_select_gather.
+ * Errors: KV_ERR_ARG, KV_ERR_CUDA.
+ */
+int kv_select_gather_segmented(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat,
+                               const void* K, const void* V, const int32_t* b, const int64_t* slot_off,
+                               int32_t n_segments, int32_t* idx, void* Kc, void* Vc, void* stream);
 
 /*
  * kv_decode_init — prepares the decode state after kv_select_gather:

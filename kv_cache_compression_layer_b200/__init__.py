@@ -25,7 +25,8 @@ META_INTS = 8
 # Every symbol include/kvcomp.h declares.
 EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
-           "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes")
+           "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes", "kv_allocate_global",
+           "kv_select_gather_segmented")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -72,6 +73,8 @@ def lib():
             "kv_sss": (C.c_int, [Ps, P, I32, P, P, P, C.c_float, C.c_float, P]),
             "kv_allocate": (C.c_int, [Ps, P, I32, Pp, P, P, P, P]),
             "kv_select_gather": (C.c_int, [Ps, P, I32, P, P, P, P, P, P, P, P, P]),
+            "kv_allocate_global": (C.c_int, [Ps, P, I32, Pp, P, P, P, P]),
+            "kv_select_gather_segmented": (C.c_int, [Ps, P, I32, P, P, P, P, P, I32, P, P, P, P]),
             "kv_decode_init": (C.c_int, [Ps, P, I32, Pp, Pc, P]),
             "kv_decode_attn_update": (C.c_int, [Ps, P, I32, Pp, Pc, P, P, P, P, P]),
             "kv_read_device_status": (C.c_int, [P, P, P]),
@@ -181,6 +184,20 @@ def kv_select_gather(shape, L, s_hat, K, V, b, slot_off, idx, Kc, Vc, stream=Non
                                                       _stream(stream)))
 
 
+def kv_allocate_global(shape, L, params, S, b, slot_off, stream=None):
+    arr, n = _L(L)
+    _check("kv_allocate_global", lib().kv_allocate_global(C.byref(shape), arr, n, C.byref(params), _ptr(S), _ptr(b),
+                                                          _ptr(slot_off), _stream(stream)))
+
+
+def kv_select_gather_segmented(shape, L, s_hat, K, V, b, slot_off, n_segments, idx, Kc, Vc, stream=None):
+    arr, n = _L(L)
+    _check("kv_select_gather_segmented",
+           lib().kv_select_gather_segmented(C.byref(shape), arr, n, _ptr(s_hat), _ptr(K), _ptr(V), _ptr(b),
+                                            _ptr(slot_off), int(n_segments), _ptr(idx), _ptr(Kc), _ptr(Vc),
+                                            _stream(stream)))
+
+
 def make_cache(Kc, Vc, A, pos, slot_off, b, meta, status, scratch=None, total_slots: Optional[int] = None,
                scratch_bytes: Optional[int] = None) -> kv_cache:
     if total_slots is None:
@@ -221,4 +238,5 @@ __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", 
            "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_score_noalloc",
            "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
-           "kv_decode_scratch_bytes", "status_string", "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]
+           "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "status_string",
+           "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]

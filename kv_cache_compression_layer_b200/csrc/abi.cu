@@ -176,7 +176,25 @@ int kv_allocate(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv
     const long long B = ((long long)params->budget_pct * L[s] * shape->n_kv_heads) / 100;
     if (B < (long long)shape->n_kv_heads * shape->w) return KV_ERR_BUDGET;
   }
-  return launch_allocate(*shape, m, *params, S, b, slot_off, static_cast<cudaStream_t>(stream));
+  return launch_allocate(*shape, m, *params, S, b, slot_off, false, static_cast<cudaStream_t>(stream));
+}
+
+int kv_allocate_global(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,
+                       const float* S, int32_t* b, int64_t* slot_off, void* stream) {
+  if (fault_injected("kv_allocate_global")) return KV_ERR_CUDA;
+  if (!shape_ok(shape) || !params) return KV_ERR_ARG;
+  if ((long long)shape->n_layers * shape->n_kv_heads > 1024) return KV_ERR_ARG;
+  RowMap m;
+  int st = make_row_map(*shape, L, n_seq, m);
+  if (st) return st;
+  if (!aligned16(S) || !aligned16(b) || !aligned16(slot_off)) return KV_ERR_ARG;
+  if (params->budget_pct < 1 || params->budget_pct > 100 || !(params->r >= 0.f && params->r <= 1.f))
+    return KV_ERR_ARG;
+  for (int s = 0; s < n_seq; ++s) {
+    const long long B = ((long long)params->budget_pct * L[s] * shape->n_kv_heads) / 100;
+    if (B < (long long)shape->n_kv_heads * shape->w) return KV_ERR_BUDGET;
+  }
+  return launch_allocate(*shape, m, *params, S, b, slot_off, true, static_cast<cudaStream_t>(stream));
 }
 
 int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat, const void* K,
@@ -190,7 +208,22 @@ int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, con
   for (const void* p : {(const void*)s_hat, K, V, (const void*)b, (const void*)slot_off, (const void*)idx,
                         (const void*)Kc, (const void*)Vc})
     if (!aligned16(p)) return KV_ERR_ARG;
-  return launch_select_gather(*shape, m, s_hat, K, V, b, slot_off, idx, Kc, Vc, static_cast<cudaStream_t>(stream));
+  return launch_select_gather(*shape, m, s_hat, K, V, b, slot_off, idx, Kc, Vc, 0, static_cast<cudaStream_t>(stream));
+}
+
+int kv_select_gather_segmented(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat,
+                               const void* K, const void* V, const int32_t* b, const int64_t* slot_off,
+                               int32_t n_segments, int32_t* idx, void* Kc, void* Vc, void* stream) {
+  if (fault_injected("kv_select_gather_segmented")) return KV_ERR_CUDA;
+  if (!shape_ok(shape) || n_segments < 1 || n_segments > kMaxSelectSegments) return KV_ERR_ARG;
+  RowMap m;
+  int st = make_row_map(*shape, L, n_seq, m);
+  if (st) return st;
+  for (const void* p : {(const void*)s_hat, K, V, (const void*)b, (const void*)slot_off, (const void*)idx,
+                        (const void*)Kc, (const void*)Vc})
+    if (!aligned16(p)) return KV_ERR_ARG;
+  return launch_select_gather(*shape, m, s_hat, K, V, b, slot_off, idx, Kc, Vc, n_segments,
+                              static_cast<cudaStream_t>(stream));
 }
 
 static bool cache_ok(const kv_cache* c) {

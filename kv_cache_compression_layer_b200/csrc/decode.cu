@@ -326,14 +326,16 @@ __global__ void decode_init_kernel(const int64_t* __restrict__ slot_off, const i
   }
 }
 
-// Largest b_i + 1 a row can have: b_h <= min(L, B - (H - 1) w) since every
-// other head of the layer keeps at least w.
+// Largest b_i + 1 a row can have: b_h <= min(L, B - (H' - 1) w) since every
+// other head sharing the budget B keeps at least w (H' = H heads of a layer,
+// or all n_layers H heads of a sequence for kv_allocate_global).
 int cap_bound(const kv_shape& sh, const RowMap& m, const kv_params& p) {
   long long mx = 0;
   for (int s = 0; s < m.n_seq; ++s) {
     const long long L = m.L[s];
-    const long long B = ((long long)p.budget_pct * L * sh.n_kv_heads) / 100;
-    const long long bmax = std::min(L, B - (long long)(sh.n_kv_heads - 1) * sh.w);
+    // the larger of the per-layer and the pooled (kv_allocate_global) bounds
+    const long long B = (long long)sh.n_layers * (((long long)p.budget_pct * L * sh.n_kv_heads) / 100);
+    const long long bmax = std::min(L, B - ((long long)sh.n_layers * sh.n_kv_heads - 1) * sh.w);
     mx = std::max(mx, bmax + 1);
   }
   return (int)mx;

@@ -70,7 +70,8 @@ struct TileHdr {
 size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* base, TcScratch* sc) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int per_row = (capb + kCH - 1) / kCH;
-  const int max_items = rows * per_row;
+  // rows hold at most per_row items each and sum(b + 1) = total_slots slots in all
+  const int max_items = (int)std::min<long long>((long long)rows * per_row, total_slots / kCH + rows);
   const int stride = (kPartO + G * d + 3) & ~3;
   const int max_bests = (per_row + 1) * kWarps;
   size_t off = 0;

@@ -30,10 +30,11 @@ int launch_score(const kv_shape& sh, const RowMap& m, const void* qwin, const vo
 int launch_sss(const RowMap& m, const float* s, float* s_hat, int32_t* kstar, float alpha, float rho,
                cudaStream_t st);
 int launch_allocate(const kv_shape& sh, const RowMap& m, const kv_params& p, const float* S, int32_t* b,
-                    int64_t* slot_off, cudaStream_t st);
+                    int64_t* slot_off, bool global, cudaStream_t st);
 int launch_select_gather(const kv_shape& sh, const RowMap& m, const float* s_hat, const void* K, const void* V,
-                         const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
+                         const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc, int nseg,
                          cudaStream_t st);
+constexpr int kMaxSelectSegments = 4096;
 size_t decode_scratch_bytes(const kv_shape& sh, const RowMap& m, const kv_params& p, long long total_slots);
 int launch_decode_init(const kv_shape& sh, const RowMap& m, const kv_params& p, const kv_cache& c,
                        cudaStream_t st);

@@ -3,7 +3,8 @@
 // row's budget goes to the highest smoothed scores; the C3 page's bypass keeps
 // every position once the budget reaches the audio length).
 //
-// select kernel (one CTA per row): smoothed scores become order-preserving
+// select kernel (one CTA per row; the WnW segment-wise variant takes the
+// row's segments in turn): smoothed scores become order-preserving
 // uint32 keys (-0 folded into +0) in shared memory; an MSB-first 8-bit radix
 // select finds the k-th largest key T and how many keys equal to T are taken;
 // a warp-ballot compaction then writes the kept indices in ascending order:
@@ -18,6 +19,7 @@ namespace {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kMaxSegments = 4096;  // segments of a row in the segment-wise selection
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -25,68 +27,47 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1)
-    select_kernel(const RowMap map, int w, const float* __restrict__ s_hat, const int32_t* __restrict__ b,
-                  const int64_t* __restrict__ slot_off, int32_t* __restrict__ idx) {
-  extern __shared__ uint32_t keys[];
-  __shared__ int hist[256];
-  __shared__ int wgt[kSelWarps], weq[kSelWarps];
-  __shared__ uint32_t sh_prefix;
-  __shared__ int sh_kk;
-
-  const int row = blockIdx.x;
-  const int L = row_len(map, row);
-  const long long koff = row_key_off(map, row);
-  const int bb = b[row];
-  int32_t* out = idx + slot_off[row];
+// The k largest keys of keys[c0s, c1s) (ties to the lower index) written to
+// out[0, k) in ascending index order; called by the whole block.
+__device__ void select_range(const uint32_t* keys, int c0s, int c1s, int k, int32_t* __restrict__ out, int* hist,
+                             int* wgt, int* weq, uint32_t* sh_prefix, int* sh_kk) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (bb >= L) {
-    for (int j = threadIdx.x; j < L; j += kSelThreads) out[j] = j;
-    return;
-  }
-  if (bb < w) return;  // not a valid budget (kv_allocate never produces one); nothing is written
-  const int n = L - w;  // candidates [0, n); the window [n, L) is always kept
-  const int k = bb - w;
-  for (int i = threadIdx.x; i < w; i += kSelThreads) out[k + i] = n + i;
-  if (k <= 0) return;
-
-  for (int j = threadIdx.x; j < n; j += kSelThreads) keys[j] = order_key(s_hat[koff + j]);
+  const int n = c1s - c0s;
+  __syncthreads();  // the keys are in place, the previous range's scratch is free
   if (threadIdx.x == 0) {
-    sh_prefix = 0;
-    sh_kk = k;
+    *sh_prefix = 0;
+    *sh_kk = k;
   }
   __syncthreads();
-
   // radix select of the k-th largest key, most significant byte first
   uint32_t mask = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    const uint32_t prefix = sh_prefix;
-    for (int j = threadIdx.x; j < n; j += kSelThreads) {
+    const uint32_t prefix = *sh_prefix;
+    for (int j = c0s + threadIdx.x; j < c1s; j += kSelThreads) {
       const uint32_t key = keys[j];
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-      int kk = sh_kk, cum = 0, dg = 0;
+      int kk = *sh_kk, cum = 0, dg = 0;
       for (dg = 255; dg > 0; --dg) {
         if (cum + hist[dg] >= kk) break;
         cum += hist[dg];
       }
-      sh_kk = kk - cum;
-      sh_prefix = prefix | ((uint32_t)dg << shift);
+      *sh_kk = kk - cum;
+      *sh_prefix = prefix | ((uint32_t)dg << shift);
     }
     mask |= 255u << shift;
     __syncthreads();
   }
-  const uint32_t T = sh_prefix;
-  const int take_eq = sh_kk;  // keys equal to T to keep, lowest indices first
+  const uint32_t T = *sh_prefix;
+  const int take_eq = *sh_kk;  // keys equal to T to keep, lowest indices first
 
   // per-warp counts over contiguous chunks, then ballot compaction in index order
   const int chunk = (((n + kSelWarps - 1) / kSelWarps) + 31) & ~31;
-  const int c0 = warp * chunk, c1 = min(n, c0 + chunk);
+  const int c0 = c0s + warp * chunk, c1 = min(c1s, c0 + chunk);
   int ngt = 0, neq = 0;
   for (int j = c0 + lane; j < c1; j += 32) {
     const uint32_t key = keys[j];
@@ -121,6 +102,65 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     if (sel && at < k) out[at] = j;
     eq_before += __popc(beq);
     sel_before += __popc(bsel);
+  }
+}
+
+// One CTA per row. nseg = 0: one top-(b - w) over the candidates [0, L - w);
+// nseg > 0: the candidates cut into nseg segments [floor(i n / nseg),
+// floor((i + 1) n / nseg)), segment i keeping q_i = floor(k len_i / n) plus
+// one for the (k - sum q) largest remainders k len_i mod n (ties to the lower
+// segment) -- WnW's segment-wise static subset.
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_kernel(const RowMap map, int w, int nseg, const float* __restrict__ s_hat, const int32_t* __restrict__ b,
+                  const int64_t* __restrict__ slot_off, int32_t* __restrict__ idx) {
+  extern __shared__ uint32_t keys[];
+  __shared__ int hist[256];
+  __shared__ int wgt[kSelWarps], weq[kSelWarps];
+  __shared__ uint32_t sh_prefix;
+  __shared__ int sh_kk;
+  __shared__ int q_s[kMaxSegments];
+
+  const int row = blockIdx.x;
+  const int L = row_len(map, row);
+  const long long koff = row_key_off(map, row);
+  const int bb = b[row];
+  int32_t* out = idx + slot_off[row];
+
+  if (bb >= L) {
+    for (int j = threadIdx.x; j < L; j += kSelThreads) out[j] = j;
+    return;
+  }
+  if (bb < w) return;  // not a valid budget (kv_allocate never produces one); nothing is written
+  const int n = L - w;  // candidates [0, n); the window [n, L) is always kept
+  const int k = bb - w;
+  for (int i = threadIdx.x; i < w; i += kSelThreads) out[k + i] = n + i;
+  if (k <= 0) return;
+  for (int j = threadIdx.x; j < n; j += kSelThreads) keys[j] = order_key(s_hat[koff + j]);
+  if (nseg <= 0) {
+    select_range(keys, 0, n, k, out, hist, wgt, weq, &sh_prefix, &sh_kk);
+    return;
+  }
+  // segment quotas: q_i = floor(k len_i / n), the remainder by largest k len_i mod n
+  for (int i = threadIdx.x; i < nseg; i += kSelThreads) {
+    const long long len = (long long)(i + 1) * n / nseg - (long long)i * n / nseg;
+    const long long fr = (long long)k * len % n;
+    long long sum_q = 0;
+    int rank = 0;
+    for (int i2 = 0; i2 < nseg; ++i2) {
+      const long long len2 = (long long)(i2 + 1) * n / nseg - (long long)i2 * n / nseg;
+      sum_q += (long long)k * len2 / n;
+      const long long fr2 = (long long)k * len2 % n;
+      rank += fr2 > fr || (fr2 == fr && i2 < i);
+    }
+    q_s[i] = (int)((long long)k * len / n) + (rank < k - sum_q ? 1 : 0);
+  }
+  __syncthreads();
+  int at = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int lo = (int)((long long)i * n / nseg), hi = (int)((long long)(i + 1) * n / nseg);
+    const int q = q_s[i];
+    if (q > 0) select_range(keys, lo, hi, q, out + at, hist, wgt, weq, &sh_prefix, &sh_kk);
+    at += q;
   }
 }
 
@@ -171,7 +211,7 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 int launch_select_gather(const kv_shape& sh, const RowMap& m, const float* s_hat, const void* K, const void* V,
-                         const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
+                         const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc, int nseg,
                          cudaStream_t st) {
   int maxL = 0;
   for (int i = 0; i < m.n_seq; ++i) maxL = std::max(maxL, m.L[i]);
@@ -180,7 +220,8 @@ int launch_select_gather(const kv_shape& sh, const RowMap& m, const float* s_hat
     cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     attr = true;
   }
-  select_kernel<<<m.n_rows, kSelThreads, (size_t)maxL * sizeof(uint32_t), st>>>(m, sh.w, s_hat, b, slot_off, idx);
+  select_kernel<<<m.n_rows, kSelThreads, (size_t)maxL * sizeof(uint32_t), st>>>(m, sh.w, nseg, s_hat, b, slot_off,
+                                                                                 idx);
   const int esz = sh.dtype == KV_BF16 ? 2 : 4;
   const int row_bytes = sh.head_dim * esz;
   gather_kernel<<<sm_count() * 8, 256, 0, st>>>(m, row_bytes, slot_off, b, idx, static_cast<const uint8_t*>(K),
