@@ -66,6 +66,8 @@ def _get():
             lib.orc_allocate_global.restype = I32
             lib.orc_decode_step.argtypes = [P, I32, I32, P, P, P, P, P, P, P, I64, D, I32, I32, I64, P]
             lib.orc_decode_step.restype = I64
+            lib.orc_voxzip_pool.argtypes = [I64, I32, P, D, I64, P, P, P, P, P, C.c_float, P, P]
+            lib.orc_voxzip_pool.restype = I64
             lib.orc_decode_run_heads.argtypes = [I64, P, I32, I32, P, P, P, P, P, I64, P, P, P, P, D, I32, P, P,
                                                  P, P, I32]
             _lib = lib
@@ -310,5 +312,26 @@ def decode_run_heads(Kc_list, Vc_list, pos_list, q, k_new, v_new, pos0, gamma, T
     return o, ev
 
 
-__all__ = ["build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
+# ------------------------------------------------------ next row: VoxZip ----
+def voxzip_pool(E_A: np.ndarray, tau_total: float, tau: np.ndarray, conf: np.ndarray, n_text: np.ndarray,
+                text_row: np.ndarray, E_T: Optional[np.ndarray] = None, conf_min: float = 0.3):
+    """VoxZip first stage on one sequence (方法概述和架构, first stage): ASR
+    segments with confidence > conf_min mapped to token ranges, each split into
+    L_t groups that are mean-pooled and fused with their text embeddings; the
+    uncovered tokens kept; all in time order. Returns (E_comp [rows][d] float64,
+    src [rows][3] int32 = first token, token count, text row or -1)."""
+    E_A = _c(E_A, np.float64)
+    L, d = E_A.shape
+    tau = _c(tau, np.float64).reshape(-1, 2)
+    n = tau.shape[0]
+    out = np.zeros((max(L, 1), d), np.float64)
+    src = np.zeros((max(L, 1), 3), np.int32)
+    et = None if E_T is None else _c(E_T, np.float64)
+    r = _get().orc_voxzip_pool(L, d, _p(E_A), float(tau_total), n, _p(tau), _p(_c(conf, np.float32)),
+                               _p(_c(n_text, np.int32)), _p(_c(text_row, np.int32)),
+                               None if et is None else _p(et), C.c_float(conf_min), _p(out), _p(src))
+    return out[:r].copy(), src[:r].copy()
+
+
+__all__ = ["voxzip_pool", "build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
            "gather", "DecodeList", "recent_count", "decode_run_heads", "default_threads"]

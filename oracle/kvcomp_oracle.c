@@ -661,3 +661,92 @@ void orc_decode_run_heads(int64_t heads, int64_t* n, int d, int g, float* Kc, fl
   drun_ctx c = {n, d, g, Kc, Vc, A, pos, cache_off, heads, steps, q, k_new, v_new, pos0, gamma, T, M, b, o, evicted};
   orc_parallel(heads, n_threads, drun_task, &c);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Next row: [VoxZip] 方法概述和架构, first stage (Semantic-Anchored Audio   */
+/* Compression) on one sequence of L audio feature rows E_A [L][d]:           */
+/*  1. keep the ASR segments whose confidence exceeds conf_min (0.3 on the    */
+/*     page) and map their timestamps to token indices,                       */
+/*     idx = floor(L * tau / tau_total);                                        */
+/*  2. split the segment's tokens evenly into L_t groups (L_t = its text     */
+/*     tokens), take the element-wise mean of each group and add the text    */
+/*     embedding of the same position;                                        */
+/*  3. keep every token that no kept segment covers as it is, and concatenate */
+/*     fused groups and background tokens in time order.                      */
+/* READINGS: a segment covers [idx_start, idx_end) (end exclusive), indices    */
+/* clamped to [0, L]; it is kept when confidence > conf_min (compared in       */
+/* float32), L_t >= 1 and idx_end > idx_start; kept segments are taken in the */
+/* given order and one that starts before the end of an earlier kept segment  */
+/* starts at that end instead (no token is pooled twice); a segment of len    */
+/* tokens forms n = min(L_t, len) groups, group j being the tokens            */
+/* [floor(j len / n), floor((j + 1) len / n)) from its start, fused with text */
+/* embedding row text_row + j. Output row descriptors src[r] = (first token,  */
+/* token count, text row or -1 for a background token).                       */
+/* ------------------------------------------------------------------------- */
+static int64_t vz_index(int64_t L, double tau, double tau_total) {
+  double x = floor((double)L * tau / tau_total);
+  if (x < 0.0) x = 0.0;
+  if (x > (double)L) x = (double)L;
+  return (int64_t)x;
+}
+
+int64_t orc_voxzip_pool(int64_t L, int d, const double* E_A, double tau_total, int64_t n_seg, const double* tau,
+                        const float* conf, const int32_t* n_text, const int32_t* text_row, const double* E_T,
+                        float conf_min, double* out, int32_t* src) {
+  int64_t* owner = (int64_t*)malloc(sizeof(int64_t) * (size_t)(L > 0 ? L : 1));
+  int64_t* seg_start = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_seg > 0 ? n_seg : 1));
+  int64_t* seg_len = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_seg > 0 ? n_seg : 1));
+  for (int64_t t = 0; t < L; ++t) owner[t] = -1;
+  /* step 1: which tokens each kept segment covers */
+  int64_t covered_to = 0;
+  for (int64_t i = 0; i < n_seg; ++i) {
+    seg_start[i] = 0;
+    seg_len[i] = 0;
+    if (!(conf[i] > conf_min) || n_text[i] < 1) continue;
+    int64_t a = vz_index(L, tau[2 * i], tau_total);
+    const int64_t e = vz_index(L, tau[2 * i + 1], tau_total);
+    if (e <= a) continue;
+    if (a < covered_to) a = covered_to;
+    for (int64_t t = a; t < e; ++t) owner[t] = i;
+    if (e > a) {
+      seg_start[i] = a;
+      seg_len[i] = e - a;
+    }
+    if (e > covered_to) covered_to = e;
+  }
+  /* steps 2 and 3: walk the sequence in time order */
+  int64_t r = 0, t = 0;
+  while (t < L) {
+    const int64_t i = owner[t];
+    if (i < 0) {
+      for (int c = 0; c < d; ++c) out[(size_t)r * d + c] = E_A[(size_t)t * d + c];
+      src[3 * r] = (int32_t)t;
+      src[3 * r + 1] = 1;
+      src[3 * r + 2] = -1;
+      ++r;
+      ++t;
+      continue;
+    }
+    const int64_t len = seg_len[i];
+    const int64_t n = n_text[i] < len ? n_text[i] : len;
+    for (int64_t j = 0; j < n; ++j) {
+      const int64_t lo = seg_start[i] + j * len / n, hi = seg_start[i] + (j + 1) * len / n;
+      for (int c = 0; c < d; ++c) {
+        double sum = 0.0;
+        for (int64_t k = lo; k < hi; ++k) sum += E_A[(size_t)k * d + c];
+        double v = sum / (double)(hi - lo);
+        if (E_T) v += E_T[((size_t)text_row[i] + (size_t)j) * d + c];
+        out[(size_t)r * d + c] = v;
+      }
+      src[3 * r] = (int32_t)lo;
+      src[3 * r + 1] = (int32_t)(hi - lo);
+      src[3 * r + 2] = (int32_t)(text_row[i] + j);
+      ++r;
+    }
+    t = seg_start[i] + len;
+  }
+  free(seg_len);
+  free(seg_start);
+  free(owner);
+  return r;
+}

@@ -26,6 +26,12 @@ pages (AudioKV, VoxZip, WnW, C3); no dataset is read or reproduced:
   18% of (layer, head) pairs multiplied by 4 (ties to the lower index);
 * spikes (ragged batch): 5% of positions per row, whose raw score is
   multiplied by 10 before smoothing (a harness step, not part of the path).
+* ASR segments for the VoxZip pooling row (``asr_segments``): audio features
+  at 12.5 tokens/s (tau_total = L / 12.5 s), speech runs of U(1, 10) s
+  separated by U(0.2, 2) s pauses, confidence U(0, 1) (about 70% above the
+  0.3 cut), 3 text tokens per second of speech (at least 1), text rows laid
+  out segment after segment; features ``E_A ~ N(0, 1)``, text embeddings
+  ``E_T ~ N(0, 0.02)`` (standard deviation).
 
 Values are drawn in float32 and rounded to nearest-even bfloat16 for the
 bf16 workloads; the returned float32 arrays hold those bf16-exact values.
@@ -42,6 +48,7 @@ from scipy.signal import lfilter
 # tensor ids of the counter-based streams
 _T_KEYS, _T_PROJ, _T_KNOISE, _T_VALUES, _T_QWIN, _T_QDEC, _T_VDEC, _T_SPIKE = range(8)
 _T_HEADSCORES = 100
+_T_ASR, _T_FEAT, _T_TEXT = 200, 201, 202
 
 
 @dataclasses.dataclass(frozen=True)
@@ -293,6 +300,49 @@ def make_batch(cfg: Config, steps: Optional[int] = None) -> Batch:
                  spikes=spikes)
 
 
+@dataclasses.dataclass
+class AsrSegments:
+    """Timestamped ASR segments of one sequence (inputs of the VoxZip pooling)."""
+    tau_total: float
+    tau: np.ndarray       # [n][2] float64 start, end (seconds)
+    conf: np.ndarray      # [n] float32
+    n_text: np.ndarray    # [n] int32 text tokens
+    text_row: np.ndarray  # [n] int32 first text-embedding row
+
+
+def asr_segments(seed: int, L: int, rate: float = 12.5) -> AsrSegments:
+    """Seeded speech/pause layout over L audio tokens at `rate` tokens/s."""
+    rng = np.random.Generator(np.random.Philox(key=[seed, _T_ASR]))
+    tau_total = L / rate
+    starts, ends = [], []
+    t = float(rng.uniform(0.0, 2.0))
+    while t < tau_total:
+        e = t + float(rng.uniform(1.0, 10.0))
+        starts.append(t)
+        ends.append(min(e, tau_total))
+        t = e + float(rng.uniform(0.2, 2.0))
+    n = len(starts)
+    tau = np.stack([np.asarray(starts), np.asarray(ends)], axis=1).reshape(n, 2).astype(np.float64)
+    conf = rng.uniform(0.0, 1.0, size=n).astype(np.float32)
+    n_text = np.maximum(1, np.floor(3.0 * (tau[:, 1] - tau[:, 0]))).astype(np.int32)
+    text_row = np.concatenate([[0], np.cumsum(n_text)[:-1]]).astype(np.int32) if n else np.zeros(0, np.int32)
+    return AsrSegments(tau_total, tau, conf, n_text, text_row)
+
+
+def audio_features(seed: int, L: int, d: int, bf16: bool = True) -> np.ndarray:
+    """E_A ~ N(0, 1), [L][d] float32 (bf16-exact when bf16)."""
+    rng = np.random.Generator(np.random.Philox(key=[seed, _T_FEAT]))
+    x = rng.standard_normal((L, d), dtype=np.float32)
+    return round_bf16(x) if bf16 else x
+
+
+def text_embeddings(seed: int, n: int, d: int, bf16: bool = True) -> np.ndarray:
+    """E_T ~ N(0, 0.02^2), [n][d] float32 (bf16-exact when bf16)."""
+    rng = np.random.Generator(np.random.Philox(key=[seed, _T_TEXT]))
+    x = (0.02 * rng.standard_normal((max(n, 0), d), dtype=np.float32)).astype(np.float32)
+    return round_bf16(x) if bf16 else x
+
+
 def small(cfg_name: str, **kw) -> Config:
     """A reduced copy of a named workload (fewer layers / shorter audio) for fast tests."""
     return CONFIGS[cfg_name].with_(**kw)
@@ -300,4 +350,4 @@ def small(cfg_name: str, **kw) -> Config:
 
 __all__ = ["Config", "CONFIGS", "Row", "Batch", "make_row", "make_batch", "keys", "values",
            "window_queries", "decode_queries", "head_scores", "spike_mask", "round_bf16",
-           "to_bf16_bits", "small"]
+           "to_bf16_bits", "small", "AsrSegments", "asr_segments", "audio_features", "text_embeddings"]
