@@ -317,12 +317,81 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if not args.no_next_rows:
+        res["next_rows"] = {"voxzip_pool": measure_voxzip(args, rank, world, dev, stream, flush)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(cfg, bt, args.cpu_rows)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+# ------------------------------------------------------- next rows (VoxZip) --
+VZ_SEQS, VZ_L, VZ_D = 8, 32768, 2048
+
+
+def measure_voxzip(args, rank, world, dev, stream, flush):
+    """kv_voxzip_pool on 8 sequences of 32768 audio feature rows (12.5 rows/s,
+    about 44 min each), d = 2048, bf16, seeded ASR segments; the features are
+    drawn on the device by a seeded generator. Timed with CUDA events per call,
+    L2 flushed between calls."""
+    import torch
+
+    import kv_cache_compression_layer_b200 as kv
+    from kv_cache_compression_layer_b200.replicas import max_over_ranks, replica_seed
+
+    base = replica_seed(11, rank)
+    segs = [synth.asr_segments(base + i, VZ_L) for i in range(VZ_SEQS)]
+    seg_off = np.concatenate([[0], np.cumsum([len(a.conf) for a in segs])]).astype(np.int64)
+    tbase = np.concatenate([[0], np.cumsum([int(a.n_text.sum()) for a in segs])]).astype(np.int64)
+    raw = kv.pack_segments(np.concatenate([a.tau for a in segs]), np.concatenate([a.conf for a in segs]),
+                           np.concatenate([a.n_text for a in segs]),
+                           np.concatenate([a.text_row + tbase[i] for i, a in enumerate(segs)]))
+    seg_dev = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(base)
+    rows = VZ_SEQS * VZ_L
+    E_A = torch.randn(rows, VZ_D, generator=g, device=dev).to(torch.bfloat16)
+    E_T = (0.02 * torch.randn(int(tbase[-1]), VZ_D, generator=g, device=dev)).to(torch.bfloat16)
+    E_comp = torch.empty(rows, VZ_D, dtype=torch.bfloat16, device=dev)
+    src = torch.empty(rows, 3, dtype=torch.int32, device=dev)
+    out_len = torch.empty(VZ_SEQS, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    tt = [a.tau_total for a in segs]
+
+    def call():
+        kv.kv_voxzip_pool([VZ_L] * VZ_SEQS, tt, seg_off, VZ_D, kv.KV_BF16, seg_dev, E_A, E_T, E_T.shape[0], E_comp,
+                          src, out_len, status, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    if status.item():
+        raise RuntimeError(f"kv_voxzip_pool status {status.item():#x}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    us = max_over_ranks(1e3 * sum(a.elapsed_time(b) for a, b in ev) / args.steps, world, dev)
+    n_out = int(out_len.sum().item())
+    s_h = src.cpu().numpy()
+    lens = out_len.cpu().numpy()
+    pooled = sum(int((s_h[i * VZ_L:i * VZ_L + lens[i], 2] >= 0).sum()) for i in range(VZ_SEQS))
+    eb = 2
+    # E_A read once, the text rows of the pooled groups read, E_comp written,
+    # one 12-byte descriptor written by the plan and read by the pool kernel
+    bytes_alg = rows * VZ_D * eb + pooled * VZ_D * eb + n_out * VZ_D * eb + 24 * n_out + len(raw)
+    peak, kind = hbm_peak()
+    gbs = bytes_alg / (us * 1e-6) / 1e9
+    return {"workload": f"{VZ_SEQS} seq x {VZ_L} feature rows, d={VZ_D}, bf16, seeded ASR segments "
+                        f"({int(seg_off[-1])} segments, {n_out} output rows)",
+            "kernels": "vz_plan_kernel + vz_pool_kernel (kv_voxzip_pool)", "us_per_call": us,
+            "rows_per_s": world * rows / (us * 1e-6), "bytes_alg": bytes_alg, "gbs": gbs, "peak": peak,
+            "frac": gbs / peak, "peak_kind": kind + " (hbm_gbs copy)", "launches_per_call": 2}
 
 
 # ------------------------------------------------------------ reference arm --
@@ -364,6 +433,7 @@ def main():
                     help="rows of the oracle sample for cpu_baseline (default: the whole batch)")
     ap.add_argument("--ref-rows", type=int, default=8, help="rows per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true", help="skip the timing of the rows beyond the path")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -1,4 +1,5 @@
-"""Python binding of libkvcomp.so (the C ABI declared in include/kvcomp.h).
+"""Python binding of libkvcomp.so (the C ABI declared in include/kvcomp.h and
+include/kvcomp_next.h).
 
 Argument marshalling only: every step of the path runs in the library's
 sm_100a kernels. Functions take torch tensors (or raw device addresses as
@@ -17,16 +18,16 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkvcomp.so")
 
 KV_OK, KV_ERR_ARG, KV_ERR_UNSUPPORTED_L, KV_ERR_BUDGET, KV_ERR_WORKSPACE, KV_ERR_CUDA, KV_ERR_TIMEOUT = range(7)
-KV_DEV_TIMEOUT, KV_DEV_BUDGET, KV_DEV_CAPACITY = 0x1, 0x2, 0x4
+KV_DEV_TIMEOUT, KV_DEV_BUDGET, KV_DEV_CAPACITY, KV_DEV_RANGE = 0x1, 0x2, 0x4, 0x8
 KV_F32, KV_BF16 = 0, 1
 KV_MAX_SEQ = 64
 META_INTS = 8
 
-# Every symbol include/kvcomp.h declares.
+# Every symbol the headers under include/ declare.
 EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes", "kv_allocate_global",
-           "kv_select_gather_segmented")
+           "kv_select_gather_segmented", "kv_voxzip_pool")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -81,6 +82,7 @@ def lib():
             "kv_status_string": (C.c_char_p, [C.c_int]),
             "kv_score_noalloc": (C.c_int, [Ps, P, I32, P, P, P, P]),
             "kv_decode_scratch_bytes": (SZ, [Ps, P, I32, Pp, I64]),
+            "kv_voxzip_pool": (C.c_int, [P, I32, P, P, I32, I32, C.c_float, P, P, P, I64, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -226,6 +228,32 @@ def kv_decode_attn_update(shape, L, params, cache: kv_cache, q_t, k_t, v_t, out,
                                        _ptr(k_t), _ptr(v_t), _ptr(out), _stream(stream)))
 
 
+# kv_asr_segment (include/kvcomp_next.h), 32 bytes
+ASR_SEGMENT_BYTES = 32
+
+
+def pack_segments(tau, conf, n_text, text_row) -> bytes:
+    """Packs per-segment arrays into kv_asr_segment records (little-endian)."""
+    import struct
+
+    out = bytearray()
+    for (t0, t1), c, n, r in zip(tau, conf, n_text, text_row):
+        out += struct.pack("<ddfiii", float(t0), float(t1), float(c), int(n), int(r), 0)
+    return bytes(out)
+
+
+def kv_voxzip_pool(L_a, tau_total, seg_off, d, dtype, segs, E_A, E_T, n_text_rows, E_comp, src, out_len, status=None,
+                   conf_min: float = 0.3, stream=None):
+    n = len(L_a)
+    La = (C.c_int32 * n)(*[int(x) for x in L_a])
+    tt = (C.c_double * n)(*[float(x) for x in tau_total])
+    so = (C.c_int32 * (n + 1))(*[int(x) for x in seg_off])
+    _check("kv_voxzip_pool",
+           lib().kv_voxzip_pool(La, n, tt, so, int(d), int(dtype), C.c_float(conf_min), _ptr(segs), _ptr(E_A),
+                                _ptr(E_T), int(n_text_rows), _ptr(E_comp), _ptr(src), _ptr(out_len), _ptr(status),
+                                _stream(stream)))
+
+
 def kv_read_device_status(status_dev, stream=None) -> int:
     host = C.c_int32(0)
     _check("kv_read_device_status", lib().kv_read_device_status(_ptr(status_dev), C.byref(host), _stream(stream)))
@@ -238,5 +266,6 @@ __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", 
            "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_score_noalloc",
            "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
-           "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "status_string",
+           "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "kv_voxzip_pool",
+           "pack_segments", "ASR_SEGMENT_BYTES", "status_string",
            "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]

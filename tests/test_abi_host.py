@@ -20,7 +20,9 @@ def L():
 
 
 def _declared():
-    hdr = open(os.path.join(ROOT, "include", "kvcomp.h")).read()
+    import glob
+
+    hdr = "".join(open(f).read() for f in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
     hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
     return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(kv_\w+)\s*\(", hdr, flags=re.M)))
 
@@ -96,6 +98,27 @@ def test_argument_errors_launch_nothing(L):
     cache = kv.kv_cache()
     st = L.kv_decode_attn_update(C.byref(sh), Larr, 1, C.byref(_params()), C.byref(cache), 16, 16, 16, 16, None)
     assert st == kv.KV_ERR_ARG
+
+
+def test_voxzip_argument_errors_launch_nothing(L):
+    def call(L_a=(1000,), tau=(80.0,), seg_off=(0, 0), d=2048, dtype=kv.KV_BF16, segs=None, E_A=16, E_T=None,
+             n_text_rows=0, E_comp=4096, src=256, out_len=512, status=None):
+        n = len(L_a)
+        return L.kv_voxzip_pool((C.c_int32 * n)(*L_a), n, (C.c_double * n)(*tau), (C.c_int32 * (n + 1))(*seg_off),
+                                d, dtype, C.c_float(0.3), segs, E_A, E_T, n_text_rows, E_comp, src, out_len,
+                                status, None)
+
+    assert call(d=3) == kv.KV_ERR_ARG  # 6-byte rows
+    assert call(d=4, dtype=kv.KV_BF16) == kv.KV_ERR_ARG  # 8-byte rows
+    assert call(tau=(0.0,)) == kv.KV_ERR_ARG
+    assert call(tau=(float("inf"),)) == kv.KV_ERR_ARG
+    assert call(L_a=(0,)) == kv.KV_ERR_ARG
+    assert call(seg_off=(0, 4097), segs=64) == kv.KV_ERR_ARG  # too many segments
+    assert call(seg_off=(0, 3), segs=None) == kv.KV_ERR_ARG
+    assert call(seg_off=(1, 3), segs=64) == kv.KV_ERR_ARG
+    assert call(E_A=24) == kv.KV_ERR_ARG  # misaligned
+    assert call(E_T=32, n_text_rows=10) == kv.KV_ERR_ARG  # text rows but no status word
+    assert len(kv.pack_segments([(0.0, 1.0)], [0.5], [1], [0])) == kv.ASR_SEGMENT_BYTES
 
 
 def test_fault_injection_env(L, monkeypatch):
