@@ -68,6 +68,10 @@ def _get():
             lib.orc_decode_step.restype = I64
             lib.orc_voxzip_pool.argtypes = [I64, I32, P, D, I64, P, P, P, P, P, C.c_float, P, P]
             lib.orc_voxzip_pool.restype = I64
+            lib.orc_wnw_chunks.argtypes = [I64, I64, I64]
+            lib.orc_wnw_chunks.restype = I64
+            lib.orc_wnw_step.argtypes = [I64, I32, P, I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P]
+            lib.orc_wnw_step.restype = I32
             lib.orc_decode_run_heads.argtypes = [I64, P, I32, I32, P, P, P, P, P, I64, P, P, P, P, D, I32, P, P,
                                                  P, P, I32]
             _lib = lib
@@ -333,5 +337,39 @@ def voxzip_pool(E_A: np.ndarray, tau_total: float, tau: np.ndarray, conf: np.nda
     return out[:r].copy(), src[:r].copy()
 
 
-__all__ = ["voxzip_pool", "build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
+# --------------------------------------------------------- next row: WnW ----
+class WnwState:
+    """One sequence's WnW chunk/block residency (方法概述和架构, 细节详述):
+    idle count per chunk (-1 = not resident), slot per block, block per slot."""
+
+    def __init__(self, L: int, chunk_len: int, stride: int, top_c: int, release_after: int, n_slots: int):
+        self.L, self.chunk_len, self.stride = L, chunk_len, stride
+        self.top_c, self.release_after, self.n_slots = top_c, release_after, n_slots
+        self.M = int(_get().orc_wnw_chunks(L, chunk_len, stride))
+        self.nb = (L + stride - 1) // stride
+        self.idle = np.full(self.M, -1, np.int32)
+        self.block_slot = np.full(self.nb, -1, np.int32)
+        self.slot_block = np.full(n_slots, -1, np.int32)
+
+    def step(self, s: np.ndarray):
+        """s [n_anchor][L] anchor attention mass. Returns (score [M] float64, selected,
+        fetch [n][2] (block, slot), release [n][2])."""
+        s = _c(s, np.float32)
+        n_anchor = s.shape[0]
+        score = np.zeros(self.M, np.float64)
+        sel = np.zeros(max(1, min(self.top_c, self.M)), np.int32)
+        cap = max(1, self.nb)
+        fetch = np.zeros((cap, 2), np.int32)
+        release = np.zeros((cap, 2), np.int32)
+        nf, nr = C.c_int32(0), C.c_int32(0)
+        st = _get().orc_wnw_step(self.L, n_anchor, _p(s), self.chunk_len, self.stride, self.top_c,
+                                 self.release_after, self.n_slots, _p(self.idle), _p(self.block_slot),
+                                 _p(self.slot_block), _p(score), _p(sel), _p(fetch), C.byref(nf), _p(release),
+                                 C.byref(nr))
+        if st:
+            raise RuntimeError("WnW slots exhausted")
+        return score, sel[:min(self.top_c, self.M)].copy(), fetch[:nf.value].copy(), release[:nr.value].copy()
+
+
+__all__ = ["WnwState", "voxzip_pool", "build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
            "gather", "DecodeList", "recent_count", "decode_run_heads", "default_threads"]

@@ -750,3 +750,107 @@ int64_t orc_voxzip_pool(int64_t L, int d, const double* E_A, double tau_total, i
   free(owner);
   return r;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Next row: [WnW] anchor heads and tidal heads ("WnW: Waxing-and-Waning KV   */
+/* Cache for Long-Form Speech LLMs", 方法概述和架构 and 细节详述): at every  */
+/* decode step the anchor heads' attention over the audio positions is summed */
+/* into the importance of overlapping time chunks (4 s long, 2 s apart); the  */
+/* top 3 chunks are selected; a chunk leaves the GPU only after 3 steps in a  */
+/* row without being selected; the tidal heads' GPU copy holds the resident   */
+/* chunks, recalled from the full copy in host memory.                        */
+/* READINGS: chunk m covers positions [m S, min(m S + C, L)) (C = chunk_len,  */
+/* S = chunk_stride, C a multiple of S), m = 0 .. M - 1 with M = 1 when        */
+/* L <= C, else ceil((L - C) / S) + 1; its score is the sum over the anchor   */
+/* rows, then over its positions, of the anchors' attention mass s (float64, */
+/* in that order); the top_c largest scores are selected (ties to the lower   */
+/* chunk; all chunks when M <= top_c); a selected chunk's idle count becomes  */
+/* 0, a resident unselected one's grows by 1 and it is released when the      */
+/* count reaches release_after (-1 = not resident). Storage is kept per block */
+/* [b S, min((b + 1) S, L)): a block is resident while a resident chunk holds */
+/* it; blocks that stop being resident free their slots, then the new blocks, */
+/* in ascending order, take the lowest free slots.                            */
+/* ------------------------------------------------------------------------- */
+int64_t orc_wnw_chunks(int64_t L, int64_t chunk_len, int64_t stride) {
+  if (L <= chunk_len) return 1;
+  return (L - chunk_len + stride - 1) / stride + 1;
+}
+
+/* One step of one sequence. idle [M], block_slot [nb], slot_block [n_slots]  */
+/* are the state (updated); score [M], selected [min(top_c, M)], fetch and    */
+/* release [..][2] (block, slot) and their counts are outputs. Returns 0, or  */
+/* 1 when the slots run out (never when n_slots >= top_c * release_after *    */
+/* chunk_len / chunk_stride).                                                 */
+int orc_wnw_step(int64_t L, int n_anchor, const float* s, int chunk_len, int stride, int top_c, int release_after,
+                 int n_slots, int32_t* idle, int32_t* block_slot, int32_t* slot_block, double* score,
+                 int32_t* selected, int32_t* fetch, int32_t* n_fetch, int32_t* release, int32_t* n_release) {
+  const int64_t M = orc_wnw_chunks(L, chunk_len, stride);
+  const int64_t nb = (L + stride - 1) / stride;
+  /* chunk importance */
+  for (int64_t m = 0; m < M; ++m) {
+    const int64_t lo = m * stride, hi = lo + chunk_len < L ? lo + chunk_len : L;
+    double acc = 0.0;
+    for (int a = 0; a < n_anchor; ++a)
+      for (int64_t j = lo; j < hi; ++j) acc += (double)s[(size_t)a * (size_t)L + (size_t)j];
+    score[m] = acc;
+  }
+  /* top_c selection: repeatedly the largest unselected score, lower chunk first */
+  const int64_t n_sel = top_c < M ? top_c : M;
+  char* chosen = (char*)calloc((size_t)(M > 0 ? M : 1), 1);
+  for (int64_t k = 0; k < n_sel; ++k) {
+    int64_t best = -1;
+    for (int64_t m = 0; m < M; ++m)
+      if (!chosen[m] && (best < 0 || score[m] > score[best])) best = m;
+    chosen[best] = 1;
+    selected[k] = (int32_t)best;
+  }
+  /* hysteresis */
+  for (int64_t m = 0; m < M; ++m) {
+    if (chosen[m]) {
+      idle[m] = 0;
+    } else if (idle[m] >= 0) {
+      idle[m] += 1;
+      if (idle[m] >= release_after) idle[m] = -1;
+    }
+  }
+  /* block residency, releases, then fetches into the lowest free slots */
+  const int64_t q = chunk_len / stride;
+  int st = 0;
+  *n_fetch = 0;
+  *n_release = 0;
+  char* resident = (char*)calloc((size_t)(nb > 0 ? nb : 1), 1);
+  for (int64_t m = 0; m < M; ++m)
+    if (idle[m] >= 0)
+      for (int64_t b = m; b < m + q && b < nb; ++b) resident[b] = 1;
+  for (int64_t b = 0; b < nb; ++b) {
+    if (block_slot[b] >= 0 && !resident[b]) {
+      release[2 * *n_release] = (int32_t)b;
+      release[2 * *n_release + 1] = block_slot[b];
+      ++*n_release;
+      slot_block[block_slot[b]] = -1;
+      block_slot[b] = -1;
+    }
+  }
+  for (int64_t b = 0; b < nb; ++b) {
+    if (resident[b] && block_slot[b] < 0) {
+      int slot = -1;
+      for (int k = 0; k < n_slots; ++k)
+        if (slot_block[k] < 0) {
+          slot = k;
+          break;
+        }
+      if (slot < 0) {
+        st = 1;
+        break;
+      }
+      slot_block[slot] = (int32_t)b;
+      block_slot[b] = slot;
+      fetch[2 * *n_fetch] = (int32_t)b;
+      fetch[2 * *n_fetch + 1] = slot;
+      ++*n_fetch;
+    }
+  }
+  free(resident);
+  free(chosen);
+  return st;
+}
