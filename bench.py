@@ -241,6 +241,7 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
+            torch.cuda._sleep(SPACER_CYCLES)  # the host enqueues the step meanwhile (outside the events)
             step_ev[i][0].record(stream)
             comp.compress(d_in["qwin"], d_in["K"], d_in["V"], d_in["S"], spikes=d_in.get("spikes"), stream=stream)
             step_ev[i][1].record(stream)
@@ -318,13 +319,20 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     if not args.no_next_rows:
-        res["next_rows"] = {"voxzip_pool": measure_voxzip(args, rank, world, dev, stream, flush)}
+        res["next_rows"] = {"voxzip_pool": measure_voxzip(args, rank, world, dev, stream, flush),
+                            "wnw_chunks_recall": measure_wnw(args, rank, world, dev, stream, flush)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(cfg, bt, args.cpu_rows)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+# A GPU-side wait of about 1 ms before each timed region, outside its events:
+# the host enqueues the region's launches meanwhile, so the events time the
+# kernels and not the host's launch gaps.
+SPACER_CYCLES = 2_000_000
 
 
 # ------------------------------------------------------- next rows (VoxZip) --
@@ -372,6 +380,7 @@ def measure_voxzip(args, rank, world, dev, stream, flush):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
+        torch.cuda._sleep(SPACER_CYCLES)
         ev[i][0].record(stream)
         call()
         ev[i][1].record(stream)
@@ -392,6 +401,87 @@ def measure_voxzip(args, rank, world, dev, stream, flush):
             "kernels": "vz_plan_kernel + vz_pool_kernel (kv_voxzip_pool)", "us_per_call": us,
             "rows_per_s": world * rows / (us * 1e-6), "bytes_alg": bytes_alg, "gbs": gbs, "peak": peak,
             "frac": gbs / peak, "peak_kind": kind + " (hbm_gbs copy)", "launches_per_call": 2}
+
+
+# ---------------------------------------------------------- next rows (WnW) --
+WNW_L, WNW_ANCHOR, WNW_TIDAL, WNW_D, WNW_STEPS = 32768, 5, 235, 128, 32
+
+
+def measure_wnw(args, rank, world, dev, stream, flush):
+    """kv_wnw_update + kv_wnw_recall over 32 decode steps of one 32768-row
+    audio (about 44 min at 12.5 rows/s) with 5 anchor and 235 tidal KV rows
+    (d = 128, bf16), 4 s / 2 s chunks, top 3, released after 3 steps. The
+    tidal rows' full copy is pinned host memory; the recall reads it over the
+    host link. Its peak is a plain pinned host-to-device copy measured here."""
+    import torch
+
+    import kv_cache_compression_layer_b200 as kv
+    from kv_cache_compression_layer_b200.replicas import max_over_ranks, replica_seed
+
+    p = kv.make_wnw_params()
+    Ls = [WNW_L]
+    seed = replica_seed(23, rank)
+    att = synth.anchor_attention(seed, WNW_L, WNW_ANCHOR, args.warmup + WNW_STEPS)
+    att_dev = torch.from_numpy(att).to(dev)
+    # host copies (2 x 2 GB, pinned): a seeded 64 MB random block, tiled
+    g = torch.Generator()
+    g.manual_seed(seed)
+    tile = 1 << 18
+    base = torch.randn(2 * tile, WNW_D, generator=g).to(torch.bfloat16)
+    K_h = torch.empty(WNW_TIDAL * WNW_L, WNW_D, dtype=torch.bfloat16, pin_memory=True)
+    V_h = torch.empty(K_h.shape, dtype=torch.bfloat16, pin_memory=True)
+    for i, r0 in enumerate(range(0, K_h.shape[0], tile)):
+        n = min(tile, K_h.shape[0] - r0)
+        K_h[r0:r0 + n] = base[(i % 2) * tile:(i % 2) * tile + n]
+        V_h[r0:r0 + n] = base[((i + 1) % 2) * tile:((i + 1) % 2) * tile + n]
+    S, cap = p.chunk_stride, p.top_c * (p.chunk_len // p.chunk_stride)
+    K_g = torch.zeros(WNW_TIDAL * p.n_slots * S, WNW_D, dtype=torch.bfloat16, device=dev)
+    V_g = torch.zeros_like(K_g)
+    state = torch.empty(kv.kv_wnw_state_ints(Ls, p), dtype=torch.int32, device=dev)
+    score = torch.empty(kv.kv_wnw_chunk_count(Ls, p), dtype=torch.float64, device=dev)
+    fetch = torch.empty(1, cap, 2, dtype=torch.int32, device=dev)
+    release = torch.empty_like(fetch)
+    counts = torch.empty(1, 2, dtype=torch.int32, device=dev)
+    kv.kv_wnw_init(Ls, p, state, stream=stream)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for t in range(args.warmup):
+        kv.kv_wnw_update(Ls, p, WNW_ANCHOR, att_dev[t], state, score, fetch, release, counts, stream=stream)
+        kv.kv_wnw_recall(Ls, p, WNW_TIDAL, WNW_D, kv.KV_BF16, fetch, counts, K_h, V_h, K_g, V_g, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(E(), E(), E()) for _ in range(WNW_STEPS)]
+    fetched = 0
+    for i in range(WNW_STEPS):
+        t = args.warmup + i
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(SPACER_CYCLES)
+        ev[i][0].record(stream)
+        kv.kv_wnw_update(Ls, p, WNW_ANCHOR, att_dev[t], state, score, fetch, release, counts, stream=stream)
+        ev[i][1].record(stream)
+        kv.kv_wnw_recall(Ls, p, WNW_TIDAL, WNW_D, kv.KV_BF16, fetch, counts, K_h, V_h, K_g, V_g, stream=stream)
+        ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        fetched += int(counts[0, 0].item())  # blocks recalled this step (read outside the events)
+    upd_us = max_over_ranks(1e3 * sum(a.elapsed_time(b) for a, b, _ in ev) / WNW_STEPS, world, dev)
+    rec_us = max_over_ranks(1e3 * sum(b.elapsed_time(c) for _, b, c in ev) / WNW_STEPS, world, dev)
+    rec_bytes = fetched * WNW_TIDAL * 2 * S * WNW_D * 2 / WNW_STEPS  # per step, host read = HBM write
+    # the host link's measured copy bandwidth: one 256 MB pinned host-to-device copy
+    blob = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    dst.copy_(blob, non_blocking=True)
+    a, b = E(), E()
+    a.record(stream)
+    dst.copy_(blob, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    h2d_gbs = (256 << 20) / (a.elapsed_time(b) * 1e-3) / 1e9
+    rec_gbs = rec_bytes / (rec_us * 1e-6) / 1e9
+    return {"workload": f"1 seq x {WNW_L} audio rows, {WNW_ANCHOR} anchor + {WNW_TIDAL} tidal KV rows, d={WNW_D}, "
+                        f"bf16, chunks 4 s / 2 s at 12.5 rows/s, top 3, release after 3, {WNW_STEPS} steps",
+            "kernels": "wnw_score_kernel + wnw_update_kernel (kv_wnw_update), wnw_recall_kernel (kv_wnw_recall)",
+            "update_us_per_step": upd_us, "recall_us_per_step": rec_us, "recalled_blocks_per_step":
+            fetched / WNW_STEPS, "recall_bytes_per_step": rec_bytes, "recall_gbs": rec_gbs,
+            "h2d_copy_gbs_measured": h2d_gbs, "recall_frac_of_h2d_copy": rec_gbs / h2d_gbs,
+            "launches_per_step": 3}
 
 
 # ------------------------------------------------------------ reference arm --

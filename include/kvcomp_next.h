@@ -7,6 +7,11 @@
  *        audio feature rows ("VoxZip: Semantic-Anchored Temporal KV Cache
  *        Compression for Long-Context Audio Inference", 方法概述和架构,
  *        first stage, steps one to three).
+ *   kv_wnw_update, kv_wnw_recall -> WnW's anchor-chunk importance with top-3
+ *        selection and release hysteresis, and the recall of the selected
+ *        chunks of the tidal heads from their full copy in host memory
+ *        ("WnW: Waxing-and-Waning KV Cache for Long-Form Speech LLMs",
+ *        方法概述和架构 and 细节详述).
  */
 #ifndef KVCOMP_NEXT_H
 #define KVCOMP_NEXT_H
@@ -75,6 +80,100 @@ int kv_voxzip_pool(const int32_t* L_a, int32_t n_seq, const double* tau_total, c
                    int32_t dtype, float conf_min, const kv_asr_segment* segs, const void* E_A, const void* E_T,
                    int64_t n_text_rows, void* E_comp, int32_t* src, int32_t* out_len, int32_t* status,
                    void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* WnW anchor chunks and tidal recall                                        */
+/* ------------------------------------------------------------------------ */
+#define KV_WNW_MAX_L (1 << 20)     /* audio rows per sequence             */
+#define KV_WNW_MAX_TOP 8           /* chunks selected per step            */
+#define KV_WNW_MAX_SLOTS 1024      /* block slots per (sequence, tidal row) */
+#define KV_WNW_MAX_CHUNK 12288     /* rows per chunk                      */
+
+/* The chunk rule, named as on the WnW page (4 s chunks every 2 s, top 3,
+ * released after 3 unselected steps), in audio rows. */
+typedef struct {
+  int32_t chunk_len;     /* C: rows per chunk (4 s of audio), <= KV_WNW_MAX_CHUNK */
+  int32_t chunk_stride;  /* S: rows between chunk starts (2 s); C % S == 0      */
+  int32_t top_c;         /* chunks selected per step, 1..KV_WNW_MAX_TOP (3)     */
+  int32_t release_after; /* unselected steps in a row before a chunk leaves (3) */
+  int32_t n_slots;       /* block slots of the GPU copy per (sequence, tidal
+                            row): top_c * release_after * C / S ..
+                            KV_WNW_MAX_SLOTS                                    */
+} kv_wnw_params;
+
+/* Chunks of a sequence of L rows: M = 1 when L <= C, else ceil((L - C) / S) + 1;
+ * chunk m covers rows [m S, min(m S + C, L)). Blocks: nb = ceil(L / S), block b
+ * covers rows [b S, min((b + 1) S, L)); chunk m holds blocks m .. m + C/S - 1
+ * (those below nb).
+ * kv_wnw_chunk_count: sum of M over the batch; kv_wnw_state_ints: int32 words
+ * of the state (per sequence: idle [M], block_slot [nb], slot_block [n_slots]).
+ * Both return -1 on invalid arguments. */
+int64_t kv_wnw_chunk_count(const int32_t* L, int32_t n_seq, const kv_wnw_params* p);
+int64_t kv_wnw_state_ints(const int32_t* L, int32_t n_seq, const kv_wnw_params* p);
+
+/* Sets every chunk and block of `state` (device, kv_wnw_state_ints words) to
+ * "not resident" (-1). Errors: KV_ERR_ARG, KV_ERR_CUDA. */
+int kv_wnw_init(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32_t* state, void* stream);
+
+/*
+ * kv_wnw_update — one decode step of WnW's anchor-chunk rule for every
+ * sequence (WnW, 方法概述和架构: anchor attention summed into time-chunk
+ * importance, top 3 chunks recalled; 细节详述: 4 s / 2 s chunks, released
+ * after 3 unselected steps in a row):
+ *   score_m = sum over anchor rows a, then over rows j of chunk m, of s[a][j]
+ *             (float64, in that order);
+ *   the top_c largest scores are selected (ties to the lower chunk; every
+ *   chunk when M <= top_c); a selected chunk's idle count becomes 0, a
+ *   resident unselected chunk's count grows by 1 and the chunk leaves when it
+ *   reaches release_after;
+ *   a block is resident while a resident chunk holds it; blocks that stop
+ *   being resident free their slots (release list), then the blocks that
+ *   become resident take the lowest free slots in ascending block order
+ *   (fetch list).
+ * Arguments:
+ *   L        host [n_seq]: audio rows per sequence, 1..KV_WNW_MAX_L.
+ *   n_anchor anchor rows (KV heads) per sequence, 1..1024.
+ *   s        device [sum_s n_anchor * L[s]] float32: sequence s's anchors one
+ *            after another, each L[s] long: the step's attention mass of the
+ *            anchor row on every audio row (e.g. summed over its query heads).
+ *   state    device, kv_wnw_state_ints words (updated).
+ *   score    device [kv_wnw_chunk_count] float64 (output): sequence after
+ *            sequence.
+ *   fetch    device [n_seq][top_c * C / S][2] int32 (output): (block, slot)
+ *            pairs, first counts[s][0] valid.
+ *   release  device [n_seq][top_c * C / S][2] int32 (output): (block, old
+ *            slot) pairs, first counts[s][1] valid.
+ *   counts   device [n_seq][2] int32 (output).
+ * Errors: KV_ERR_ARG, KV_ERR_CUDA.
+ */
+int kv_wnw_update(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32_t n_anchor, const float* s,
+                  int32_t* state, double* score, int32_t* fetch, int32_t* release, int32_t* counts, void* stream);
+
+/*
+ * kv_wnw_recall — copies the blocks of the fetch lists of kv_wnw_update from
+ * the tidal rows' full K/V copies in host memory into their GPU copies (WnW,
+ * 方法概述和架构: tidal heads keep the full KV on the CPU and hold only the
+ * recalled chunks on the GPU). One kernel reads the host memory directly
+ * (pinned, mapped) with 16-byte loads; the caller picks the stream, so the
+ * copy can run beside the decode step.
+ *   L, n_seq, p        as kv_wnw_update.
+ *   n_tidal            tidal rows per sequence, >= 1.
+ *   d, dtype           row width (d * element size a multiple of 16 bytes) and
+ *                      KV_BF16 or KV_F32.
+ *   fetch, counts      device, from kv_wnw_update.
+ *   K_host, V_host     pinned host memory (cudaHostAlloc or registered),
+ *                      [sum_s n_tidal * L[s]][d]: sequence s's tidal rows one
+ *                      after another, each L[s] long.
+ *   K_gpu, V_gpu       device [n_seq * n_tidal * n_slots * S][d]: slot k of
+ *                      tidal row r of sequence s starts at row
+ *                      ((s * n_tidal + r) * n_slots + k) * S; a short last
+ *                      block leaves the rest of its slot untouched.
+ * Errors: KV_ERR_ARG (also when K_host or V_host is not pinned host memory),
+ * KV_ERR_CUDA.
+ */
+int kv_wnw_recall(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32_t n_tidal, int32_t d, int32_t dtype,
+                  const int32_t* fetch, const int32_t* counts, const void* K_host, const void* V_host, void* K_gpu,
+                  void* V_gpu, void* stream);
 
 #ifdef __cplusplus
 }

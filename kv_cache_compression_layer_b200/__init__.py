@@ -27,13 +27,19 @@ META_INTS = 8
 EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes", "kv_allocate_global",
-           "kv_select_gather_segmented", "kv_voxzip_pool")
+           "kv_select_gather_segmented", "kv_voxzip_pool", "kv_wnw_chunk_count", "kv_wnw_state_ints",
+           "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class kv_shape(C.Structure):
     _fields_ = [("n_layers", C.c_int32), ("n_kv_heads", C.c_int32), ("group", C.c_int32), ("head_dim", C.c_int32),
                 ("w", C.c_int32), ("dtype", C.c_int32)]
+
+
+class kv_wnw_params(C.Structure):
+    _fields_ = [("chunk_len", C.c_int32), ("chunk_stride", C.c_int32), ("top_c", C.c_int32),
+                ("release_after", C.c_int32), ("n_slots", C.c_int32)]
 
 
 class kv_params(C.Structure):
@@ -65,6 +71,7 @@ def lib():
         L = C.CDLL(LIB_PATH)
         P, I32, SZ, I64 = C.c_void_p, C.c_int32, C.c_size_t, C.c_int64
         Ps, Pp, Pc = C.POINTER(kv_shape), C.POINTER(kv_params), C.POINTER(kv_cache)
+        Pw = C.POINTER(kv_wnw_params)
         sig = {
             "kv_rows": (I64, [Ps, I32]),
             "kv_check_lengths": (C.c_int, [Ps, P, I32]),
@@ -83,6 +90,11 @@ def lib():
             "kv_score_noalloc": (C.c_int, [Ps, P, I32, P, P, P, P]),
             "kv_decode_scratch_bytes": (SZ, [Ps, P, I32, Pp, I64]),
             "kv_voxzip_pool": (C.c_int, [P, I32, P, P, I32, I32, C.c_float, P, P, P, I64, P, P, P, P, P]),
+            "kv_wnw_chunk_count": (I64, [P, I32, Pw]),
+            "kv_wnw_state_ints": (I64, [P, I32, Pw]),
+            "kv_wnw_init": (C.c_int, [P, I32, Pw, P, P]),
+            "kv_wnw_update": (C.c_int, [P, I32, Pw, I32, P, P, P, P, P, P, P]),
+            "kv_wnw_recall": (C.c_int, [P, I32, Pw, I32, I32, I32, P, P, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -254,6 +266,43 @@ def kv_voxzip_pool(L_a, tau_total, seg_off, d, dtype, segs, E_A, E_T, n_text_row
                                 _stream(stream)))
 
 
+def make_wnw_params(chunk_len: int = 50, chunk_stride: int = 25, top_c: int = 3, release_after: int = 3,
+                    n_slots: Optional[int] = None) -> kv_wnw_params:
+    """WnW's chunk rule in audio rows (defaults: 4 s / 2 s at 12.5 rows/s, top 3, 3 steps);
+    n_slots defaults to the bound top_c * release_after * chunk_len / chunk_stride."""
+    if n_slots is None:
+        n_slots = top_c * release_after * (chunk_len // max(1, chunk_stride))
+    return kv_wnw_params(chunk_len, chunk_stride, top_c, release_after, n_slots)
+
+
+def kv_wnw_chunk_count(L, p: kv_wnw_params) -> int:
+    arr, n = _L(L)
+    return lib().kv_wnw_chunk_count(arr, n, C.byref(p))
+
+
+def kv_wnw_state_ints(L, p: kv_wnw_params) -> int:
+    arr, n = _L(L)
+    return lib().kv_wnw_state_ints(arr, n, C.byref(p))
+
+
+def kv_wnw_init(L, p, state, stream=None):
+    arr, n = _L(L)
+    _check("kv_wnw_init", lib().kv_wnw_init(arr, n, C.byref(p), _ptr(state), _stream(stream)))
+
+
+def kv_wnw_update(L, p, n_anchor, s, state, score, fetch, release, counts, stream=None):
+    arr, n = _L(L)
+    _check("kv_wnw_update", lib().kv_wnw_update(arr, n, C.byref(p), int(n_anchor), _ptr(s), _ptr(state), _ptr(score),
+                                                _ptr(fetch), _ptr(release), _ptr(counts), _stream(stream)))
+
+
+def kv_wnw_recall(L, p, n_tidal, d, dtype, fetch, counts, K_host, V_host, K_gpu, V_gpu, stream=None):
+    arr, n = _L(L)
+    _check("kv_wnw_recall", lib().kv_wnw_recall(arr, n, C.byref(p), int(n_tidal), int(d), int(dtype), _ptr(fetch),
+                                                _ptr(counts), _ptr(K_host), _ptr(V_host), _ptr(K_gpu), _ptr(V_gpu),
+                                                _stream(stream)))
+
+
 def kv_read_device_status(status_dev, stream=None) -> int:
     host = C.c_int32(0)
     _check("kv_read_device_status", lib().kv_read_device_status(_ptr(status_dev), C.byref(host), _stream(stream)))
@@ -267,5 +316,6 @@ __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", 
            "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "kv_voxzip_pool",
-           "pack_segments", "ASR_SEGMENT_BYTES", "status_string",
+           "pack_segments", "ASR_SEGMENT_BYTES", "kv_wnw_params", "make_wnw_params", "kv_wnw_chunk_count",
+           "kv_wnw_state_ints", "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "status_string",
            "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]

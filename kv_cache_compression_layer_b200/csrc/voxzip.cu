@@ -9,11 +9,11 @@
 // (first row, row count, text row) descriptor per output row; the whole CTA
 // writes the gap after the last segment.
 //
-// pool kernel (persistent, all SMs): a warp owns a 1 KB slice of one output
-// row, reads the slice of each of the row's source rows with 16-byte loads
-// (two rows, four pieces a lane, in flight), sums in float32 in row order,
-// divides once, adds the text embedding and rounds once. Copied rows are
-// exact.
+// pool kernel (persistent, one wave of resident CTAs): a warp owns a 1 KB
+// slice of one output row, reads the slice of each of the row's source rows
+// with 16-byte loads (two rows, four pieces a lane, in flight), sums in
+// float32 in row order, divides once, adds the text embedding and rounds
+// once. Copied rows are exact.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -374,14 +374,19 @@ extern "C" int kv_voxzip_pool(const int32_t* L_a, int32_t n_seq, const double* t
   const int slices = (d * esz + kSliceBytes - 1) / kSliceBytes;
   const long long units = rows * slices;
   const long long want = (units * 32 + kPoolThreads - 1) / kPoolThreads;
-  const int grid = (int)std::max(1ll, std::min<long long>(want, (long long)sm_count() * 8));
+  // one wave: as many CTAs as are resident at once (no tail of late CTAs)
+  auto grid_of = [&](const void* kernel) {
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPoolThreads, 0);
+    return (int)std::max(1ll, std::min<long long>(want, (long long)sm_count() * std::max(1, per_sm)));
+  };
   if (dtype == KV_BF16)
-    vz_pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, st>>>(
+    vz_pool_kernel<__nv_bfloat16><<<grid_of((const void*)vz_pool_kernel<__nv_bfloat16>), kPoolThreads, 0, st>>>(
         m, d, slices, units, static_cast<const __nv_bfloat16*>(E_A), static_cast<const __nv_bfloat16*>(E_T),
         E_T ? 1 : 0, static_cast<__nv_bfloat16*>(E_comp), src, out_len);
   else
-    vz_pool_kernel<float><<<grid, kPoolThreads, 0, st>>>(m, d, slices, units, static_cast<const float*>(E_A),
-                                                         static_cast<const float*>(E_T), E_T ? 1 : 0,
-                                                         static_cast<float*>(E_comp), src, out_len);
+    vz_pool_kernel<float><<<grid_of((const void*)vz_pool_kernel<float>), kPoolThreads, 0, st>>>(
+        m, d, slices, units, static_cast<const float*>(E_A), static_cast<const float*>(E_T), E_T ? 1 : 0,
+        static_cast<float*>(E_comp), src, out_len);
   return cuda_status(cudaGetLastError());
 }

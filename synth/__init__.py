@@ -32,6 +32,12 @@ pages (AudioKV, VoxZip, WnW, C3); no dataset is read or reproduced:
   0.3 cut), 3 text tokens per second of speech (at least 1), text rows laid
   out segment after segment; features ``E_A ~ N(0, 1)``, text embeddings
   ``E_T ~ N(0, 0.02)`` (standard deviation).
+* anchor attention for the WnW row (``anchor_attention``): per step and
+  anchor row a mass of g (the query heads of the KV head) spread as 10% over
+  the first tenth of the audio (the sink), 60% in a Gaussian bump of 25 rows
+  (2 s) around a focus that walks through the audio with the decode step
+  (jittered per anchor by U{-50..50} rows), 30% uniform, times U(0.5, 1.5)
+  noise per row before normalising.
 
 Values are drawn in float32 and rounded to nearest-even bfloat16 for the
 bf16 workloads; the returned float32 arrays hold those bf16-exact values.
@@ -48,7 +54,7 @@ from scipy.signal import lfilter
 # tensor ids of the counter-based streams
 _T_KEYS, _T_PROJ, _T_KNOISE, _T_VALUES, _T_QWIN, _T_QDEC, _T_VDEC, _T_SPIKE = range(8)
 _T_HEADSCORES = 100
-_T_ASR, _T_FEAT, _T_TEXT = 200, 201, 202
+_T_ASR, _T_FEAT, _T_TEXT, _T_ANCHOR = 200, 201, 202, 203
 
 
 @dataclasses.dataclass(frozen=True)
@@ -343,6 +349,24 @@ def text_embeddings(seed: int, n: int, d: int, bf16: bool = True) -> np.ndarray:
     return round_bf16(x) if bf16 else x
 
 
+def anchor_attention(seed: int, L: int, n_anchor: int, steps: int, g: int = 4) -> np.ndarray:
+    """[steps][n_anchor][L] float32 attention mass of the anchor rows, each summing to g."""
+    rng = np.random.Generator(np.random.Philox(key=[seed, _T_ANCHOR]))
+    out = np.empty((steps, n_anchor, L), np.float32)
+    x = np.arange(L, dtype=np.float64)
+    sink = np.where(x < max(1, L // 10), 1.0, 0.0)
+    sink /= sink.sum()
+    for t in range(steps):
+        focus = (t + 0.5) * L / steps
+        for a in range(n_anchor):
+            c = focus + rng.integers(-50, 51)
+            bump = np.exp(-0.5 * ((x - c) / 25.0) ** 2)
+            bump /= max(bump.sum(), 1e-300)
+            p = (0.1 * sink + 0.6 * bump + 0.3 / L) * rng.uniform(0.5, 1.5, L)
+            out[t, a] = (g * p / p.sum()).astype(np.float32)
+    return out
+
+
 def small(cfg_name: str, **kw) -> Config:
     """A reduced copy of a named workload (fewer layers / shorter audio) for fast tests."""
     return CONFIGS[cfg_name].with_(**kw)
@@ -350,4 +374,5 @@ def small(cfg_name: str, **kw) -> Config:
 
 __all__ = ["Config", "CONFIGS", "Row", "Batch", "make_row", "make_batch", "keys", "values",
            "window_queries", "decode_queries", "head_scores", "spike_mask", "round_bf16",
-           "to_bf16_bits", "small", "AsrSegments", "asr_segments", "audio_features", "text_embeddings"]
+           "to_bf16_bits", "small", "AsrSegments", "asr_segments", "audio_features", "text_embeddings",
+           "anchor_attention"]

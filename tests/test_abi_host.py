@@ -121,6 +121,27 @@ def test_voxzip_argument_errors_launch_nothing(L):
     assert len(kv.pack_segments([(0.0, 1.0)], [0.5], [1], [0])) == kv.ASR_SEGMENT_BYTES
 
 
+def test_wnw_argument_errors_launch_nothing(L):
+    p = kv.make_wnw_params()
+    assert kv.kv_wnw_chunk_count([110], p) == 4 and kv.kv_wnw_state_ints([110], p) == 4 + 5 + 18
+    assert kv.kv_wnw_chunk_count([50], p) == 1 and kv.kv_wnw_chunk_count([51], p) == 2
+    for bad in (kv.kv_wnw_params(50, 30, 3, 3, 18), kv.kv_wnw_params(50, 25, 3, 3, 17),
+                kv.kv_wnw_params(50, 25, 9, 3, 54), kv.kv_wnw_params(50, 25, 3, 0, 18),
+                kv.kv_wnw_params(50, 0, 3, 3, 18), kv.kv_wnw_params(50, 25, 3, 3, 1025)):
+        assert kv.kv_wnw_chunk_count([110], bad) == -1
+    Larr = (C.c_int32 * 1)(1000)
+    st = L.kv_wnw_update(Larr, 1, C.byref(p), 0, 16, 16, 16, 16, 16, 16, None)  # no anchors
+    assert st == kv.KV_ERR_ARG
+    st = L.kv_wnw_update(Larr, 1, C.byref(p), 5, 16, 16, 20, 16, 16, 16, None)  # misaligned float64 scores
+    assert st == kv.KV_ERR_ARG
+    host = (C.c_uint8 * 4096)()  # pageable memory is refused before any launch
+    addr = (C.addressof(host) + 15) // 16 * 16
+    st = L.kv_wnw_recall(Larr, 1, C.byref(p), 2, 128, kv.KV_BF16, 16, 16, addr, addr, 4096, 8192, None)
+    assert st == kv.KV_ERR_ARG
+    st = L.kv_wnw_recall(Larr, 1, C.byref(p), 2, 4, kv.KV_BF16, 16, 16, addr, addr, 4096, 8192, None)  # 8 B rows
+    assert st == kv.KV_ERR_ARG
+
+
 def test_fault_injection_env(L, monkeypatch):
     sh = _shape()
     Larr = (C.c_int32 * 1)(6000)
