@@ -72,6 +72,14 @@ def _get():
             lib.orc_wnw_chunks.restype = I64
             lib.orc_wnw_step.argtypes = [I64, I32, P, I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P]
             lib.orc_wnw_step.restype = I32
+            lib.orc_splitmix64.argtypes = [C.c_uint64, C.c_uint64]
+            lib.orc_splitmix64.restype = C.c_uint64
+            lib.orc_c3_build.argtypes = [I64, I32, P, I32, I32, C.c_uint64, P, P, P, P, P, P, P]
+            lib.orc_c3_build.restype = I64
+            lib.orc_c3_frontier.argtypes = [I64, I64, I32, P, P, P]
+            lib.orc_c3_frontier.restype = I64
+            lib.orc_c3_step.argtypes = [I64, I32, I32, P, P, P, I64, P, P, P, P, P, I64, P, P, I64, D, I32, P, P, P]
+            lib.orc_c3_step.restype = I64
             lib.orc_decode_run_heads.argtypes = [I64, P, I32, I32, P, P, P, P, P, I64, P, P, P, P, D, I32, P, P,
                                                  P, P, I32]
             _lib = lib
@@ -371,5 +379,55 @@ class WnwState:
         return score, sel[:min(self.top_c, self.M)].copy(), fetch[:nf.value].copy(), release[:nr.value].copy()
 
 
-__all__ = ["WnwState", "voxzip_pool", "build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
+# ---------------------------------------------------------- next row: C3 ----
+def splitmix64(seed: int, k: int) -> int:
+    """Output k (from 0) of SplitMix64 seeded with `seed` (Steele, Lea and Flood, 2014)."""
+    return int(_get().orc_splitmix64(seed, k))
+
+
+class C3Row:
+    """One (layer, KV head) row of C3 ("C3: Speech-Guided KV Retrieval for
+    Long-Context SpeechLLM Inference"): the bisecting 2-means index of its keys,
+    the active frontier and its relevance EMA; `step` scores the frontier by the
+    group's best cosine, retrieves up to B keys cluster by cluster, attends
+    exactly, updates the EMA and runs R split/merge exchanges."""
+
+    def __init__(self, K: np.ndarray, V: np.ndarray, leaf_max: int = 4, iters: int = 8, seed: int = 0,
+                 granularity: int = 16):
+        self.K = _c(K, np.float32)
+        self.V = _c(V, np.float32)
+        L, d = self.K.shape
+        self.L, self.d = L, d
+        n = max(2 * L, 2)
+        self.perm = np.zeros(max(L, 1), np.int32)
+        self.lo, self.cnt, self.left, self.parent, self.depth = (np.zeros(n, np.int32) for _ in range(5))
+        self.cent = np.zeros((n, d), np.float64)
+        self.n_nodes = int(_get().orc_c3_build(L, d, _p(self.K), leaf_max, iters, seed, _p(self.perm), _p(self.lo),
+                                               _p(self.cnt), _p(self.left), _p(self.parent), _p(self.depth),
+                                               _p(self.cent)))
+        front = np.zeros(max(self.n_nodes, 1), np.int32)
+        self.A = int(_get().orc_c3_frontier(self.n_nodes, L, granularity, _p(self.left), _p(self.depth), _p(front)))
+        self.front = front[:self.A].copy()
+        self.e = np.zeros(self.n_nodes, np.float64)
+
+    def members(self, node: int) -> np.ndarray:
+        return self.perm[self.lo[node]:self.lo[node] + self.cnt[node]]
+
+    def step(self, q: np.ndarray, B: int, lam: float = 0.5, R: int = 2):
+        """q [G][d]. Returns (o [G][d] float64, selected positions, sigma of the frontier at entry)."""
+        q = _c(q, np.float32)
+        G = q.shape[0]
+        sigma = np.zeros(max(self.A, 1), np.float64)
+        sel = np.zeros(max(self.L, 1), np.int32)
+        o = np.zeros((G, self.d), np.float64)
+        front = self.front.copy()
+        n = _get().orc_c3_step(self.L, self.d, G, _p(self.K), _p(self.V), _p(q), self.n_nodes, _p(self.perm),
+                               _p(self.lo), _p(self.cnt), _p(self.left), _p(self.cent), self.A, _p(front),
+                               _p(self.e), int(B), float(lam), int(R), _p(sigma), _p(sel), _p(o))
+        sig = sigma[:self.A].copy()
+        self.front = front
+        return o, sel[:n].copy(), sig
+
+
+__all__ = ["splitmix64", "C3Row", "WnwState", "voxzip_pool", "build", "score", "rdft", "kstar", "irdft_lowpass", "sss", "allocate", "BudgetError", "select",
            "gather", "DecodeList", "recent_count", "decode_run_heads", "default_threads"]

@@ -854,3 +854,255 @@ int orc_wnw_step(int64_t L, int n_anchor, const float* s, int chunk_len, int str
   free(chosen);
   return st;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Next row: [C3] ("C3: Speech-Guided KV Retrieval for Long-Context SpeechLLM */
+/* Inference"), the key-space index, shared-GQA competition and adaptive     */
+/* resolution, per (layer, KV head) row of L audio keys K [L][d]:            */
+/*  - prefill: recursive bisecting 2-means over the keys (8 iterations per    */
+/*    split, seed 0); every node's centroid is the mean of its keys;          */
+/*  - the active frontier starts at the cut of mean node size about 16 and    */
+/*    always partitions the L positions;                                      */
+/*  - step t: sigma_n = max over the G query heads of cos(q_g, c_n); clusters */
+/*    in descending sigma give their keys until B are taken; exact attention  */
+/*    over those keys; e_n = lambda e_n + (1 - lambda) sigma_n; R exchanges,  */
+/*    each splitting the highest-e node into its children (which inherit e)   */
+/*    and merging the lowest sibling pair into its parent (max of the two).   */
+/* READINGS: a node with more than leaf_max (4) keys is split; the 2-means    */
+/* starts from two distinct member keys picked by SplitMix64 (outputs 2n and  */
+/* 2n + 1 of the generator seeded with `seed`, n = node id), assigns by       */
+/* squared Euclidean distance (ties to the left child) and recomputes means  */
+/* (an empty side keeps its centroid), 8 times; a split that leaves a side    */
+/* empty falls back to halving the members; node ids are given breadth-first  */
+/* (a split node's children get the next two ids); a node's members, in      */
+/* index order, are its left child's then its right child's (a leaf's in     */
+/* ascending position): centroids sum in that order, and a cluster that does  */
+/* not fit the budget gives its first members in it. The initial frontier is */
+/* every node at depth D0 = round(log2(L / granularity)) (the largest D with  */
+/* (granularity 2^D)^2 <= 2 L^2) plus the leaves above it. Cosine with a zero */
+/* vector is 0. Clusters are ranked by sigma, ties to the lower node id. e    */
+/* starts at 0. An exchange picks the split node by largest e (ties to the    */
+/* lower id) among frontier nodes with children, and the merge pair by        */
+/* smallest max(e) (ties to the lower parent id) among sibling pairs both on  */
+/* the frontier and not containing the split node; nodes created earlier in   */
+/* the same step are not candidates; an exchange without both candidates is   */
+/* skipped. L <= B bypasses retrieval (all keys, no update).                  */
+/* ------------------------------------------------------------------------- */
+uint64_t orc_splitmix64(uint64_t seed, uint64_t k) {
+  uint64_t z = seed + (k + 1) * 0x9e3779b97f4a7c15ull;
+  z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
+  z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
+  return z ^ (z >> 31);
+}
+
+/* The tree: node n owns perm[lo[n] .. lo[n] + cnt[n]) (positions, index order), */
+/* children left[n], left[n] + 1 (or -1), parent[n], depth[n], centroid        */
+/* cent[n][d]. Arrays sized 2 L. Returns the node count.                       */
+int64_t orc_c3_build(int64_t L, int d, const float* K, int leaf_max, int iters, uint64_t seed, int32_t* perm,
+                     int32_t* lo, int32_t* cnt, int32_t* left, int32_t* parent, int32_t* depth, double* cent) {
+  for (int64_t j = 0; j < L; ++j) perm[j] = (int32_t)j;
+  int64_t n_nodes = 1;
+  lo[0] = 0;
+  cnt[0] = (int32_t)L;
+  parent[0] = -1;
+  depth[0] = 0;
+  int32_t* side = (int32_t*)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
+  int32_t* tmp = (int32_t*)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
+  double* c = (double*)malloc(sizeof(double) * 2 * (size_t)d);
+  double* acc = (double*)malloc(sizeof(double) * 2 * (size_t)d);
+  for (int64_t nd = 0; nd < n_nodes; ++nd) { /* breadth first: children are appended */
+    left[nd] = -1;
+    const int32_t n = cnt[nd];
+    const int32_t* m = perm + lo[nd];
+    if (n <= leaf_max || n < 2) continue;
+    const int64_t i0 = (int64_t)(orc_splitmix64(seed, 2 * (uint64_t)nd) % (uint64_t)n);
+    const int64_t i1 = (i0 + 1 + (int64_t)(orc_splitmix64(seed, 2 * (uint64_t)nd + 1) % (uint64_t)(n - 1))) % n;
+    for (int k = 0; k < d; ++k) {
+      c[k] = K[(size_t)m[i0] * d + k];
+      c[d + k] = K[(size_t)m[i1] * d + k];
+    }
+    for (int it = 0; it < iters; ++it) {
+      int64_t n1 = 0;
+      for (int32_t j = 0; j < n; ++j) {
+        double d0 = 0.0, d1 = 0.0;
+        for (int k = 0; k < d; ++k) {
+          const double x = K[(size_t)m[j] * d + k];
+          d0 += (x - c[k]) * (x - c[k]);
+          d1 += (x - c[d + k]) * (x - c[d + k]);
+        }
+        side[j] = d1 < d0 ? 1 : 0;
+        n1 += side[j];
+      }
+      for (int k = 0; k < 2 * d; ++k) acc[k] = 0.0;
+      for (int32_t j = 0; j < n; ++j)
+        for (int k = 0; k < d; ++k) acc[side[j] * d + k] += K[(size_t)m[j] * d + k];
+      if (n - n1 > 0)
+        for (int k = 0; k < d; ++k) c[k] = acc[k] / (double)(n - n1);
+      if (n1 > 0)
+        for (int k = 0; k < d; ++k) c[d + k] = acc[d + k] / (double)n1;
+    }
+    int32_t n0 = 0;
+    for (int32_t j = 0; j < n; ++j) n0 += side[j] == 0;
+    if (n0 == 0 || n0 == n) { /* fall back to halving in position order */
+      n0 = (n + 1) / 2;
+      for (int32_t j = 0; j < n; ++j) side[j] = j >= n0;
+    }
+    int32_t a = 0, b = n0;
+    for (int32_t j = 0; j < n; ++j) tmp[side[j] ? b++ : a++] = m[j];
+    memcpy(perm + lo[nd], tmp, sizeof(int32_t) * (size_t)n);
+    const int64_t l = n_nodes, r = n_nodes + 1;
+    left[nd] = (int32_t)l;
+    lo[l] = lo[nd];
+    cnt[l] = n0;
+    lo[r] = lo[nd] + n0;
+    cnt[r] = n - n0;
+    parent[l] = parent[r] = (int32_t)nd;
+    depth[l] = depth[r] = depth[nd] + 1;
+    n_nodes += 2;
+  }
+  /* centroids: the mean of every node's keys, summed in index order */
+  for (int64_t nd = 0; nd < n_nodes; ++nd) {
+    for (int k = 0; k < d; ++k) {
+      double s = 0.0;
+      for (int32_t j = 0; j < cnt[nd]; ++j) s += K[(size_t)perm[lo[nd] + j] * d + k];
+      cent[(size_t)nd * d + k] = s / (double)cnt[nd];
+    }
+  }
+  free(acc);
+  free(c);
+  free(tmp);
+  free(side);
+  return n_nodes;
+}
+
+/* The initial frontier (node ids, ascending) into front; returns its size. */
+int64_t orc_c3_frontier(int64_t n_nodes, int64_t L, int granularity, const int32_t* left, const int32_t* depth,
+                        int32_t* front) {
+  int D0 = 0; /* the cut whose mean node size is nearest granularity (log scale) */
+  while (D0 < 40) {
+    const double next = (double)granularity * (double)((int64_t)1 << (D0 + 1));
+    if (next * next > 2.0 * (double)L * (double)L) break;
+    ++D0;
+  }
+  int64_t A = 0;
+  for (int64_t nd = 0; nd < n_nodes; ++nd)
+    if (depth[nd] == D0 || (depth[nd] < D0 && left[nd] < 0)) front[A++] = (int32_t)nd;
+  return A;
+}
+
+static double cosine(const double* a, const double* b, int d) {
+  double ab = 0.0, aa = 0.0, bb = 0.0;
+  for (int k = 0; k < d; ++k) {
+    ab += a[k] * b[k];
+    aa += a[k] * a[k];
+    bb += b[k] * b[k];
+  }
+  if (aa == 0.0 || bb == 0.0) return 0.0;
+  return ab / (sqrt(aa) * sqrt(bb));
+}
+
+/* One decode step of one row. front [A] and e [n_nodes] are updated.        */
+/* sigma [A] (scores of the frontier at entry, in its order), sel [min(B, L)] */
+/* (positions, ascending) and o [G][d] are outputs. Returns the number of     */
+/* selected positions.                                                        */
+int64_t orc_c3_step(int64_t L, int d, int G, const float* K, const float* V, const float* q, int64_t n_nodes,
+                    const int32_t* perm, const int32_t* lo, const int32_t* cnt, const int32_t* left,
+                    const double* cent, int64_t A, int32_t* front, double* e, int64_t B,
+                    double lambda, int R, double* sigma, int32_t* sel, double* o) {
+  int64_t n_sel = 0;
+  char* taken = (char*)calloc((size_t)(L > 0 ? L : 1), 1);
+  const int bypass = L <= B;
+  if (bypass) {
+    for (int64_t j = 0; j < L; ++j) taken[j] = 1;
+  } else {
+    double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t i = 0; i < A; ++i) {
+      double best = -INFINITY;
+      for (int g = 0; g < G; ++g) {
+        for (int k = 0; k < d; ++k) qv[k] = q[(size_t)g * d + k];
+        const double cs = cosine(qv, cent + (size_t)front[i] * d, d);
+        if (cs > best) best = cs;
+      }
+      sigma[i] = best;
+    }
+    free(qv);
+    /* clusters in descending sigma (ties: lower node id) give their keys */
+    char* used = (char*)calloc((size_t)(A > 0 ? A : 1), 1);
+    int64_t got = 0;
+    while (got < B) {
+      int64_t bi = -1;
+      for (int64_t i = 0; i < A; ++i)
+        if (!used[i] && (bi < 0 || sigma[i] > sigma[bi] || (sigma[i] == sigma[bi] && front[i] < front[bi]))) bi = i;
+      if (bi < 0) break;
+      used[bi] = 1;
+      const int32_t nd = front[bi];
+      /* a cluster that does not fit gives its first members in index order */
+      for (int32_t j = 0; j < cnt[nd] && got < B; ++j, ++got) taken[perm[lo[nd] + j]] = 1;
+    }
+    free(used);
+  }
+  for (int64_t j = 0; j < L; ++j)
+    if (taken[j]) sel[n_sel++] = (int32_t)j;
+  /* exact attention over the selected keys */
+  const double scale = 1.0 / sqrt((double)d);
+  double* lg = (double*)malloc(sizeof(double) * (size_t)(n_sel > 0 ? n_sel : 1));
+  for (int g = 0; g < G; ++g) {
+    double mx = -INFINITY;
+    for (int64_t i = 0; i < n_sel; ++i) {
+      double dot = 0.0;
+      for (int k = 0; k < d; ++k) dot += (double)q[(size_t)g * d + k] * (double)K[(size_t)sel[i] * d + k];
+      lg[i] = dot * scale;
+      if (lg[i] > mx) mx = lg[i];
+    }
+    double den = 0.0;
+    for (int64_t i = 0; i < n_sel; ++i) den += exp(lg[i] - mx);
+    for (int k = 0; k < d; ++k) {
+      double acc = 0.0;
+      for (int64_t i = 0; i < n_sel; ++i) acc += exp(lg[i] - mx) / den * (double)V[(size_t)sel[i] * d + k];
+      o[(size_t)g * d + k] = acc;
+    }
+  }
+  free(lg);
+  free(taken);
+  if (bypass) return n_sel;
+  /* relevance EMA of the frontier */
+  for (int64_t i = 0; i < A; ++i) e[front[i]] = lambda * e[front[i]] + (1.0 - lambda) * sigma[i];
+  /* R exchanges: split the most relevant node, merge the least relevant sibling pair */
+  char* on = (char*)calloc((size_t)n_nodes, 1);
+  char* fresh = (char*)calloc((size_t)n_nodes, 1);
+  for (int64_t i = 0; i < A; ++i) on[front[i]] = 1;
+  for (int r = 0; r < R; ++r) {
+    int64_t s = -1;
+    for (int64_t nd = 0; nd < n_nodes; ++nd)
+      if (on[nd] && !fresh[nd] && left[nd] >= 0 && (s < 0 || e[nd] > e[s])) s = nd;
+    if (s < 0) break;
+    int64_t p = -1;
+    double pv = 0.0;
+    for (int64_t nd = 0; nd < n_nodes; ++nd) {
+      if (left[nd] < 0) continue;
+      const int64_t a = left[nd], b = left[nd] + 1;
+      if (!on[a] || !on[b] || fresh[a] || fresh[b] || a == s || b == s) continue;
+      const double v = e[a] > e[b] ? e[a] : e[b];
+      if (p < 0 || v < pv) {
+        p = nd;
+        pv = v;
+      }
+    }
+    if (p < 0) break;
+    const int64_t c0 = left[s];
+    on[s] = 0;
+    on[c0] = on[c0 + 1] = 1;
+    fresh[c0] = fresh[c0 + 1] = 1;
+    e[c0] = e[c0 + 1] = e[s];
+    on[left[p]] = on[left[p] + 1] = 0;
+    on[p] = 1;
+    fresh[p] = 1;
+    e[p] = pv;
+  }
+  int64_t a = 0;
+  for (int64_t nd = 0; nd < n_nodes; ++nd)
+    if (on[nd]) front[a++] = (int32_t)nd;
+  free(fresh);
+  free(on);
+  return n_sel;
+}
