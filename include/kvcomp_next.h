@@ -12,6 +12,11 @@
  *        chunks of the tidal heads from their full copy in host memory
  *        ("WnW: Waxing-and-Waning KV Cache for Long-Form Speech LLMs",
  *        方法概述和架构 and 细节详述).
+ *   kv_c3_build, kv_c3_step -> C3's key-space index (bisecting 2-means),
+ *        shared-GQA cluster competition for a budget of B audio keys, exact
+ *        attention over them and adaptive resolution (relevance EMA with
+ *        split/merge exchanges) ("C3: Speech-Guided KV Retrieval for
+ *        Long-Context SpeechLLM Inference").
  */
 #ifndef KVCOMP_NEXT_H
 #define KVCOMP_NEXT_H
@@ -174,6 +179,92 @@ int kv_wnw_update(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32
 int kv_wnw_recall(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32_t n_tidal, int32_t d, int32_t dtype,
                   const int32_t* fetch, const int32_t* counts, const void* K_host, const void* V_host, void* K_gpu,
                   void* V_gpu, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* C3 key-space retrieval                                                    */
+/* ------------------------------------------------------------------------ */
+#define KV_C3_MAX_BUDGET 8192 /* B, at most */
+
+/* The method's settings, named as on the C3 page (defaults in brackets). */
+typedef struct {
+  int32_t leaf_max;    /* a node with more keys is split (4)                   */
+  int32_t iters;       /* 2-means iterations per split (8), 1..64              */
+  int32_t granularity; /* mean node size of the initial frontier (16), >= 4    */
+  int32_t budget;      /* B: audio keys retrieved per row and step, 1..KV_C3_MAX_BUDGET */
+  double lambda;       /* weight of the history in the relevance EMA (0.5)     */
+  int32_t exchanges;   /* R: split/merge exchanges per step (2), 0..64         */
+  int32_t reserved;    /* set to 0                                             */
+  uint64_t seed;       /* seed of the 2-means initialisation (0)               */
+} kv_c3_params;
+
+/* Where each array of a C3 index lives, as byte offsets into the index buffer.
+ * Per-key arrays hold row i at key offset koff_i (kvcomp.h's convention), per-
+ * node arrays at 2 * koff_i (a row has at most 2 L nodes), cent at
+ * 2 * koff_i * d; hdr is [rows][4] int32: node count, frontier size A,
+ * retrieved keys, 0. */
+typedef struct {
+  uint64_t perm;  /* int32 per key: positions in index order                   */
+  uint64_t lo;    /* int32 per node: first index of the node's members         */
+  uint64_t cnt;   /* int32 per node: members                                   */
+  uint64_t left;  /* int32 per node: left child (right = left + 1), or -1      */
+  uint64_t depth; /* int32 per node                                            */
+  uint64_t e;     /* float64 per node: relevance EMA                           */
+  uint64_t cent;  /* float64 per node x d: centroid                            */
+  uint64_t front; /* int32 per node: the frontier's node ids, ascending        */
+  uint64_t sigma; /* float64 per node: the last step's score of frontier entry */
+  uint64_t sel;   /* int32 per key: the last step's retrieved positions        */
+  uint64_t hdr;   /* int32 [rows][4]                                           */
+  uint64_t bytes; /* size of the whole index                                   */
+} kv_c3_layout;
+
+/* Layout of the index of a batch; KV_ERR_ARG on invalid arguments. */
+int kv_c3_index_layout(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_c3_params* p,
+                       kv_c3_layout* out);
+
+/*
+ * kv_c3_build — prefill: the key-space index of every row (C3, index built
+ * per layer and KV head by recursive bisecting k-means, 8 iterations, seed 0;
+ * initial frontier at mean granularity 16):
+ *   a node with more than leaf_max keys is split by 2-means (squared
+ *   Euclidean distance in float64, ties to the left child) started from two
+ *   distinct members picked by SplitMix64 (outputs 2n and 2n + 1 of the
+ *   generator seeded with `seed`, n = the node's id in its row); an empty side
+ *   keeps its centroid; a split that leaves a side empty halves the members;
+ *   node ids are breadth-first; a node's members, in index order, are its left
+ *   child's then its right child's (a leaf's in ascending position); its
+ *   centroid is their mean (float64, summed in index order); the frontier is
+ *   every node at depth round(log2(L / granularity)) plus the leaves above it;
+ *   every EMA starts at 0.
+ *   K      device [sum L][d] in shape->dtype (d = head_dim).
+ *   index  device, kv_c3_index_layout().bytes, 8-byte aligned.
+ * Runs one launch per tree level and synchronises `stream` after each (the
+ * level count depends on the data). Errors: KV_ERR_ARG, KV_ERR_UNSUPPORTED_L,
+ * KV_ERR_CUDA.
+ */
+int kv_c3_build(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_c3_params* p, const void* K,
+                void* index, void* stream);
+
+/*
+ * kv_c3_step — one decode step of every row (C3: shared-GQA competition over
+ * the frontier, exact attention over the retrieved keys, adaptive resolution):
+ *   sigma_n = max over the g query heads of cos(q_g, c_n) (float64);
+ *   frontier clusters in descending sigma (ties: lower node id) give their
+ *   members in index order until B keys are taken;
+ *   out_g = softmax(q_g K_sel^T / sqrt(d)) V_sel over the retrieved keys
+ *   (float32 accumulation);
+ *   e_n = lambda e_n + (1 - lambda) sigma_n on the frontier, then R exchanges:
+ *   the frontier node with children and the largest e (ties: lower id) is
+ *   replaced by its children (which take its e), and the sibling pair on the
+ *   frontier with the smallest max(e) (ties: lower parent id), not holding
+ *   that node, by its parent (which takes that max); nodes made in the same
+ *   step are not candidates; an exchange lacking either is skipped.
+ *   A row with L <= B attends over all its keys and keeps its state.
+ *   K, V   device [sum L][d]; q device [rows][g][d]; out device [rows][g][d],
+ *          all in shape->dtype. index from kv_c3_build (updated).
+ * Errors: KV_ERR_ARG, KV_ERR_UNSUPPORTED_L, KV_ERR_CUDA.
+ */
+int kv_c3_step(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_c3_params* p, const void* K,
+               const void* V, const void* q, void* index, void* out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -28,7 +28,7 @@ EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots"
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes", "kv_allocate_global",
            "kv_select_gather_segmented", "kv_voxzip_pool", "kv_wnw_chunk_count", "kv_wnw_state_ints",
-           "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall")
+           "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "kv_c3_index_layout", "kv_c3_build", "kv_c3_step")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -40,6 +40,16 @@ class kv_shape(C.Structure):
 class kv_wnw_params(C.Structure):
     _fields_ = [("chunk_len", C.c_int32), ("chunk_stride", C.c_int32), ("top_c", C.c_int32),
                 ("release_after", C.c_int32), ("n_slots", C.c_int32)]
+
+
+class kv_c3_params(C.Structure):
+    _fields_ = [("leaf_max", C.c_int32), ("iters", C.c_int32), ("granularity", C.c_int32), ("budget", C.c_int32),
+                ("lam", C.c_double), ("exchanges", C.c_int32), ("reserved", C.c_int32), ("seed", C.c_uint64)]
+
+
+class kv_c3_layout(C.Structure):
+    _fields_ = [(n, C.c_uint64) for n in ("perm", "lo", "cnt", "left", "depth", "e", "cent", "front", "sigma", "sel",
+                                          "hdr", "bytes")]
 
 
 class kv_params(C.Structure):
@@ -72,6 +82,7 @@ def lib():
         P, I32, SZ, I64 = C.c_void_p, C.c_int32, C.c_size_t, C.c_int64
         Ps, Pp, Pc = C.POINTER(kv_shape), C.POINTER(kv_params), C.POINTER(kv_cache)
         Pw = C.POINTER(kv_wnw_params)
+        Pc3, Pl3 = C.POINTER(kv_c3_params), C.POINTER(kv_c3_layout)
         sig = {
             "kv_rows": (I64, [Ps, I32]),
             "kv_check_lengths": (C.c_int, [Ps, P, I32]),
@@ -95,6 +106,9 @@ def lib():
             "kv_wnw_init": (C.c_int, [P, I32, Pw, P, P]),
             "kv_wnw_update": (C.c_int, [P, I32, Pw, I32, P, P, P, P, P, P, P]),
             "kv_wnw_recall": (C.c_int, [P, I32, Pw, I32, I32, I32, P, P, P, P, P, P, P]),
+            "kv_c3_index_layout": (C.c_int, [Ps, P, I32, Pc3, Pl3]),
+            "kv_c3_build": (C.c_int, [Ps, P, I32, Pc3, P, P, P]),
+            "kv_c3_step": (C.c_int, [Ps, P, I32, Pc3, P, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -303,6 +317,31 @@ def kv_wnw_recall(L, p, n_tidal, d, dtype, fetch, counts, K_host, V_host, K_gpu,
                                                 _stream(stream)))
 
 
+def make_c3_params(budget: int, leaf_max: int = 4, iters: int = 8, granularity: int = 16, lam: float = 0.5,
+                   exchanges: int = 2, seed: int = 0) -> kv_c3_params:
+    """C3's settings (defaults as on the C3 page: 8 iterations, seed 0, granularity 16, lambda 0.5, R 2)."""
+    return kv_c3_params(leaf_max, iters, granularity, budget, lam, exchanges, 0, seed)
+
+
+def kv_c3_index_layout(shape, L, p) -> kv_c3_layout:
+    arr, n = _L(L)
+    out = kv_c3_layout()
+    _check("kv_c3_index_layout", lib().kv_c3_index_layout(C.byref(shape), arr, n, C.byref(p), C.byref(out)))
+    return out
+
+
+def kv_c3_build(shape, L, p, K, index, stream=None):
+    arr, n = _L(L)
+    _check("kv_c3_build", lib().kv_c3_build(C.byref(shape), arr, n, C.byref(p), _ptr(K), _ptr(index),
+                                            _stream(stream)))
+
+
+def kv_c3_step(shape, L, p, K, V, q, index, out, stream=None):
+    arr, n = _L(L)
+    _check("kv_c3_step", lib().kv_c3_step(C.byref(shape), arr, n, C.byref(p), _ptr(K), _ptr(V), _ptr(q),
+                                          _ptr(index), _ptr(out), _stream(stream)))
+
+
 def kv_read_device_status(status_dev, stream=None) -> int:
     host = C.c_int32(0)
     _check("kv_read_device_status", lib().kv_read_device_status(_ptr(status_dev), C.byref(host), _stream(stream)))
@@ -317,5 +356,6 @@ __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", 
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "kv_voxzip_pool",
            "pack_segments", "ASR_SEGMENT_BYTES", "kv_wnw_params", "make_wnw_params", "kv_wnw_chunk_count",
-           "kv_wnw_state_ints", "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "status_string",
+           "kv_wnw_state_ints", "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "kv_c3_params", "kv_c3_layout",
+           "make_c3_params", "kv_c3_index_layout", "kv_c3_build", "kv_c3_step", "status_string",
            "Compressor", "EXPORTS", "KV_F32", "KV_BF16", "META_INTS"]

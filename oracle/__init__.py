@@ -394,6 +394,8 @@ class C3Row:
 
     def __init__(self, K: np.ndarray, V: np.ndarray, leaf_max: int = 4, iters: int = 8, seed: int = 0,
                  granularity: int = 16):
+        if iters < 1:
+            raise ValueError("iters >= 1")
         self.K = _c(K, np.float32)
         self.V = _c(V, np.float32)
         L, d = self.K.shape

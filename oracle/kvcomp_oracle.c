@@ -886,7 +886,7 @@ int orc_wnw_step(int64_t L, int n_anchor, const float* s, int chunk_len, int str
 /* smallest max(e) (ties to the lower parent id) among sibling pairs both on  */
 /* the frontier and not containing the split node; nodes created earlier in   */
 /* the same step are not candidates; an exchange without both candidates is   */
-/* skipped. L <= B bypasses retrieval (all keys, no update).                  */
+/* skipped. L <= B bypasses retrieval (all keys, no update). iters >= 1.      */
 /* ------------------------------------------------------------------------- */
 uint64_t orc_splitmix64(uint64_t seed, uint64_t k) {
   uint64_t z = seed + (k + 1) * 0x9e3779b97f4a7c15ull;
