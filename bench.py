@@ -321,6 +321,17 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_next_rows:
         res["next_rows"] = {"voxzip_pool": measure_voxzip(args, rank, world, dev, stream, flush),
                             "wnw_chunks_recall": measure_wnw(args, rank, world, dev, stream, flush)}
+        try:  # the newest row: a failure here is reported and leaves the line intact
+            c3 = measure_c3(args, rank, world, dev, stream, flush, cfg, d_in)
+        except Exception as exc:  # noqa: BLE001
+            c3 = {"error": f"{type(exc).__name__}: {exc}"[:300], "build_ms": -1.0, "us_per_step": -1.0}
+        # every rank takes the same collectives, failed or not
+        c3["build_ms"] = max_over_ranks(c3["build_ms"], world, dev)
+        c3["us_per_step"] = max_over_ranks(c3["us_per_step"], world, dev)
+        if "error" not in c3:
+            c3["gbs"] = c3["bytes_alg_per_step"] / (c3["us_per_step"] * 1e-6) / 1e9
+            c3["frac"] = c3["gbs"] / c3["peak"]
+        res["next_rows"]["c3_retrieval"] = c3
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(cfg, bt, args.cpu_rows)
     if world > 1:
@@ -482,6 +493,64 @@ def measure_wnw(args, rank, world, dev, stream, flush):
             fetched / WNW_STEPS, "recall_bytes_per_step": rec_bytes, "recall_gbs": rec_gbs,
             "h2d_copy_gbs_measured": h2d_gbs, "recall_frac_of_h2d_copy": rec_gbs / h2d_gbs,
             "launches_per_step": 3}
+
+
+# ----------------------------------------------------------- next rows (C3) --
+C3_BUDGET, C3_STEPS = 256, 32
+
+
+def measure_c3(args, rank, world, dev, stream, flush, cfg, d_in):
+    """kv_c3_build over the main workload's K (every layer and KV head), then
+    kv_c3_step for 32 decode steps with its decode queries: budget 256 keys,
+    granularity 16, lambda 0.5, R = 2. The build synchronises once per tree
+    level, so its time includes those host round trips."""
+    import torch
+
+    import kv_cache_compression_layer_b200 as kv
+
+    bf = cfg.dtype == "bf16"
+    shape = kv.make_shape(cfg.n_layers, cfg.n_kv_heads, cfg.group, cfg.head_dim, 1, kv.KV_BF16 if bf else kv.KV_F32)
+    p = kv.make_c3_params(C3_BUDGET)
+    lay = kv.kv_c3_index_layout(shape, cfg.L, p)
+    index = torch.empty(lay.bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(cfg.rows, cfg.group, cfg.head_dim, dtype=d_in["q"].dtype, device=dev)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    torch.cuda.synchronize()
+    b0, b1 = E(), E()
+    b0.record(stream)
+    kv.kv_c3_build(shape, cfg.L, p, d_in["K"], index, stream=stream)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    build_ms = b0.elapsed_time(b1)
+    D = d_in["q"].shape[0]
+    for t in range(args.warmup):
+        kv.kv_c3_step(shape, cfg.L, p, d_in["K"], d_in["V"], d_in["q"][t % D], index, out, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(E(), E()) for _ in range(C3_STEPS)]
+    for i in range(C3_STEPS):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(SPACER_CYCLES)
+        ev[i][0].record(stream)
+        kv.kv_c3_step(shape, cfg.L, p, d_in["K"], d_in["V"], d_in["q"][(args.warmup + i) % D], index, out,
+                      stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * sum(a.elapsed_time(b) for a, b in ev) / C3_STEPS  # this rank's; the caller takes the max
+    hdr = index[lay.hdr:lay.hdr + 16 * cfg.rows].view(torch.int32).view(cfg.rows, 4).cpu().numpy()
+    eb = 2 if bf else 4
+    # per step: the frontier's float64 centroids read, the retrieved K and V rows read, the queries and outputs
+    A = int(hdr[:, 1].sum())
+    kept = int(hdr[:, 2].sum())
+    bytes_alg = A * cfg.head_dim * 8 + kept * 2 * cfg.head_dim * eb + 2 * cfg.rows * cfg.group * cfg.head_dim * eb
+    peak, kind = hbm_peak()
+    gbs = bytes_alg / (us * 1e-6) / 1e9
+    return {"workload": f"{cfg.name}: {cfg.rows} rows, L={list(cfg.L)}, d={cfg.head_dim}, g={cfg.group}, {cfg.dtype}, "
+                        f"budget {C3_BUDGET} keys, granularity 16, lambda 0.5, R 2, {C3_STEPS} steps "
+                        f"(frontier {A} clusters)",
+            "kernels": "c3_plan/split/centroid/frontier (kv_c3_build); c3_score, c3_select, c3_attn, c3_update "
+                       "(kv_c3_step)",
+            "build_ms": build_ms, "us_per_step": us, "bytes_alg_per_step": bytes_alg, "gbs": gbs, "peak": peak,
+            "frac": gbs / peak, "peak_kind": kind + " (hbm_gbs copy)", "launches_per_step": 4}
 
 
 # ------------------------------------------------------------ reference arm --
