@@ -142,6 +142,29 @@ def test_wnw_argument_errors_launch_nothing(L):
     assert st == kv.KV_ERR_ARG
 
 
+def test_c3_argument_errors_launch_nothing(L):
+    sh = kv.make_shape(2, 2, 4, 64, 1, kv.KV_BF16)
+    p = kv.make_c3_params(128)
+    lay = kv.kv_c3_index_layout(sh, [700, 1500], p)
+    # the per-node float64 centroids dominate: 2 nodes per key x d x 8 bytes
+    assert lay.bytes >= 2 * (4 * 700 + 4 * 1500) * 64 * 8 and lay.hdr % 256 == 0 and lay.cent % 256 == 0
+    bad_params = [kv.make_c3_params(0), kv.make_c3_params(8193), kv.make_c3_params(128, iters=0),
+                  kv.make_c3_params(128, granularity=3), kv.make_c3_params(128, lam=1.5),
+                  kv.make_c3_params(128, exchanges=65), kv.make_c3_params(128, leaf_max=0)]
+    Larr = (C.c_int32 * 2)(700, 1500)
+    out = kv.kv_c3_layout()
+    for bp in bad_params:
+        assert L.kv_c3_index_layout(C.byref(sh), Larr, 2, C.byref(bp), C.byref(out)) == kv.KV_ERR_ARG
+    wide = kv.make_shape(2, 2, 4, 96, 1, kv.KV_BF16)  # head_dim 96
+    assert L.kv_c3_index_layout(C.byref(wide), Larr, 2, C.byref(p), C.byref(out)) == kv.KV_ERR_ARG
+    big_g = kv.make_shape(2, 2, 17, 64, 1, kv.KV_BF16)
+    assert L.kv_c3_index_layout(C.byref(big_g), Larr, 2, C.byref(p), C.byref(out)) == kv.KV_ERR_ARG
+    Llong = (C.c_int32 * 1)(40000)
+    assert L.kv_c3_index_layout(C.byref(sh), Llong, 1, C.byref(p), C.byref(out)) == kv.KV_ERR_UNSUPPORTED_L
+    assert L.kv_c3_build(C.byref(sh), Larr, 2, C.byref(p), 256, 4096 + 8, None) == kv.KV_ERR_ARG  # misaligned index
+    assert L.kv_c3_step(C.byref(sh), Larr, 2, C.byref(p), 256, 256, None, 4096, 4096, None) == kv.KV_ERR_ARG
+
+
 def test_fault_injection_env(L, monkeypatch):
     sh = _shape()
     Larr = (C.c_int32 * 1)(6000)
