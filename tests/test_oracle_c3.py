@@ -178,3 +178,14 @@ def test_root_split_is_eight_lloyd_iterations(seed):
     a = r.left[0]
     assert sorted(r.members(a).tolist()) == np.nonzero(side == 0)[0].tolist()
     assert sorted(r.members(a + 1).tolist()) == np.nonzero(side == 1)[0].tolist()
+
+
+def test_resolution_levels_32_16_8_4():
+    """The cuts one level above and one and two below the initial frontier have mean node
+    sizes near 32, 8 and 4 (the resolutions the page lists around granularity 16)."""
+    r, _ = _row(4096, 32)
+    D0 = int(r.depth[r.front].max())
+    for D, want in ((D0 - 1, 32), (D0, 16), (D0 + 1, 8), (D0 + 2, 4)):
+        cut = [n for n in range(r.n_nodes) if r.depth[n] == D or (r.depth[n] < D and r.left[n] < 0)]
+        assert sum(r.cnt[n] for n in cut) == r.L  # every cut partitions the keys
+        assert want / 1.6 <= r.L / len(cut) <= want * 1.6, (D, r.L / len(cut))
