@@ -318,7 +318,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-    if not args.no_next_rows:
+    if not args.no_next_rows and world == 1:  # per-GPU kernel timings; the scaling runs skip them
         res["next_rows"] = {"voxzip_pool": measure_voxzip(args, rank, world, dev, stream, flush),
                             "wnw_chunks_recall": measure_wnw(args, rank, world, dev, stream, flush)}
         try:  # the newest row: a failure here is reported and leaves the line intact
