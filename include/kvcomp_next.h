@@ -78,7 +78,8 @@ typedef struct {
  *              feature row (within the sequence), rows pooled into it, text
  *              row (-1 for a copied row).
  *   out_len    device [n_seq] int32 (output).
- *   status     device int32 or NULL: KV_DEV_RANGE is OR-ed in (see above).
+ *   status     device int32: KV_DEV_RANGE is OR-ed in (see above); may be
+ *              NULL only when E_T is NULL.
  * E_A, E_T and E_comp must not overlap. Errors: KV_ERR_ARG, KV_ERR_CUDA.
  */
 int kv_voxzip_pool(const int32_t* L_a, int32_t n_seq, const double* tau_total, const int32_t* seg_off, int32_t d,
@@ -260,7 +261,8 @@ int kv_c3_build(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv
  *   step are not candidates; an exchange lacking either is skipped.
  *   A row with L <= B attends over all its keys and keeps its state.
  *   K, V   device [sum L][d]; q device [rows][g][d]; out device [rows][g][d],
- *          all in shape->dtype. index from kv_c3_build (updated).
+ *          all in shape->dtype. index from kv_c3_build with the same shape,
+ *          lengths and parameters (updated; not checked against them).
  * Errors: KV_ERR_ARG, KV_ERR_UNSUPPORTED_L, KV_ERR_CUDA.
  */
 int kv_c3_step(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_c3_params* p, const void* K,
