@@ -332,6 +332,11 @@ def run_ours(args, rank, world, local_rank):
             c3["gbs"] = c3["bytes_alg_per_step"] / (c3["us_per_step"] * 1e-6) / 1e9
             c3["frac"] = c3["gbs"] / c3["peak"]
         res["next_rows"]["c3_retrieval"] = c3
+        try:
+            res["next_rows"]["pooled_alloc_segmented_select"] = measure_variants(args, dev, stream, flush, cfg, comp,
+                                                                                 d_in, shape, params)
+        except Exception as exc:  # noqa: BLE001
+            res["next_rows"]["pooled_alloc_segmented_select"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(cfg, bt, args.cpu_rows)
     if world > 1:
@@ -493,6 +498,64 @@ def measure_wnw(args, rank, world, dev, stream, flush):
             fetched / WNW_STEPS, "recall_bytes_per_step": rec_bytes, "recall_gbs": rec_gbs,
             "h2d_copy_gbs_measured": h2d_gbs, "recall_frac_of_h2d_copy": rec_gbs / h2d_gbs,
             "launches_per_step": 3}
+
+
+# ------------------------------------------- next rows (step 3 and 4 variants) --
+VARIANT_SEGMENTS = 32
+
+
+def measure_variants(args, dev, stream, flush, cfg, comp, d_in, shape, params):
+    """kv_allocate_global over the main workload's head scores, then
+    kv_select_gather_segmented (32 segments a row) on the smoothed scores the
+    timed steps left in the Compressor, into buffers of their own. N = 1."""
+    import torch
+
+    import kv_cache_compression_layer_b200 as kv
+
+    rows, d = cfg.rows, cfg.head_dim
+    total = kv.kv_total_slots(shape, cfg.L, params)
+    b = torch.empty(rows, dtype=torch.int32, device=dev)
+    off = torch.empty(rows + 1, dtype=torch.int64, device=dev)
+    idx = torch.empty(total, dtype=torch.int32, device=dev)
+    Kc = torch.empty(total, d, dtype=d_in["K"].dtype, device=dev)
+    Vc = torch.empty_like(Kc)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def once():
+        kv.kv_allocate_global(shape, cfg.L, params, d_in["S"], b, off, stream=stream)
+        kv.kv_select_gather_segmented(shape, cfg.L, comp.s_hat, d_in["K"], d_in["V"], b, off, VARIANT_SEGMENTS, idx,
+                                      Kc, Vc, stream=stream)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    ev = [(E(), E(), E()) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(SPACER_CYCLES)
+        ev[i][0].record(stream)
+        kv.kv_allocate_global(shape, cfg.L, params, d_in["S"], b, off, stream=stream)
+        ev[i][1].record(stream)
+        kv.kv_select_gather_segmented(shape, cfg.L, comp.s_hat, d_in["K"], d_in["V"], b, off, VARIANT_SEGMENTS, idx,
+                                      Kc, Vc, stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    alloc_us = 1e3 * sum(a.elapsed_time(x) for a, x, _ in ev) / args.steps
+    sel_us = 1e3 * sum(x.elapsed_time(c) for _, x, c in ev) / args.steps
+    bb = b.cpu().numpy().astype(np.int64)
+    eb = Kc.element_size()
+    L_rows = np.array([cfg.L[cfg.row_triplet(r)[0]] for r in range(rows)], np.int64)
+    # smoothed scores read, indices written, kept K and V read and written compacted
+    sel_bytes = int((4 * L_rows + 4 * bb + 4 * d * eb * bb).sum())
+    peak, kind = hbm_peak()
+    gbs = sel_bytes / (sel_us * 1e-6) / 1e9
+    return {"workload": f"{cfg.name}: {rows} rows, L={list(cfg.L)}, d={d}, {cfg.dtype}, one budget over the "
+                        f"{cfg.n_layers * cfg.n_kv_heads} heads of a sequence, {VARIANT_SEGMENTS} segments a row",
+            "kernels": "allocate_kernel + slot_offsets_kernel (kv_allocate_global); select_kernel + gather_kernel "
+                       "(kv_select_gather_segmented)",
+            "allocate_us": alloc_us, "select_gather_us": sel_us, "select_gather_bytes_alg": sel_bytes,
+            "select_gather_gbs": gbs, "peak": peak, "select_gather_frac": gbs / peak,
+            "peak_kind": kind + " (hbm_gbs copy)", "launches_per_call": 4}
 
 
 # ----------------------------------------------------------- next rows (C3) --
