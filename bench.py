@@ -7,7 +7,11 @@ the workload's decode steps (kv_decode_attn_update, all layers per launch).
 `value` = audio tokens of the batch processed per second of step time (for N
 ranks: N x that, each rank running its own replica; no data-path collective).
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3b]
+Default workload: the ragged batch (8 sequences, L 2000-16000, 28 layers,
+28 q / 4 kv heads, budget 25%, 128 decode steps), the largest that fits one
+GPU; --config names another.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config ragged]
        python bench.py --impl reference ...   (the CPU oracle as the arm)
 Multi-GPU: python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
 """
@@ -164,18 +168,41 @@ def oracle_sample(cfg: synth.Config, bt: synth.Batch, rows, n_threads: int):
     return time.perf_counter() - t0
 
 
+def sample_rows(cfg: synth.Config, n: int):
+    """n rows spread evenly over the batch (the same number from every
+    sequence when n is a multiple of n_seq), so the sample has the batch's
+    length mix."""
+    n = max(1, min(n, cfg.rows))
+    return sorted({int(x) for x in np.linspace(0, cfg.rows - 1, n).round()})
+
+
+def sample_tokens(cfg: synth.Config, rows) -> float:
+    """Audio tokens a sample of rows stands for: each of a sequence's
+    n_layers x n_kv_heads rows carries 1/(n_layers x n_kv_heads) of its L."""
+    per_seq = cfg.n_layers * cfg.n_kv_heads
+    return float(sum(cfg.row_L(r) for r in rows)) / per_seq
+
+
+def config_dict(cfg: synth.Config, world: int) -> dict:
+    """The workload description both arms print (identical keys and values)."""
+    return {"workload": describe(cfg), "n_seq": cfg.n_seq, "rows": cfg.rows,
+            "l2": "256 MB write between timed steps (outside the events)",
+            "parallelism": f"replicas x{world} (rows independent, no collective)"}
+
+
 def cpu_baseline(cfg, bt, n_rows_sample: int):
+    """The oracle timed on a bounded sample of the batch's rows (all host threads)."""
     import oracle as orc
 
     threads = orc.default_threads()
-    rows = list(range(min(n_rows_sample, cfg.rows)))
+    rows = sample_rows(cfg, n_rows_sample)
     orc.build()
     secs = oracle_sample(cfg, bt, rows, threads)
-    full = secs * cfg.rows / len(rows)  # the rows of one batch are independent
-    tokens = sum(cfg.L)
-    return {"value": tokens / full, "unit": UNIT, "cores": min(threads, len(rows)), "kind": "oracle",
-            "sample": f"{len(rows)} of {cfg.rows} rows through the whole path incl. {cfg.decode_steps} decode steps "
-                      f"({secs:.2f} s), scaled to one batch"}
+    return {"value": sample_tokens(cfg, rows) / secs, "unit": UNIT, "cores": min(threads, len(rows)),
+            "kind": "oracle", "seconds": secs,
+            "sample": f"{len(rows)} of {cfg.rows} rows ({len(rows) // cfg.n_seq if len(rows) % cfg.n_seq == 0 else '~'}"
+                      f" per sequence) through the whole path incl. {cfg.decode_steps} decode steps, timed "
+                      f"{secs:.2f} s; value = the sample's share of the batch's audio tokens / that time"}
 
 
 # ------------------------------------------------------------------ our arm --
@@ -287,7 +314,8 @@ def run_ours(args, rank, world, local_rank):
     dec_bytes = int(((b + 1) * (2 * eb * d + 8) + 2 * eb * d).sum())
     dec_avg_us = sum(dec_us) / len(dec_us)
     L_rows = np.array([cfg.L[cfg.row_triplet(r)[0]] for r in range(cfg.rows)], np.int64)
-    comp_bytes = int((2 * eb * d * (L_rows + 3 * b)).sum())
+    # K read once, kept V read once, compacted K and V written once
+    comp_bytes = int((eb * d * (L_rows + 3 * b)).sum())
     comp_avg_ms = sum(comp_ms) / len(comp_ms)
     peak, peak_kind = hbm_peak()
     dec_gbs = dec_bytes / (dec_avg_us * 1e-6) / 1e9
@@ -302,9 +330,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
         "data": "synthetic (seeded AR(1) keys, diagonal-band queries; stands in for long-audio workloads)",
-        "config": {"workload": describe(cfg), "n_seq": cfg.n_seq, "rows": cfg.rows,
-                   "l2": "256 MB write between timed steps (outside the events)",
-                   "parallelism": f"replicas x{world} (rows independent, no collective)"},
+        "config": config_dict(cfg, world),
         "stages": {"compress_ms": comp_avg_ms, "compress_tokens_per_s": world * tokens / (comp_avg_ms * 1e-3),
                    "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
                    "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
@@ -563,51 +589,60 @@ C3_BUDGET, C3_STEPS = 256, 32
 
 
 def measure_c3(args, rank, world, dev, stream, flush, cfg, d_in):
-    """kv_c3_build over the main workload's K (every layer and KV head), then
-    kv_c3_step for 32 decode steps with its decode queries: budget 256 keys,
-    granularity 16, lambda 0.5, R = 2. The build synchronises once per tree
-    level, so its time includes those host round trips."""
+    """kv_c3_build over the K of the main workload's longest sequence (every
+    layer and KV head of it), then kv_c3_step for 32 decode steps with its
+    decode queries: budget 256 keys, granularity 16, lambda 0.5, R = 2. The
+    build synchronises once per tree level, so its time includes those host
+    round trips."""
     import torch
 
     import kv_cache_compression_layer_b200 as kv
 
     bf = cfg.dtype == "bf16"
     shape = kv.make_shape(cfg.n_layers, cfg.n_kv_heads, cfg.group, cfg.head_dim, 1, kv.KV_BF16 if bf else kv.KV_F32)
+    seq = int(np.argmax(cfg.L))
+    rps = cfg.n_layers * cfg.n_kv_heads
+    r0, r1 = seq * rps, (seq + 1) * rps
+    k0 = sum(rps * cfg.L[s] for s in range(seq))
+    Ls = [cfg.L[seq]]
+    K = d_in["K"][k0:k0 + rps * Ls[0]]
+    V = d_in["V"][k0:k0 + rps * Ls[0]]
+    Q = d_in["q"][:, r0:r1]
     p = kv.make_c3_params(C3_BUDGET)
-    lay = kv.kv_c3_index_layout(shape, cfg.L, p)
+    lay = kv.kv_c3_index_layout(shape, Ls, p)
     index = torch.empty(lay.bytes, dtype=torch.uint8, device=dev)
-    out = torch.empty(cfg.rows, cfg.group, cfg.head_dim, dtype=d_in["q"].dtype, device=dev)
+    out = torch.empty(rps, cfg.group, cfg.head_dim, dtype=d_in["q"].dtype, device=dev)
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     torch.cuda.synchronize()
     b0, b1 = E(), E()
     b0.record(stream)
-    kv.kv_c3_build(shape, cfg.L, p, d_in["K"], index, stream=stream)
+    kv.kv_c3_build(shape, Ls, p, K, index, stream=stream)
     b1.record(stream)
     torch.cuda.synchronize()
     build_ms = b0.elapsed_time(b1)
-    D = d_in["q"].shape[0]
+    D = Q.shape[0]
     for t in range(args.warmup):
-        kv.kv_c3_step(shape, cfg.L, p, d_in["K"], d_in["V"], d_in["q"][t % D], index, out, stream=stream)
+        kv.kv_c3_step(shape, Ls, p, K, V, Q[t % D].contiguous(), index, out, stream=stream)
     torch.cuda.synchronize()
     ev = [(E(), E()) for _ in range(C3_STEPS)]
+    qs = [Q[(args.warmup + i) % D].contiguous() for i in range(C3_STEPS)]
     for i in range(C3_STEPS):
         flush.fill_(i & 0xFF)
         torch.cuda._sleep(SPACER_CYCLES)
         ev[i][0].record(stream)
-        kv.kv_c3_step(shape, cfg.L, p, d_in["K"], d_in["V"], d_in["q"][(args.warmup + i) % D], index, out,
-                      stream=stream)
+        kv.kv_c3_step(shape, Ls, p, K, V, qs[i], index, out, stream=stream)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     us = 1e3 * sum(a.elapsed_time(b) for a, b in ev) / C3_STEPS  # this rank's; the caller takes the max
-    hdr = index[lay.hdr:lay.hdr + 16 * cfg.rows].view(torch.int32).view(cfg.rows, 4).cpu().numpy()
+    hdr = index[lay.hdr:lay.hdr + 16 * rps].view(torch.int32).view(rps, 4).cpu().numpy()
     eb = 2 if bf else 4
     # per step: the frontier's float64 centroids read, the retrieved K and V rows read, the queries and outputs
     A = int(hdr[:, 1].sum())
     kept = int(hdr[:, 2].sum())
-    bytes_alg = A * cfg.head_dim * 8 + kept * 2 * cfg.head_dim * eb + 2 * cfg.rows * cfg.group * cfg.head_dim * eb
+    bytes_alg = A * cfg.head_dim * 8 + kept * 2 * cfg.head_dim * eb + 2 * rps * cfg.group * cfg.head_dim * eb
     peak, kind = hbm_peak()
     gbs = bytes_alg / (us * 1e-6) / 1e9
-    return {"workload": f"{cfg.name}: {cfg.rows} rows, L={list(cfg.L)}, d={cfg.head_dim}, g={cfg.group}, {cfg.dtype}, "
+    return {"workload": f"{cfg.name}, sequence {seq}: {rps} rows, L={Ls[0]}, d={cfg.head_dim}, g={cfg.group}, {cfg.dtype}, "
                         f"budget {C3_BUDGET} keys, granularity 16, lambda 0.5, R 2, {C3_STEPS} steps "
                         f"(frontier {A} clusters)",
             "kernels": "c3_plan/split/centroid/frontier (kv_c3_build); c3_score, c3_select, c3_attn, c3_update "
@@ -618,28 +653,32 @@ def measure_c3(args, rank, world, dev, stream, flush, cfg, d_in):
 
 # ------------------------------------------------------------ reference arm --
 def run_reference(args, rank, world):
-    """The CPU oracle as the reference arm, on a bounded sample of the workload."""
+    """The CPU oracle as the reference arm: every step runs the whole path on
+    the same bounded sample of the workload's rows (all host threads); the
+    line reports the time it measured for that sample."""
     if rank != 0:
         return
     import oracle as orc
 
     orc.build()
     cfg = synth.CONFIGS[args.config]
-    rows = list(range(min(args.ref_rows, cfg.rows)))
+    rows = sample_rows(cfg, args.ref_rows)
     bt = synth.make_batch(cfg)
     threads = orc.default_threads()
     for _ in range(args.warmup):
-        oracle_sample(cfg, bt, rows[:1], threads)
+        oracle_sample(cfg, bt, rows, threads)
     secs = [oracle_sample(cfg, bt, rows, threads) for _ in range(args.steps)]
-    full = (sum(secs) / len(secs)) * cfg.rows / len(rows)
-    value = sum(cfg.L) / full
+    step_s = sum(secs) / len(secs)
+    value = sample_tokens(cfg, rows) / step_s
+    sample = (f"{len(rows)} of {cfg.rows} rows per step through the whole path incl. {cfg.decode_steps} decode "
+              f"steps; value = the sample's share of the batch's audio tokens / the measured step time")
     res = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": full * 1e3, "higher_is_better": True,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic (seeded AR(1) keys, diagonal-band queries)",
-           "config": {"workload": describe(cfg), "n_seq": cfg.n_seq, "rows": cfg.rows},
+           "data": "synthetic (seeded AR(1) keys, diagonal-band queries; stands in for long-audio workloads)",
+           "config": config_dict(cfg, world),
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, len(rows)), "kind": "oracle",
-                            "sample": f"{len(rows)} of {cfg.rows} rows per step, scaled to one batch"},
+                            "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
@@ -649,11 +688,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="3b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", default="ragged", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-rows", type=int, default=1 << 20,
-                    help="rows of the oracle sample for cpu_baseline (default: the whole batch)")
-    ap.add_argument("--ref-rows", type=int, default=8, help="rows per step of the reference (oracle) arm")
+    ap.add_argument("--cpu-rows", type=int, default=64,
+                    help="rows of the oracle sample for cpu_baseline, spread over the batch")
+    ap.add_argument("--ref-rows", type=int, default=64,
+                    help="rows per step of the reference (oracle) arm, spread over the batch")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true", help="skip the timing of the rows beyond the path")
     args = ap.parse_args()

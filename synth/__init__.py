@@ -45,7 +45,9 @@ bf16 workloads; the returned float32 arrays hold those bf16-exact values.
 from __future__ import annotations
 
 import dataclasses
+import os
 import math
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, List, Optional, Sequence
 
 import numpy as np
@@ -287,23 +289,43 @@ class Batch:
         return np.concatenate([[0], np.cumsum(self.L_rows)]).astype(np.int64)
 
 
-def make_batch(cfg: Config, steps: Optional[int] = None) -> Batch:
+def make_batch(cfg: Config, steps: Optional[int] = None, threads: int = 0) -> Batch:
+    """Every row of the workload, generated row by row (each row from its own
+    seeded streams, so the result does not depend on `threads`) into
+    preallocated concatenated arrays; rows are generated on a thread pool."""
     steps = cfg.decode_steps if steps is None else steps
     rows = list(range(cfg.rows))
-    parts = [make_row(cfg, *cfg.row_triplet(r), steps=steps) for r in rows]
-    spikes = None
-    if cfg.spike_frac > 0:
-        spikes = np.concatenate([p.spikes for p in parts])
-    return Batch(cfg=cfg, rows=rows,
-                 L_rows=np.array([p.L for p in parts], np.int64),
-                 qwin=np.stack([p.qwin for p in parts]),
-                 K=np.concatenate([p.K for p in parts]),
-                 V=np.concatenate([p.V for p in parts]),
-                 S=head_scores(cfg),
-                 q_dec=np.ascontiguousarray(np.stack([p.q_dec for p in parts], axis=1)),
-                 k_dec=np.ascontiguousarray(np.stack([p.k_dec for p in parts], axis=1)),
-                 v_dec=np.ascontiguousarray(np.stack([p.v_dec for p in parts], axis=1)),
-                 spikes=spikes)
+    L_rows = np.array([cfg.row_L(r) for r in rows], np.int64)
+    off = np.concatenate([[0], np.cumsum(L_rows)]).astype(np.int64)
+    g, d, R = cfg.group, cfg.head_dim, cfg.R
+    qwin = np.empty((cfg.rows, R, d), np.float32)
+    K = np.empty((int(off[-1]), d), np.float32)
+    V = np.empty((int(off[-1]), d), np.float32)
+    q_dec = np.empty((steps, cfg.rows, g, d), np.float32)
+    k_dec = np.empty((steps, cfg.rows, d), np.float32)
+    v_dec = np.empty((steps, cfg.rows, d), np.float32)
+    spikes = np.empty(int(off[-1]), bool) if cfg.spike_frac > 0 else None
+
+    def fill(r: int) -> None:
+        p = make_row(cfg, *cfg.row_triplet(r), steps=steps)
+        qwin[r] = p.qwin
+        K[off[r]:off[r + 1]] = p.K
+        V[off[r]:off[r + 1]] = p.V
+        q_dec[:, r] = p.q_dec
+        k_dec[:, r] = p.k_dec
+        v_dec[:, r] = p.v_dec
+        if spikes is not None:
+            spikes[off[r]:off[r + 1]] = p.spikes
+
+    n_thr = threads or min(32, os.cpu_count() or 1)
+    if n_thr <= 1 or cfg.rows <= 1:
+        for r in rows:
+            fill(r)
+    else:
+        with ThreadPoolExecutor(max_workers=n_thr) as ex:
+            list(ex.map(fill, rows))
+    return Batch(cfg=cfg, rows=rows, L_rows=L_rows, qwin=qwin, K=K, V=V, S=head_scores(cfg),
+                 q_dec=q_dec, k_dec=k_dec, v_dec=v_dec, spikes=spikes)
 
 
 @dataclasses.dataclass
