@@ -161,8 +161,13 @@ int kv_sss(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* 
  *   B = floor(budget_pct * L * H / 100);  B_rem = B - H * w;
  *   x_h = w + r * B_rem / H + (1 - r) * B_rem * S_h / sum_h S_h;
  *   b_h = floor(x_h), the remainder +1 to the largest fractional parts (ties
- *   to the lower head), heads above L capped at L with the rest re-allocated.
- *   Computed in float64 in a fixed operation order (see DESIGN).
+ *   to the lower head), heads above L capped at L with the rest re-allocated
+ *   over the other heads; sum_h S_h = 0 splits evenly.
+ *   Computed in float64, every operation rounded to nearest on its own (no
+ *   fused multiply-add), in this order, so the result is reproducible bit for
+ *   bit: sumS = ((S_0 + S_1) + S_2) + ... in head order; t1 = r * B_rem;
+ *   t1 = t1 / H; t2 = (1 - r) * B_rem; t2 = t2 * S_h; t2 = t2 / sumS;
+ *   x_h = (w + t1) + t2 (r and S_h widened exactly from float32).
  *   S        : device, [n_layers][H] float32 per-head audio relevance.
  *   b        : device, [rows] int32 (output).
  *   slot_off : device, [rows + 1] int64 (output): prefix of b_i + 1.
@@ -266,8 +271,9 @@ int kv_decode_attn_update(const kv_shape* shape, const int32_t* L, int32_t n_seq
  * Same arguments, layout and result as kv_score, minus the workspace: the
  * scratch is a file-scope device array of KV_NOALLOC_SCRATCH_BYTES held by
  * every GPU that loads this library until the process exits.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Each call looks up the array's device address (cudaGetSymbolAddress);
+ *     the first call on a device may load the library's device code there,
+ *     so make that first call before any stream capture.
  *   - Batches whose scratch (kv_workspace_bytes) exceeds the limit return
  *     KV_ERR_WORKSPACE and launch nothing.
  *   - Every call shares the one array and it keeps the last call's contents;
@@ -275,13 +281,30 @@ int kv_decode_attn_update(const kv_shape* shape, const int32_t* L, int32_t n_seq
  *     (different streams, or different threads' streams) race on it: order
  *     them on one stream or synchronise between them.
  *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
- *     Device-side errors are recorded in the array's status word, which this
- *     variant does not expose.
+ *     Device-side errors (a bounded wait that ran out) go to the array's
+ *     status word: read it with kv_score_noalloc_status.
  * Errors: as kv_score (KV_ERR_WORKSPACE when the batch is too large).
  */
 #define KV_NOALLOC_SCRATCH_BYTES (8u << 20)
 int kv_score_noalloc(const kv_shape* shape, const int32_t* L, int32_t n_seq, const void* qwin, const void* K,
                      float* s, void* stream);
+
+/* The device status word (KV_DEV_* bits) of the last kv_score_noalloc call
+ * on the current device, copied to *status_host after `stream` (synchronises
+ * it; issue it on the scoring call's stream). Returns KV_OK, KV_ERR_ARG or
+ * KV_ERR_CUDA. */
+int kv_score_noalloc_status(int32_t* status_host, void* stream);
+
+/* Time limit of the library's bounded device waits, in nanoseconds of the
+ * GPU's global timer, for every launch made after the call (process-wide,
+ * all devices); returns the previous limit. Default 2 000 000 000 (2 s).
+ * A wait that runs out records KV_DEV_TIMEOUT in the call's status word; the
+ * kernel lets its copies and tensor-core operations in flight finish (a drain
+ * with a fixed limit of its own), releases its tensor memory and returns.
+ * 0 makes every wait give up unless what it waits for has already happened,
+ * which drives the timeout paths in tests. (No counterpart on the pages: a
+ * safety limit of this implementation.) */
+uint64_t kv_set_wait_limit_ns(uint64_t limit_ns);
 
 /* Copies the device status word to the host (synchronises `stream`);
  * returns KV_OK or KV_ERR_CUDA. */

@@ -28,7 +28,8 @@ EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots"
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes", "kv_allocate_global",
            "kv_select_gather_segmented", "kv_voxzip_pool", "kv_wnw_chunk_count", "kv_wnw_state_ints",
-           "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "kv_c3_index_layout", "kv_c3_build", "kv_c3_step")
+           "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "kv_c3_index_layout", "kv_c3_build", "kv_c3_step",
+           "kv_set_wait_limit_ns", "kv_score_noalloc_status")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -99,6 +100,8 @@ def lib():
             "kv_read_device_status": (C.c_int, [P, P, P]),
             "kv_status_string": (C.c_char_p, [C.c_int]),
             "kv_score_noalloc": (C.c_int, [Ps, P, I32, P, P, P, P]),
+            "kv_score_noalloc_status": (C.c_int, [P, P]),
+            "kv_set_wait_limit_ns": (C.c_uint64, [C.c_uint64]),
             "kv_decode_scratch_bytes": (SZ, [Ps, P, I32, Pp, I64]),
             "kv_voxzip_pool": (C.c_int, [P, I32, P, P, I32, I32, C.c_float, P, P, P, I64, P, P, P, P, P]),
             "kv_wnw_chunk_count": (I64, [P, I32, Pw]),
@@ -191,6 +194,21 @@ def kv_score_noalloc(shape, L, qwin, K, s, stream=None):
     arr, n = _L(L)
     _check("kv_score_noalloc", lib().kv_score_noalloc(C.byref(shape), arr, n, _ptr(qwin), _ptr(K), _ptr(s),
                                                       _stream(stream)))
+
+
+def kv_score_noalloc_status(stream=None) -> int:
+    """The device status word of the last kv_score_noalloc call on the current device."""
+    host = C.c_int32(0)
+    _check("kv_score_noalloc_status", lib().kv_score_noalloc_status(C.byref(host), _stream(stream)))
+    return host.value
+
+
+def kv_set_wait_limit_ns(limit_ns: int) -> int:
+    """Sets the limit of the library's bounded device waits for later launches; returns the previous one."""
+    return int(lib().kv_set_wait_limit_ns(int(limit_ns)))
+
+
+DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
 
 
 def kv_sss(shape, L, s, s_hat, kstar, alpha: float, rho: float, stream=None):
@@ -352,7 +370,7 @@ from .pipeline import Compressor  # noqa: E402  (the torch-side convenience wrap
 
 __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", "make_params", "make_cache",
            "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_score_noalloc",
-           "kv_sss",
+           "kv_score_noalloc_status", "kv_set_wait_limit_ns", "DEFAULT_WAIT_LIMIT_NS", "kv_sss",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "kv_voxzip_pool",
            "pack_segments", "ASR_SEGMENT_BYTES", "kv_wnw_params", "make_wnw_params", "kv_wnw_chunk_count",

@@ -3,6 +3,7 @@
 // argument documentation are in include/kvcomp.h.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -82,6 +83,9 @@ bool encode_rows_bf16(CUtensorMap* map, const void* base, int d, long long rows,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+static std::atomic<unsigned long long> g_wait_limit_ns{kWaitLimitNs};
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 static bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -256,6 +260,10 @@ int kv_decode_attn_update(const kv_shape* shape, const int32_t* L, int32_t n_seq
   if (st) return st;
   if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(out)) return KV_ERR_ARG;
   return launch_decode(*shape, m, *params, *cache, q_t, k_t, v_t, out, static_cast<cudaStream_t>(stream));
+}
+
+uint64_t kv_set_wait_limit_ns(uint64_t limit_ns) {
+  return g_wait_limit_ns.exchange(limit_ns, std::memory_order_relaxed);
 }
 
 int kv_read_device_status(const int32_t* status_dev, int32_t* status_host, void* stream) {

@@ -52,11 +52,12 @@ struct C3Arr {
   uint8_t* fresh;  // per node
   int32_t* tasks;  // (row, node) pairs: the splits of the current level
   int32_t* count;  // [4]
+  int32_t* parent; // per node: the node it was split from (-1 for the root)
 };
 
 // Scratch of the index that the public layout does not name.
 struct C3Scratch {
-  uint64_t side, tmp, taken, on, fresh, tasks, count;
+  uint64_t side, tmp, taken, on, fresh, tasks, count, parent;
 };
 
 uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
@@ -87,6 +88,7 @@ void layout_of(long long T, int rows, int d, kv_c3_layout& L, C3Scratch& S) {
   S.on = take(nodes);
   S.fresh = take(nodes);
   S.count = take(16);
+  S.parent = take(nodes * 4);
   L.bytes = o;
 }
 
@@ -101,6 +103,7 @@ C3Arr arrays_of(void* index, const kv_c3_layout& L, const C3Scratch& S) {
   a.fresh = a.base + S.fresh;
   a.tasks = reinterpret_cast<int32_t*>(a.base + S.tasks);
   a.count = reinterpret_cast<int32_t*>(a.base + S.count);
+  a.parent = reinterpret_cast<int32_t*>(a.base + S.parent);
   return a;
 }
 
@@ -163,6 +166,7 @@ __global__ void __launch_bounds__(256) c3_init_kernel(const RowMap m, C3Arr a) {
     a.cnt()[no] = L;
     a.left()[no] = -1;
     a.depth()[no] = 0;
+    a.parent[no] = -1;
     int32_t* h = a.hdr() + (long long)row * kHdr;
     h[0] = 1;  // nodes
     h[1] = 0;  // level begin (until the frontier kernel stores A here)
@@ -191,6 +195,7 @@ __global__ void __launch_bounds__(kScanThreads) c3_plan_kernel(const RowMap m, C
         a.left()[no + n] = c;
         a.depth()[no + c] = a.depth()[no + c + 1] = a.depth()[no + n] + 1;
         a.left()[no + c] = a.left()[no + c + 1] = -1;
+        a.parent[no + c] = a.parent[no + c + 1] = n;
         const int q = atomicAdd(a.count, 1);
         a.tasks[2 * q] = row;
         a.tasks[2 * q + 1] = n;
@@ -516,28 +521,68 @@ __device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16* p, float v)
 }
 
 constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = kAttnThreads / 32;
 
-// Exact attention of one query head over the retrieved keys (float32).
+// Up to four consecutive elements of a K or V row as float32.
+template <typename T>
+__device__ __forceinline__ void ld4(const T* p, int n, float (&v)[4]);
+template <>
+__device__ __forceinline__ void ld4<float>(const float* p, int n, float (&v)[4]) {
+  if (n == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = v[3] = 0.f;
+  }
+}
+template <>
+__device__ __forceinline__ void ld4<__nv_bfloat16>(const __nv_bfloat16* p, int n, float (&v)[4]) {
+  if (n == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  } else {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    v[0] = a.x; v[1] = a.y; v[2] = v[3] = 0.f;
+  }
+}
+
+// Exact attention of one query head over the retrieved keys (float32): a warp
+// per key for the logits (each lane d/32 consecutive elements), then p V with
+// the keys split over the warps (lanes over the dimensions) and the warps'
+// partial sums added in warp order.
 template <typename T>
 __global__ void __launch_bounds__(kAttnThreads)
     c3_attn_kernel(const RowMap m, C3Arr a, const T* __restrict__ K, const T* __restrict__ V,
-                   const T* __restrict__ q, T* __restrict__ out, int G, int d) {
-  __shared__ float lg[KV_C3_MAX_BUDGET];
+                   const T* __restrict__ q, T* __restrict__ out, int G, int d, int B) {
+  extern __shared__ float dyn_s[];  // logits [B], then the retrieved positions [B]
+  float* lg = dyn_s;
+  int* sel_s = reinterpret_cast<int*>(dyn_s + B);
   __shared__ float qv[128];
   __shared__ float red[32];
+  __shared__ float po[kAttnWarps][128];
   const int row = blockIdx.x, g = blockIdx.y;
   const long long ko = row_key_off(m, row);
-  const int n = a.hdr()[(long long)row * kHdr + 2];
+  const int n = min(a.hdr()[(long long)row * kHdr + 2], B);  // the select kernel retrieves at most B
   const int32_t* sel = a.sel() + ko;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per = d / 32;  // elements per lane: 2 or 4
   const T* qr = q + ((long long)row * G + g) * d;
   for (int k = threadIdx.x; k < d; k += kAttnThreads) qv[k] = (float)ld(qr + k);
+  for (int i = threadIdx.x; i < n; i += kAttnThreads) sel_s[i] = sel[i];
   __syncthreads();
   const float scale = rsqrtf((float)d);
-  for (int i = warp; i < n; i += kAttnThreads / 32) {
-    const T* kr = K + (ko + sel[i]) * d;
+  float qa[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) qa[t] = t < per ? qv[lane * per + t] : 0.f;
+  for (int i = warp; i < n; i += kAttnWarps) {
+    float kv4[4];
+    ld4(K + (ko + sel_s[i]) * d + lane * per, per, kv4);
     float s = 0.f;
-    for (int k = lane; k < d; k += 32) s += qv[k] * (float)ld(kr + k);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) s = fmaf(qa[t], kv4[t], s);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) lg[i] = s * scale;
@@ -550,7 +595,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   if (lane == 0) red[warp] = mx;
   __syncthreads();
   mx = red[0];
-  for (int w = 1; w < kAttnThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+  for (int w = 1; w < kAttnWarps; ++w) mx = fmaxf(mx, red[w]);
   __syncthreads();
   float sum = 0.f;
   for (int i = threadIdx.x; i < n; i += kAttnThreads) {
@@ -563,11 +608,28 @@ __global__ void __launch_bounds__(kAttnThreads)
   if (lane == 0) red[warp] = sum;
   __syncthreads();
   sum = 0.f;
-  for (int w = 0; w < kAttnThreads / 32; ++w) sum += red[w];
+  for (int w = 0; w < kAttnWarps; ++w) sum += red[w];
+  // p V: warp w takes the keys [w n / 8, (w + 1) n / 8), lane the elements lane * per ...
+  {
+    const int i0 = (int)((long long)n * warp / kAttnWarps), i1 = (int)((long long)n * (warp + 1) / kAttnWarps);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int i = i0; i < i1; ++i) {
+      float vv[4];
+      ld4(V + (ko + sel_s[i]) * d + lane * per, per, vv);
+      const float p = lg[i];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) acc[t] = fmaf(p, vv[t], acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (t < per) po[warp][lane * per + t] = acc[t];
+  }
+  __syncthreads();
   T* orow = out + ((long long)row * G + g) * d;
   for (int k = threadIdx.x; k < d; k += kAttnThreads) {
     float acc = 0.f;
-    for (int i = 0; i < n; ++i) acc += lg[i] * (float)ld(V + (ko + sel[i]) * d + k);
+    for (int w = 0; w < kAttnWarps; ++w) acc += po[w][k];
     st_out(orow + k, acc / sum);
   }
 }
@@ -642,21 +704,31 @@ __global__ void __launch_bounds__(kScanThreads)
   __syncthreads();
   for (int i = threadIdx.x; i < A; i += kScanThreads) on[fr[i]] = 1;
   __syncthreads();
+  // Every candidate of an exchange is a node of the step's starting frontier
+  // that is still on and was not made in this step (nodes made in the step are
+  // fresh), so both searches walk the frontier list instead of every node; the
+  // winners (ties to the lower node id) are the same.
+  const int32_t* parent = a.parent + no;
   for (int r = 0; r < R; ++r) {
     double sv = 0.0;
     int s = -1;
-    for (int n = threadIdx.x; n < nodes; n += kScanThreads)
+    for (int i = threadIdx.x; i < A; i += kScanThreads) {
+      const int n = fr[i];
       if (on[n] && !fresh[n] && left[n] >= 0 && wins(e[n], n, sv, s, true)) {
         sv = e[n];
         s = n;
       }
+    }
     block_pick(sv, s, true, shv, shi);
     if (s < 0) break;
+    // merge: the parent of two siblings still on the frontier (x its left child)
     double pv = 0.0;
     int p = -1;
-    for (int n = threadIdx.x; n < nodes; n += kScanThreads) {
-      if (left[n] < 0) continue;
-      const int x = left[n], y = x + 1;
+    for (int i = threadIdx.x; i < A; i += kScanThreads) {
+      const int x = fr[i];
+      const int n = parent[x];
+      if (n < 0 || left[n] != x) continue;
+      const int y = x + 1;
       if (!on[x] || !on[y] || fresh[x] || fresh[y] || x == s || y == s) continue;
       const double v = e[x] > e[y] ? e[x] : e[y];
       if (wins(v, n, pv, p, false)) {
@@ -804,20 +876,27 @@ int kv_c3_step(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_
   const int d = shape->head_dim, G = shape->group, B = p->budget;
   const int Lmax = max_len(m);
   const dim3 sgrid((2 * Lmax + 127) / 128, m.n_rows);
+  const size_t attn_smem = 2 * (size_t)B * sizeof(float);  // logits and retrieved positions
   if (shape->dtype == KV_BF16) {
     using T = __nv_bfloat16;
     c3_score_kernel<T><<<sgrid, 128, 0, cs>>>(m, a, static_cast<const T*>(q), G, d, B);
     c3_select_kernel<<<m.n_rows, kScanThreads, 0, cs>>>(m, a, B);
-    c3_attn_kernel<T><<<dim3(m.n_rows, G), kAttnThreads, 0, cs>>>(m, a, static_cast<const T*>(K),
-                                                                 static_cast<const T*>(V), static_cast<const T*>(q),
-                                                                 static_cast<T*>(out), G, d);
+    if (cudaFuncSetAttribute(c3_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem) !=
+        cudaSuccess)
+      return KV_ERR_CUDA;
+    c3_attn_kernel<T><<<dim3(m.n_rows, G), kAttnThreads, attn_smem, cs>>>(
+        m, a, static_cast<const T*>(K), static_cast<const T*>(V), static_cast<const T*>(q), static_cast<T*>(out), G,
+        d, B);
   } else {
     using T = float;
     c3_score_kernel<T><<<sgrid, 128, 0, cs>>>(m, a, static_cast<const T*>(q), G, d, B);
     c3_select_kernel<<<m.n_rows, kScanThreads, 0, cs>>>(m, a, B);
-    c3_attn_kernel<T><<<dim3(m.n_rows, G), kAttnThreads, 0, cs>>>(m, a, static_cast<const T*>(K),
-                                                                 static_cast<const T*>(V), static_cast<const T*>(q),
-                                                                 static_cast<T*>(out), G, d);
+    if (cudaFuncSetAttribute(c3_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem) !=
+        cudaSuccess)
+      return KV_ERR_CUDA;
+    c3_attn_kernel<T><<<dim3(m.n_rows, G), kAttnThreads, attn_smem, cs>>>(
+        m, a, static_cast<const T*>(K), static_cast<const T*>(V), static_cast<const T*>(q), static_cast<T*>(out), G,
+        d, B);
   }
   c3_update_kernel<<<m.n_rows, kScanThreads, 0, cs>>>(m, a, B, p->lambda, p->exchanges);
   return cuda_status(cudaGetLastError());

@@ -76,36 +76,67 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{.reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p;}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: gives up once `abort` is raised by another thread of the CTA,
 // or after limit_ns of its own, in which case it raises `abort` and records
 // KV_DEV_TIMEOUT in the device status word. Returns false when it gave up.
+// A limit of 0 gives up on any wait whose phase has not completed already
+// (no suspended try), which lets a test drive every kernel's timeout path.
 struct Guard {
   volatile int* abort;  // shared-memory flag of the CTA
   int* status;          // device status word
   unsigned long long limit_ns;
 };
 
+__device__ __forceinline__ bool give_up(const Guard& g) {
+  *g.abort = 1;
+  atomicOr(g.status, KV_DEV_TIMEOUT);
+  return false;
+}
+
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Guard& g) {
+  if (g.limit_ns == 0) return mbar_test_wait(bar, parity) ? true : give_up(g);
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*g.abort) return false;
-    if (globaltimer() - t0 > g.limit_ns) {
-      *g.abort = 1;
-      atomicOr(g.status, KV_DEV_TIMEOUT);
-      return false;
-    }
+    if (globaltimer() - t0 > g.limit_ns) return give_up(g);
   }
 }
 
-// Wait used while draining after an abort: ignores the abort flag.
-__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+// Wait used while draining after an abort (copies or MMAs already issued
+// must land before the CTA releases its shared or tensor memory): ignores the
+// abort flag and has a limit of its own, independent of the waits' limit.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   uint64_t t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > limit_ns) return false;
+    if (globaltimer() - t0 > kDrainLimitNs) return false;
   }
+}
+
+// Named barrier over `nthreads` threads that also ANDs a predicate across them:
+// every participant gets the same result.
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{.reg .pred p, q; setp.ne.u32 p, %3, 0; bar.red.and.pred q, %1, %2, p; selp.u32 %0, 1, 0, q;}"
+      : "=r"(r)
+      : "r"(id), "r"(nthreads), "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------------- TMA
@@ -177,6 +208,18 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                : "memory");
 }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The same wait, with the 32 registers a tcgen05.ld filled as operands, so no
+// use of them can be scheduled before it.
+__device__ __forceinline__ void tc_wait_ld_regs(float (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]),
+                 "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]),
+                 "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]),
+                 "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+               :
+               : "memory");
+}
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -222,6 +265,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Arrive at a named barrier without waiting (the producer side of a hand-off).
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Programmatic dependent launch: let the next kernel in the stream start its

@@ -203,12 +203,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(const DecArg
           for (int e = 0; e < 4; ++e) acc[g][e] = fmaf(p, vv[e], acc[g][e]);
         }
     }
+    // the warps add their partials in warp order: a fixed summation order, so a
+    // step's result does not depend on scheduling
+    for (int w = 0; w < kDecWarps; ++w) {
+      if (warp == w) {
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
-      if (g < G)
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (e < per) atomicAdd(&o_s[g * d + lane * per + e], acc[g][e]);
+            for (int e = 0; e < 4; ++e)
+              if (e < per) o_s[g * d + lane * per + e] += acc[g][e];
+      }
+      __syncthreads();
+    }
   }
   cluster.sync();
 
@@ -414,12 +421,12 @@ int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (sh.dtype == KV_BF16) {
-      cudaFuncSetAttribute(decode_simple_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           200 * 1024);
-      e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<__nv_bfloat16>, a);
+      e = cudaFuncSetAttribute(decode_simple_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024);
+      if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<__nv_bfloat16>, a);
     } else {
-      cudaFuncSetAttribute(decode_simple_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<float>, a);
+      e = cudaFuncSetAttribute(decode_simple_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, decode_simple_kernel<float>, a);
     }
   }
   return cuda_status(e);

@@ -165,7 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cl_kernel(const __grid_con
   int k = 0;
   for (;; ++k) {
     const int stg = grp * kGStages + (k & 1);
-    const bool got = !aborted && wait_bounded(&full[stg], (k >> 1) & 1, gd);
+    // the group decides together whether the stage arrived (its warps' barriers
+    // and warp-wide instructions must not part)
+    const bool got = named_bar_and(1 + grp, 128, !aborted && wait_bounded(&full[stg], (k >> 1) & 1, gd));
     if (!got) aborted = true;
     const int st0 = got ? st0_s[stg] : -1;
     if (st0 < 0) break;
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cl_kernel(const __grid_con
     abort_s = 1;
     if (gt == 0)  // let this group's copies in flight land before the CTA goes on
       for (int tt = k; tt < nreal_s[grp]; ++tt)
-        wait_drain(&full[grp * kGStages + (tt & 1)], (tt >> 1) & 1, P.limit_ns);
+        wait_drain(&full[grp * kGStages + (tt & 1)], (tt >> 1) & 1);
   }
   // the group's running (max, sum, O): warps combined into (gm, gl) and og
   {
@@ -301,13 +303,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cl_kernel(const __grid_con
     if (g_ok)
       for (int w4 = 0; w4 < 4; ++w4) M0 = fmaxf(M0, red_m[grp * 4 + w4][g0]);
     const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
-    if (g_ok) {
+    // the group's warps add their O in warp order (a fixed summation order, so
+    // a step's result does not depend on scheduling); lanes own distinct columns
 #pragma unroll
-      for (int i = 0; i < 2 * NDC; ++i) {
-        const int col = i * 8 + q4 * 2;
-        atomicAdd(&og[g0 * D + ogswz(g0, col)], o[i][0] * f0);
-        atomicAdd(&og[g0 * D + ogswz(g0, col + 1)], o[i][1] * f0);
+    for (int w4 = 0; w4 < 4; ++w4) {
+      if (wq == w4 && g_ok) {
+#pragma unroll
+        for (int i = 0; i < 2 * NDC; ++i) {
+          const int col = i * 8 + q4 * 2;
+          og[g0 * D + ogswz(g0, col)] += o[i][0] * f0;
+          og[g0 * D + ogswz(g0, col + 1)] += o[i][1] * f0;
+        }
       }
+      if (w4 < 3) named_bar_sync(1 + grp, 128);
     }
     if (gt < G) {
       float M = -INFINITY;
@@ -514,7 +522,7 @@ int launch_cl(const kv_shape& sh, const RowMap& m, int capb, int C, long long to
   int cols = 32;
   while (cols < kGroups * P.cpg) cols <<= 1;
   P.ncols = cols;
-  P.limit_ns = kWaitLimitNs;
+  P.limit_ns = wait_limit_ns();
   const int stage_bytes = 2 * kTcSlots * sh.head_dim * 2 + kQBytes;
   const size_t smem = 1024 + (size_t)kStages * stage_bytes + (size_t)kGroups * sh.group * sh.head_dim * 4;
   CUtensorMap tmK, tmV, tmQ;

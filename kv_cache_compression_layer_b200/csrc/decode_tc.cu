@@ -5,11 +5,15 @@
 //
 // Every row's b + 1 slots are cut into work items of kCH slots; one CTA per
 // SM takes a contiguous run of items, so each CTA owns a contiguous range of
-// the slot space.
+// the slot space. The runs are cut at equal shares of a cost that counts the
+// slots and charges each row once more (a row costs its groups a combine of
+// their running softmax state and a partial written out), so CTAs holding
+// many short rows get fewer slots.
 //
 // Attention phase. Twelve warps form three groups of four. The CTA's items
-// are walked as a sequence of 64-slot tiles and group k takes the tiles with
-// index = k (mod 3). Each group feeds itself: its first thread streams its
+// are cut into three contiguous runs, one per group, walked as 64-slot tiles
+// (a row change then costs one group, not all three, a combine). Each group
+// feeds itself: its first thread streams its
 // tiles (K and V as 128-byte swizzled TMA boxes, the row's g query rows as a
 // bulk copy, a header with the row's step state) into the group's two
 // stages, and refills a stage as soon as the group has finished with it.
@@ -44,7 +48,7 @@ struct TcScratch {
   int2* items;     // [max_items] (row, chunk)
   float* part;     // [max_items * kGroups][stride]: max[G] at 0, sum[G] at G, O[G][d] at kPartO,
                    // per (first item of a group's segment, group)
-  float* logits;   // [total_slots][G] logits in log2 units
+  float* logits;   // [total_slots][8] logits in log2 units (heads >= G hold -inf)
   int* plist;      // [rows][max_per_row * kGroups] list entries (PEnt: per-head max and sum, index,
                    // step stamp), one place per (item that starts a group's segment, group)
   int* done;       // [rows] slots of the row finished in the current step
@@ -52,8 +56,16 @@ struct TcScratch {
   int4* bests;     // [rows][max_bests] proposals (A bits, pos, slot, -)
   unsigned* attn_done;  // [rows] slots of the row attended so far (grows by the row's capacity
                         // every step; the decode init clears it)
+  long long* row_cost;  // [rows + 1] prefix of the rows' costs (slots + kRowCost)
+  int* cta_u;           // [kMaxCtas + 1] first item of each CTA's run; cta_u[kMaxCtas] = the grid it was cut for
   int max_items, max_per_row, stride, max_bests;
 };
+
+// The cost of a row beyond its slots when cutting the CTAs' runs, in slots: a
+// row change makes a group combine its four warps' softmax state and write a
+// partial, during which its stages wait.
+constexpr int kRowCost = 256;
+constexpr int kMaxCtas = 1024;
 
 struct TcArgs {
   DecArgs a;
@@ -84,7 +96,7 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
   const size_t o_part = off;
   off += al((size_t)max_items * kGroups * stride * 4);
   const size_t o_log = off;
-  off += al((size_t)total_slots * G * 4);
+  off += al((size_t)total_slots * kTcMaxG * 4);
   const size_t o_pl = off;
   off += al((size_t)rows * per_row * kGroups * 80);
   const size_t o_done = off;
@@ -95,6 +107,10 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
   off += al((size_t)rows * max_bests * 16);
   const size_t o_ad = off;
   off += al((size_t)rows * 4);
+  const size_t o_rc = off;
+  off += al((size_t)(rows + 1) * 8);
+  const size_t o_cu = off;
+  off += al((size_t)(kMaxCtas + 1) * 4);
   if (sc && base) {
     sc->n_items = reinterpret_cast<int*>(base + o_n);
     sc->item_off = reinterpret_cast<int*>(base + o_ioff);
@@ -106,6 +122,8 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
     sc->best_n = reinterpret_cast<int*>(base + o_bn);
     sc->bests = reinterpret_cast<int4*>(base + o_best);
     sc->attn_done = reinterpret_cast<unsigned*>(base + o_ad);
+    sc->row_cost = reinterpret_cast<long long*>(base + o_rc);
+    sc->cta_u = reinterpret_cast<int*>(base + o_cu);
     sc->max_items = max_items;
     sc->max_per_row = per_row;
     sc->stride = stride;
@@ -114,18 +132,25 @@ size_t tc_layout(int rows, int G, int d, int capb, long long total_slots, char* 
   return off;
 }
 
-// Builds the work items of every row (rows cut into kCH-slot chunks) and
-// clears the per-row step counters; one block.
-__global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off, TcScratch sc,
+// Builds the work items of every row (rows cut into kCH-slot chunks), clears
+// the per-row step counters, and cuts the items into n_cta runs of equal cost
+// (slots + kRowCost per row); one block.
+__global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off, TcScratch sc, int n_cta,
                                 int32_t* __restrict__ status) {
   __shared__ int warp_tot[32];
+  __shared__ long long warp_cost[32];
   __shared__ int carry;
+  __shared__ long long carry_cost;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) carry = 0;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    carry_cost = 0;
+  }
   __syncthreads();
   for (int base = 0; base < n_rows; base += blockDim.x) {
     const int i = base + threadIdx.x;
     int own = 0;
+    long long cost = 0;
     if (i < n_rows) {
       const long long cap = slot_off[i + 1] - slot_off[i];
       own = (int)((cap + kCH - 1) / kCH);
@@ -133,32 +158,74 @@ __global__ void tc_items_kernel(int n_rows, const int64_t* __restrict__ slot_off
         atomicOr(status, KV_DEV_CAPACITY);
         own = sc.max_per_row;
       }
+      cost = cap + kRowCost;
     }
     int v = own;
+    long long vc = cost;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += y;
+      const long long yc = __shfl_up_sync(0xffffffffu, vc, o);
+      if (lane >= o) {
+        v += y;
+        vc += yc;
+      }
     }
-    if (lane == 31) warp_tot[warp] = v;
+    if (lane == 31) {
+      warp_tot[warp] = v;
+      warp_cost[warp] = vc;
+    }
     __syncthreads();
     int wb = 0;
-    for (int k = 0; k < warp; ++k) wb += warp_tot[k];
+    long long wbc = 0;
+    for (int k = 0; k < warp; ++k) {
+      wb += warp_tot[k];
+      wbc += warp_cost[k];
+    }
     const int incl = carry + wb + v;
+    const long long incl_c = carry_cost + wbc + vc;
     if (i < n_rows) {
       sc.done[i] = 0;
       sc.best_n[i] = 0;
       sc.attn_done[i] = 0;
       sc.item_off[i] = incl - own;
+      sc.row_cost[i] = incl_c - cost;
       for (int c = 0; c < own; ++c) sc.items[incl - own + c] = make_int2(i, c);
     }
     __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry = incl;
+    if (threadIdx.x == blockDim.x - 1) {
+      carry = incl;
+      carry_cost = incl_c;
+    }
     __syncthreads();
   }
   if (threadIdx.x == 0) {
     sc.item_off[n_rows] = carry;
+    sc.row_cost[n_rows] = carry_cost;
     *sc.n_items = carry;
+  }
+  __syncthreads();
+  // CTA b starts at the first item whose cost prefix reaches total * b / n_cta:
+  // item c of row i starts at P_i (c = 0) or P_i + kRowCost + c kCH (c >= 1)
+  const long long total = carry_cost;
+  const int n_items = carry;
+  for (int i = threadIdx.x; i < n_rows; i += blockDim.x) {
+    const long long P0 = sc.row_cost[i], P1 = sc.row_cost[i + 1];
+    const int own = sc.item_off[i + 1] - sc.item_off[i];
+    // the boundaries b with P0 < total * b / n_cta <= P1
+    int b = (int)((P0 * n_cta) / total);
+    while ((total * b) / n_cta <= P0) ++b;
+    for (; b < n_cta && (total * b) / n_cta <= P1; ++b) {
+      const long long T = (total * b) / n_cta;
+      long long c = (T - P0 - kRowCost + kCH - 1) / kCH;
+      if (c < 1) c = 1;
+      sc.cta_u[b] = c < own ? sc.item_off[i] + (int)c : sc.item_off[i] + own;
+    }
+  }
+  if (threadIdx.x == 0) {
+    sc.cta_u[0] = 0;
+    sc.cta_u[n_cta] = n_items;
+    sc.cta_u[kMaxCtas] = n_cta;
   }
 }
 
@@ -233,13 +300,6 @@ __device__ __forceinline__ bool walk_advance(Walk& w, const DecArgs& a, int max_
   return true;
 }
 
-// Moves to the next tile that group `grp` takes.
-__device__ __forceinline__ bool walk_next(Walk& w, int grp, const DecArgs& a, int max_per_row) {
-  for (;;) {
-    if (!walk_advance(w, a, max_per_row)) return false;
-    if (w.it % kGroups == grp) return true;
-  }
-}
 
 // Streams the walk's current tile into a stage: header, K and V boxes, query rows.
 template <int D>
@@ -468,23 +528,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const Guard gd{&abort_s, a.status, P.limit_ns};
   const int maxp = sc.max_per_row * kGroups;
   const int n_items = *sc.n_items;
-  const int u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
-  const int u1 = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
+  // this CTA's run of items: cut by cost at decode init for this grid, else equal counts
+  int u0, u1;
+  if (sc.cta_u[kMaxCtas] == (int)gridDim.x) {
+    u0 = sc.cta_u[blockIdx.x];
+    u1 = sc.cta_u[blockIdx.x + 1];
+  } else {
+    u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
+    u1 = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
+  }
 
   // ---------------------------------------------------------------- attention
   {
     Walk& w = walk_s[grp];
     if (gt == 0) {
       const uint64_t stream_policy = make_policy_evict_first();  // K and V are read once per step
-      int more = walk_first(w, a, sc, u0, u1);
-      if (more && w.it % kGroups != grp) more = walk_next(w, grp, a, sc.max_per_row);
+      // this group's contiguous share of the CTA's items
+      const int gu0 = u0 + (int)((long long)(u1 - u0) * grp / kGroups);
+      const int gu1 = u0 + (int)((long long)(u1 - u0) * (grp + 1) / kGroups);
+      int more = walk_first(w, a, sc, gu0, gu1);
       int ended = 0, n_real = 0;
       for (int s = 0; s < kGStages && !ended; ++s) {
         const int stg = grp * kGStages + s;
         if (more) {
           issue_tile<D>(w, ring + stg * STAGE, &full[stg], &hdr[stg], &tmK, &tmV, &tmQ, a, stream_policy);
           ++n_real;
-          more = walk_next(w, grp, a, sc.max_per_row);
+          more = walk_advance(w, a, sc.max_per_row);
         } else {
           hdr[stg].row = -1;
           mbar_arrive(&full[stg]);
@@ -528,7 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     int k = 0;
     for (;; ++k) {
       const int stg = grp * kGStages + (k & 1);
-      const bool got = !aborted && wait_bounded(&full[stg], (k >> 1) & 1, gd);
+      // the group decides together whether the stage arrived (its warps' barriers
+      // and warp-wide instructions must not part)
+      const bool got = named_bar_and(1 + grp, 128, !aborted && wait_bounded(&full[stg], (k >> 1) & 1, gd));
       if (!got) aborted = true;
       const int hrow = got ? hdr[stg].row : -1;  // -1: sentinel (or abort)
       if (hrow != cur_row || hrow < 0) {
@@ -547,15 +618,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           if (g_ok)
             for (int w4 = 0; w4 < 4; ++w4) M0 = fmaxf(M0, red_m[grp * 4 + w4][g0]);
           const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
-          if (g_ok) {
+          // the group's warps add their O in warp order (a fixed summation order,
+          // so a step's result does not depend on scheduling); lanes own distinct columns
 #pragma unroll
-            for (int i = 0; i < 2 * NDC; ++i) {
-              const int col = i * 8 + q4 * 2;
-              atomicAdd(&og[g0 * D + ogswz(g0, col)], o[i][0] * f0);
-              atomicAdd(&og[g0 * D + ogswz(g0, col + 1)], o[i][1] * f0);
+          for (int w4 = 0; w4 < 4; ++w4) {
+            if ((warp & 3) == w4 && g_ok) {
+#pragma unroll
+              for (int i = 0; i < 2 * NDC; ++i) {
+                const int col = i * 8 + q4 * 2;
+                og[g0 * D + ogswz(g0, col)] += o[i][0] * f0;
+                og[g0 * D + ogswz(g0, col + 1)] += o[i][1] * f0;
+              }
             }
+            named_bar_sync(1 + grp, 128);
           }
-          named_bar_sync(1 + grp, 128);
           const int pidx = seg_u * kGroups + grp;
           float* part = sc.part + (long long)pidx * sc.stride;
           // the row's list place of this partial: (the segment's first item in the row, group)
@@ -665,7 +741,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const int j = jb + (e & 1) + (e >> 1) * 8;
         const bool valid = row_ok && j < n && j < h.c1;
         x[e] = valid ? x[e] * a.scale2 : -INFINITY;
-        if (valid && g_ok) st_f32_hint(sc.logits + (base + j) * G + g0, x[e], keep_policy);
+        // eight logits per slot: the lanes of heads >= G store -inf, so the finish
+        // reads every slot's logits as two aligned float4 whatever G is
+        if (valid) st_f32_hint(sc.logits + (base + j) * kTcMaxG + g0, g_ok ? x[e] : -INFINITY, keep_policy);
       }
       // online softmax update of this warp's running (max, sum, O)
       float tm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
@@ -708,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (more_s[grp]) {
           issue_tile<D>(w, stage, &full[stg], &hdr[stg], &tmK, &tmV, &tmQ, a, make_policy_evict_first());
           ++nreal_s[grp];
-          more_s[grp] = walk_next(w, grp, a, sc.max_per_row);
+          more_s[grp] = walk_advance(w, a, sc.max_per_row);
         } else if (!ended_s[grp]) {
           hdr[stg].row = -1;
           mbar_arrive(&full[stg]);
@@ -723,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     if (aborted) {
       abort_s = 1;
       if (gt == 0)  // let this group's copies in flight land before the CTA exits
-        for (int t = k; t < nreal_s[grp]; ++t) wait_drain(&full[grp * kGStages + (t & 1)], (t >> 1) & 1, P.limit_ns);
+        for (int t = k; t < nreal_s[grp]; ++t) wait_drain(&full[grp * kGStages + (t & 1)], (t >> 1) & 1);
     }
   }
   __syncthreads();
@@ -752,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   int* st_pos = reinterpret_cast<int*>(st_A + kStgSlots);    // [kStgSlots]
   long long stg0 = 0;
   int nst = 0;
-  if (G == kTcMaxG) {
+  {
     const int rn0 = min(kRowsBatch, r_hi - r_lo + 1);
     stg0 = max(S0, rowc[0].base);
     const long long stg1 = min(S1, rowc[rn0 - 1].base + rowc[rn0 - 1].cap);
@@ -815,83 +893,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         float lse[kTcMaxG];
 #pragma unroll
         for (int g = 0; g < kTcMaxG; ++g) lse[g] = g < G ? rs[ri].lse[g] : 0.f;
-        if (G == kTcMaxG) {
-          // lane pairs share a slot: each lane loads 4 of its 8 logits, so a warp's
-          // request is 512 contiguous bytes
-          constexpr int U = UP;
-          const int half = lane & 1, sl = lane >> 1;
-          float lh[4];
+        // lane pairs share a slot: each lane loads 4 of its 8 logits, so a warp's
+        // request is 512 contiguous bytes
+        constexpr int U = UP;
+        const int half = lane & 1, sl = lane >> 1;
+        float lh[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) lh[k] = half ? lse[4 + k] : lse[k];
-          for (long long s0 = p0; s0 < p1; s0 += 16 * U) {
-            float4 lv[U];
-            float Av[U];
-            int pv[U];
-            if (s0 >= stg0 && min(s0 + 16 * U, p1) <= stg0 + nst) {  // staged in shared memory
-#pragma unroll
-              for (int uu = 0; uu < U; ++uu) {
-                const int k = (int)(min(s0 + uu * 16 + sl, p1 - 1) - stg0);
-                lv[uu] = *reinterpret_cast<const float4*>(st_lg + k * kTcMaxG + half * 4);
-                Av[uu] = st_A[k];
-                pv[uu] = st_pos[k];
-              }
-            } else {
-#pragma unroll
-              for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
-                const long long s = min(s0 + uu * 16 + sl, p1 - 1);
-                lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
-                Av[uu] = __ldcg(a.A + s);
-                pv[uu] = __ldcg(a.pos + s);
-              }
-            }
+        for (int k = 0; k < 4; ++k) lh[k] = half ? lse[4 + k] : lse[k];
+        for (long long s0 = p0; s0 < p1; s0 += 16 * U) {
+          float4 lv[U];
+          float Av[U];
+          int pv[U];
+          if (s0 >= stg0 && min(s0 + 16 * U, p1) <= stg0 + nst) {  // staged in shared memory
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {
-              float ps = ex2_approx(lv[uu].x - lh[0]) + ex2_approx(lv[uu].y - lh[1]) + ex2_approx(lv[uu].z - lh[2]) +
-                         ex2_approx(lv[uu].w - lh[3]);
-              ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-              const long long s = s0 + uu * 16 + sl;
-              const int j = (int)(s - rbase);
-              if (half == 0 && s < p1 && j < rn_) {
-                const float Anew = (j == rnext ? 0.f : a.gamma * Av[uu]) + ps;
-                st_f32_hint_nc(a.A + s, Anew, keep);  // read again by the next step
-                const int pj = j == rnext ? rpos_new : pv[uu];
-                if (j >= a.T && pj < rpos_thr) {
-                  const Best c{Anew, pj, j};
-                  if (better(c, best)) best = c;
-                }
-              }
+              const int k = (int)(min(s0 + uu * 16 + sl, p1 - 1) - stg0);
+              lv[uu] = *reinterpret_cast<const float4*>(st_lg + k * kTcMaxG + half * 4);
+              Av[uu] = st_A[k];
+              pv[uu] = st_pos[k];
             }
-          }
-        } else {
-          constexpr int U = 4;  // slots per lane in flight
-          for (long long s0 = p0; s0 < p1; s0 += 32 * U) {
-            float lg[U][kTcMaxG];
-            float Av[U];
-            int pv[U];
+          } else {
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
-              const long long s = min(s0 + uu * 32 + lane, p1 - 1);
+              const long long s = min(s0 + uu * 16 + sl, p1 - 1);
+              lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
               Av[uu] = __ldcg(a.A + s);
               pv[uu] = __ldcg(a.pos + s);
-              const float* lgp = sc.logits + s * G;
-#pragma unroll
-              for (int g = 0; g < kTcMaxG; ++g) lg[uu][g] = g < G ? __ldcg(lgp + g) : -INFINITY;
             }
+          }
 #pragma unroll
-            for (int uu = 0; uu < U; ++uu) {
-              const long long s = s0 + uu * 32 + lane;
-              const int j = (int)(s - rbase);
-              if (s < p1 && j < rn_) {
-                float ps = 0.f;
-#pragma unroll
-                for (int g = 0; g < kTcMaxG; ++g) ps += ex2_approx(lg[uu][g] - lse[g]);
-                const float Anew = (j == rnext ? 0.f : a.gamma * Av[uu]) + ps;
-                st_f32_hint_nc(a.A + s, Anew, keep);  // read again by the next step
-                const int pj = j == rnext ? rpos_new : pv[uu];
-                if (j >= a.T && pj < rpos_thr) {
-                  const Best c{Anew, pj, j};
-                  if (better(c, best)) best = c;
-                }
+          for (int uu = 0; uu < U; ++uu) {
+            float ps = ex2_approx(lv[uu].x - lh[0]) + ex2_approx(lv[uu].y - lh[1]) + ex2_approx(lv[uu].z - lh[2]) +
+                       ex2_approx(lv[uu].w - lh[3]);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+            const long long s = s0 + uu * 16 + sl;
+            const int j = (int)(s - rbase);
+            if (half == 0 && s < p1 && j < rn_) {
+              const float Anew = (j == rnext ? 0.f : a.gamma * Av[uu]) + ps;
+              st_f32_hint_nc(a.A + s, Anew, keep);  // read again by the next step
+              const int pj = j == rnext ? rpos_new : pv[uu];
+              if (j >= a.T && pj < rpos_thr) {
+                const Best c{Anew, pj, j};
+                if (better(c, best)) best = c;
               }
             }
           }
@@ -1034,7 +1077,8 @@ int launch_tc_init(const kv_shape& sh, const RowMap& m, int capb, long long tota
   // list entries carry the step they belong to: clear the stamps of any earlier decode
   if (cudaMemsetAsync(sc.plist, 0, (size_t)m.n_rows * sc.max_per_row * kGroups * sizeof(PEnt), st) != cudaSuccess)
     return KV_ERR_CUDA;
-  tc_items_kernel<<<1, 1024, 0, st>>>(m.n_rows, c.slot_off, sc, c.status);
+  const int n_cta = std::min(sm_count(), kMaxCtas);  // the decode grid (one CTA per SM)
+  tc_items_kernel<<<1, 1024, 0, st>>>(m.n_rows, c.slot_off, sc, n_cta, c.status);
   return cuda_status(cudaGetLastError());
 }
 
@@ -1043,7 +1087,7 @@ int launch_tc(const kv_shape& sh, const RowMap& m, int capb, long long total_slo
   if (total_slots >= (1ll << 31)) return KV_ERR_ARG;  // slot indices are TMA coordinates (int32)
   TcArgs P;
   P.a = a;
-  P.limit_ns = kWaitLimitNs;
+  P.limit_ns = wait_limit_ns();
   const size_t need = tc_layout(m.n_rows, sh.group, sh.head_dim, capb, total_slots, (char*)c.scratch, &P.sc);
   if (!c.scratch || c.scratch_bytes < need) return KV_ERR_WORKSPACE;
   const int stage_bytes = 2 * kTcSlots * sh.head_dim * 2 + kQBytes;
@@ -1061,7 +1105,7 @@ int launch_tc(const kv_shape& sh, const RowMap& m, int capb, long long total_slo
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(sm_count());  // one CTA per SM (shared memory), all resident for the grid barrier
+  cfg.gridDim = dim3(std::min(sm_count(), kMaxCtas));  // one CTA per SM (shared memory), all resident
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;

@@ -41,9 +41,11 @@ int launch_decode_init(const kv_shape& sh, const RowMap& m, const kv_params& p, 
 int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const kv_cache& c, const void* q_t,
                   const void* k_t, const void* v_t, void* out, cudaStream_t st);
 
-// Bounded device waits give up after this long (a safety net; never reached
-// by a correct run).
+// Bounded device waits give up after this long by default (a safety net;
+// never reached by a correct run); kv_set_wait_limit_ns changes it for later
+// launches, and wait_limit_ns() is the value a launch passes to its kernels.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+unsigned long long wait_limit_ns();
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? KV_OK : KV_ERR_CUDA; }
 

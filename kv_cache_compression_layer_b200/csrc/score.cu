@@ -13,8 +13,15 @@
 // Both passes are persistent (one CTA per SM, contiguous runs of tiles) and
 // warp-specialised: warp 0 issues TMA loads of Q and a 4-stage ring of K
 // tiles, warp 1 issues tcgen05.mma into a double-buffered TMEM accumulator,
-// warps 2-9 (two groups of four, one group per accumulator buffer) read TMEM
-// with tcgen05.ld and do the softmax arithmetic.
+// warps 2-17 read TMEM with tcgen05.ld and do the softmax arithmetic: four
+// groups of four warps (one warp per TMEM lane quarter), two groups per
+// accumulator buffer. In pass 1 the two groups of a buffer take the two
+// halves of the window rows (a warp whose 32 rows all lie at or beyond R does
+// nothing); in pass 2 they take the two halves of the R columns, and the
+// first half hands its per-key sums to the second through shared memory
+// (added in a fixed order). The exponentials are the binding unit, so the
+// epilogue reads TMEM in 32-column chunks and overlaps each chunk's load with
+// the previous chunk's arithmetic; pass 1 keeps a running maximum per row.
 //
 // fp32 path (fp32 inputs): the same three steps on CUDA cores (FFMA), since
 // a tf32 contraction would not meet the fp32 tolerance.
@@ -28,7 +35,8 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kQRows = 256;
-constexpr int kThreads = 320;
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kQChunkBytes = kQRows * 128;      // 256 rows x 64 bf16
 constexpr int kKChunkBytes = kTileKeys * 128;   // 128 keys x 64 bf16
 constexpr int kKStageBytes = 2 * kKChunkBytes;  // d <= 128
@@ -37,7 +45,8 @@ constexpr int kSmemK = 2 * kQChunkBytes;
 constexpr int kSmemBar = kSmemK + kStages * kKStageBytes;
 constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int kSmemMisc = kSmemBar + kNumBars * 8;
-constexpr int kSmemTotal = kSmemMisc + 16;
+constexpr int kSmemPart = kSmemMisc + 16;                  // pass 2: [buffer][parity][128 keys] float
+constexpr int kSmemTotal = kSmemPart + 2 * 2 * kTileKeys * 4;
 constexpr int kSmemAlloc = kSmemTotal + 1024;  // slack for 1024-byte alignment
 
 struct TcArgs {
@@ -47,12 +56,27 @@ struct TcArgs {
   int nk;     // 64-element chunks of d (1 or 2)
   int total_tiles;
   float c;    // log2(e) / sqrt(d)
+  int Rs;     // row stride of lse2: R rounded up to 4 (16-byte rows)
   float2* partial;     // pass 1 out: [total_tiles][R] (tile max, tile sum)
-  const float* lse2;   // pass 2 in:  [rows][R]
+  const float* lse2;   // pass 2 in:  [rows][Rs]
   float* s;            // pass 2 out: [sum L]
   int* status;
   unsigned long long limit_ns;
 };
+
+// Epilogue warps with work per accumulator buffer: pass 1, the (row half,
+// lane quarter) pairs holding some row < R; pass 2, four per column half that
+// holds a 32-column chunk (the first half is empty when there is one chunk).
+template <int PASS>
+__host__ __device__ constexpr int epi_active_warps(int R, int n2) {
+  if (PASS == 1) {
+    int n = 0;
+    for (int h = 0; h < 2; ++h)
+      for (int q = 0; q < 4; ++q) n += h * 128 + q * 32 < R ? 1 : 0;
+    return n;
+  }
+  return ((n2 + 31) / 32) / 2 > 0 ? 8 : 4;
+}
 
 template <int PASS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -87,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], epi_active_warps<PASS>(a.R, a.n2));
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -140,12 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         k_issued[st] = true;
         k_parity[st] = (it / kStages) & 1;
       }
-      if (aborted || *abort_flag) {
-        // let the copies in flight land before the CTA's shared memory goes away
-        for (int st = 0; st < kStages; ++st)
-          if (k_issued[st]) wait_drain(&full_k[st], k_parity[st], a.limit_ns);
-        if (have_q) wait_drain(q_full, q_parity, a.limit_ns);
-      }
+      // let every copy issued land before the CTA's shared memory goes away (after
+      // a normal run they all have; after an abort raised anywhere some may not)
+      (void)aborted;
+      for (int st = 0; st < kStages; ++st)
+        if (k_issued[st]) wait_drain(&full_k[st], k_parity[st]);
+      if (have_q) wait_drain(q_full, q_parity);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
@@ -192,79 +216,120 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every issued MMA has finished before TMEM is released
       tc_commit(drain);
-      wait_drain(drain, 0, a.limit_ns);
+      wait_drain(drain, 0);
     }
   } else {
     // ------------------------------------------------------ epilogue
-    const int eg = (warp - 2) >> 2;  // accumulator buffer this group owns
-    const int quarter = warp & 3;    // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int e = warp - 2;
+    const int quarter = warp & 3;         // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int bf = (e >> 2) >> 1;         // accumulator buffer of this warp's group
+    const int half = (e >> 2) & 1;        // pass 1: rows [128 half, ...); pass 2: column half
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    for (int u = u0 + eg; u < u1; u += 2) {
+    const int nc = (a.n2 + 31) / 32;      // pass 2: 32-column chunks of the accumulator
+    const int c_lo = half ? nc / 2 : 0, c_hi = half ? nc : nc / 2;
+    const bool active = PASS == 1 ? half * 128 + quarter * 32 < a.R : c_lo < c_hi;
+    const bool pair = PASS == 2 && nc / 2 > 0;  // both column halves active: hand-off through shared memory
+    const int n_pair = 32 * epi_active_warps<PASS>(a.R, a.n2);  // pass 2: the buffer's threads
+    float* part = reinterpret_cast<float*>(smem + kSmemPart);
+    for (int u = u0 + bf; active && u < u1; u += 2) {
       const int it = u - u0;
       int row, tile;
       tile_to_row(a.map, u, row, tile);
       const int nvalid = min(kTileKeys, row_len(a.map, row) - tile * kTileKeys);
-      if (!wait_bounded(&acc_full[eg], (it >> 1) & 1, g)) break;
+      // the warp (pass 2: the buffer's warps) leave together: tensor-memory loads are
+      // warp-wide and the column halves meet at a barrier
+      bool ok = __all_sync(0xffffffffu, wait_bounded(&acc_full[bf], (it >> 1) & 1, g));
+      if (pair) ok = named_bar_and(1 + bf, n_pair, ok);
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + lane_addr + eg * 256;
-      float x[4][32];
+      const uint32_t tbase = tmem + lane_addr + bf * 256;
+      float xa[32], xb[32];
+      // every tensor-memory load of this warp has completed: the buffer may be refilled
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[bf]);
+      };
       if (PASS == 1) {
-        for (int h = 0; h * 128 < a.R; ++h) {
+        // this thread's window row: running max m and sum Z over the tile's keys,
+        // chunk by chunk (chunks of keys at or beyond nvalid are skipped)
+        const uint32_t hb = tbase + half * 128;
+        const int r = half * 128 + quarter * 32 + lane;
+        float m = -INFINITY, Z = 0.f;
+        auto rowstats = [&](const float (&x)[32], int ch) {
+          if (ch * 32 >= nvalid) return;
+          float mx = -INFINITY;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) tmem_ld32(tbase + h * 128 + cc * 32, x[cc]);
-          tc_wait_ld();
-          const bool last = (h + 1) * 128 >= a.R;
-          if (last) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[eg]);
+          for (int i = 0; i < 32; ++i)
+            if (ch * 32 + i < nvalid) mx = fmaxf(mx, x[i]);
+          if (mx > m) {
+            Z = m == -INFINITY ? 0.f : Z * ex2_approx((m - mx) * a.c);
+            m = mx;
           }
-          const int r = h * 128 + quarter * 32 + lane;
-          float m = -INFINITY;
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (cc * 32 + i < nvalid) m = fmaxf(m, x[cc][i]);
           const float mc = m * a.c;
-          float Z = 0.f;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (cc * 32 + i < nvalid) Z += ex2_approx(fmaf(x[cc][i], a.c, -mc));
-          if (r < a.R) a.partial[(long long)u * a.R + r] = make_float2(m, Z);
-        }
+          for (int i = 0; i < 32; ++i)
+            if (ch * 32 + i < nvalid) Z += ex2_approx(fmaf(x[i], a.c, -mc));
+        };
+        tmem_ld32(hb, xa);
+        tc_wait_ld_regs(xa);
+        tmem_ld32(hb + 32, xb);
+        rowstats(xa, 0);
+        tc_wait_ld_regs(xb);
+        tmem_ld32(hb + 64, xa);
+        rowstats(xb, 1);
+        tc_wait_ld_regs(xa);
+        tmem_ld32(hb + 96, xb);
+        rowstats(xa, 2);
+        tc_wait_ld_regs(xb);
+        release();
+        rowstats(xb, 3);
+        if (r < a.R) a.partial[(long long)u * a.R + r] = make_float2(m, Z);
       } else {
+        // this thread's key: the sum over its half of the window rows of
+        // exp2(x c - lse_r), chunk by chunk
         const int j = quarter * 32 + lane;
-        const float* lse = a.lse2 + (long long)row * a.R;
+        const float* lse = a.lse2 + (long long)row * a.Rs;
         float sum = 0.f;
-        for (int cb = 0; cb * 128 < a.R; ++cb) {
+        auto colsum = [&](const float (&x)[32], int ch) {
+          const int col = ch * 32;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            if (cb * 128 + cc * 32 < a.n2) tmem_ld32(tbase + cb * 128 + cc * 32, x[cc]);
-          tc_wait_ld();
-          if ((cb + 1) * 128 >= a.R) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[eg]);
-          }
+          for (int i = 0; i < 32; i += 4) {
+            if (col + i < a.R) {
+              const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse + col + i));
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int col = cb * 128 + cc * 32;
-            if (col < a.R) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse + col + i));
-                sum += ex2_approx(fmaf(x[cc][i + 0], a.c, -l4.x));
-                sum += ex2_approx(fmaf(x[cc][i + 1], a.c, -l4.y));
-                sum += ex2_approx(fmaf(x[cc][i + 2], a.c, -l4.z));
-                sum += ex2_approx(fmaf(x[cc][i + 3], a.c, -l4.w));
-              }
+              for (int q = 0; q < 4; ++q)
+                if (col + i + q < a.R) sum += ex2_approx(fmaf(x[i + q], a.c, -lv[q]));
             }
           }
+        };
+        tmem_ld32(tbase + c_lo * 32, xa);
+        tc_wait_ld_regs(xa);
+        for (int ch = c_lo; ch < c_hi; ch += 2) {  // xa holds chunk ch
+          const bool has1 = ch + 1 < c_hi, has2 = ch + 2 < c_hi;
+          if (has1) tmem_ld32(tbase + (ch + 1) * 32, xb);
+          else release();
+          colsum(xa, ch);
+          if (has1) {
+            tc_wait_ld_regs(xb);
+            if (has2) tmem_ld32(tbase + (ch + 2) * 32, xa);
+            else release();
+            colsum(xb, ch + 1);
+            if (has2) tc_wait_ld_regs(xa);
+          }
         }
-        if (j < nvalid) a.s[row_key_off(a.map, row) + (long long)tile * kTileKeys + j] = sum;
+        float* pb = part + (bf * 2 + ((it >> 1) & 1)) * kTileKeys;
+        if (pair && half == 0) {  // hand the first half's sums to the second
+          pb[j] = sum;
+          named_bar_arrive(3 + bf, n_pair);
+        } else {
+          if (pair) {
+            named_bar_sync(3 + bf, n_pair);
+            sum = pb[j] + sum;  // first half + second half, in that order
+          }
+          if (j < nvalid) a.s[row_key_off(a.map, row) + (long long)tile * kTileKeys + j] = sum;
+        }
       }
     }
   }
@@ -277,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Softmax denominators of every (row, window row) from the tile partials.
-__global__ void score_merge_kernel(const RowMap map, int R, float c, const float2* __restrict__ partial,
+__global__ void score_merge_kernel(const RowMap map, int R, int Rs, float c, const float2* __restrict__ partial,
                                    float* __restrict__ lse2) {
   const int row = blockIdx.x, r = threadIdx.x;
   if (r >= R) return;
@@ -294,7 +359,7 @@ __global__ void score_merge_kernel(const RowMap map, int R, float c, const float
       Z += p.y * exp2f((p.x - m) * c);
     }
   }
-  lse2[(long long)row * R + r] = m * c + log2f(Z);
+  lse2[(long long)row * Rs + r] = m * c + log2f(Z);
 }
 
 // fp32 inputs: row statistics of one 128-key tile on CUDA cores.
@@ -353,7 +418,7 @@ __global__ void score_f32_colsum_kernel(const RowMap map, int R, int d, float c,
   }
   const float* Qr = qwin + (long long)row * R * d;
   for (int i = threadIdx.x; i < R * d; i += blockDim.x) Qs[(i / d) * dp + i % d] = Qr[i];
-  for (int i = threadIdx.x; i < R; i += blockDim.x) Ls[i] = lse2[(long long)row * R + i];
+  for (int i = threadIdx.x; i < R; i += blockDim.x) Ls[i] = lse2[(long long)row * ((R + 3) & ~3) + i];
   __syncthreads();
   const int j = threadIdx.x;
   if (j >= nvalid) return;
@@ -374,7 +439,7 @@ ScoreWs score_ws_layout(const RowMap& m, int R) {
   w.status_off = 0;
   w.partial_off = 256;
   w.lse_off = w.partial_off + (((size_t)tiles * R * sizeof(float2) + 255) & ~size_t(255));
-  w.bytes = w.lse_off + (((size_t)m.n_rows * R * sizeof(float) + 255) & ~size_t(255));
+  w.bytes = w.lse_off + (((size_t)m.n_rows * ((R + 3) & ~3) * sizeof(float) + 255) & ~size_t(255));
   return w;
 }
 
@@ -396,14 +461,16 @@ int launch_score(const kv_shape& sh, const RowMap& m, const void* qwin, const vo
     CUtensorMap tmQ, tmK;
     if (!encode_rows_bf16(&tmQ, qwin, d, (long long)m.n_rows * R, kQRows)) return KV_ERR_CUDA;
     if (!encode_rows_bf16(&tmK, K, d, total_keys(m), kTileKeys)) return KV_ERR_CUDA;
-    static std::once_flag attr_once;
-    std::call_once(attr_once, [] {
-      cudaFuncSetAttribute(score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-      cudaFuncSetAttribute(score_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    });
+    // per-device settings: made on every launch (cheap), for whichever device is current
+    if (cudaFuncSetAttribute(score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(score_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
+            cudaSuccess)
+      return KV_ERR_CUDA;
     TcArgs a;
     a.map = m;
     a.R = R;
+    a.Rs = (R + 3) & ~3;
     a.n2 = ((R + 15) / 16) * 16;
     a.nk = d / 64;
     a.total_tiles = total_tiles;
@@ -412,23 +479,23 @@ int launch_score(const kv_shape& sh, const RowMap& m, const void* qwin, const vo
     a.lse2 = lse2;
     a.s = s;
     a.status = status;
-    a.limit_ns = kWaitLimitNs;
+    a.limit_ns = wait_limit_ns();
     const int grid = std::min(sm_count(), total_tiles);
     score_tc_kernel<1><<<grid, kThreads, kSmemAlloc, st>>>(tmQ, tmK, a);
-    score_merge_kernel<<<m.n_rows, merge_threads, 0, st>>>(m, R, c, partial, lse2);
+    score_merge_kernel<<<m.n_rows, merge_threads, 0, st>>>(m, R, (R + 3) & ~3, c, partial, lse2);
     score_tc_kernel<2><<<grid, kThreads, kSmemAlloc, st>>>(tmQ, tmK, a);
   } else {
     const size_t sm1 = (size_t)(kTileKeys + R) * (d + 1) * sizeof(float);
     const size_t sm2 = sm1 + (size_t)R * sizeof(float);
-    static std::once_flag attr_once;
-    std::call_once(attr_once, [] {
-      cudaFuncSetAttribute(score_f32_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-      cudaFuncSetAttribute(score_f32_colsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    });
+    if (cudaFuncSetAttribute(score_f32_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(score_f32_colsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024) !=
+            cudaSuccess)
+      return KV_ERR_CUDA;
     const float* q = static_cast<const float*>(qwin);
     const float* Kf = static_cast<const float*>(K);
     score_f32_stats_kernel<<<total_tiles, 128, sm1, st>>>(m, R, d, c, q, Kf, partial);
-    score_merge_kernel<<<m.n_rows, merge_threads, 0, st>>>(m, R, c, partial, lse2);
+    score_merge_kernel<<<m.n_rows, merge_threads, 0, st>>>(m, R, (R + 3) & ~3, c, partial, lse2);
     score_f32_colsum_kernel<<<total_tiles, 128, sm2, st>>>(m, R, d, c, q, Kf, lse2, s);
   }
   return cuda_status(cudaGetLastError());

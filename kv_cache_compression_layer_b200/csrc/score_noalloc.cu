@@ -11,8 +11,6 @@
 // device array below, sized for batches up to KV_NOALLOC_SCRATCH_BYTES of
 // scratch, which every GPU that loads the library holds until the process
 // exits.
-#include <mutex>
-
 #include "internal.h"
 
 namespace kvc {
@@ -20,22 +18,14 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_score_scratch[KV_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side symbol is only a stand-in, never a device address).
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a stand-in, never a device address, so it is looked up
+// on every call (a cheap host query): a cached address could outlive the
+// module after a device reset.
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KV_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_score_scratch) != cudaSuccess || !p) return KV_ERR_CUDA;
-    g_addr[dev] = p;
-  }
-  *out = g_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_score_scratch) != cudaSuccess || !p) return KV_ERR_CUDA;
+  *out = p;
   return KV_OK;
 }
 
@@ -53,4 +43,14 @@ extern "C" int kv_score_noalloc(const kv_shape* shape, const int32_t* L, int32_t
   const int st = scratch_address(&scratch);
   if (st != KV_OK) return st;
   return kv_score(shape, L, n_seq, qwin, K, s, scratch, KV_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// The status word of the last kv_score_noalloc call on the current device
+// sits at the start of the array (kv_score's workspace layout).
+extern "C" int kv_score_noalloc_status(int32_t* status_host, void* stream) {
+  if (!status_host) return KV_ERR_ARG;
+  void* scratch = nullptr;
+  const int st = scratch_address(&scratch);
+  if (st != KV_OK) return st;
+  return kv_read_device_status(static_cast<const int32_t*>(scratch), status_host, stream);
 }

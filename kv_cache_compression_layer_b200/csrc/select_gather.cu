@@ -3,8 +3,9 @@
 // row's budget goes to the highest smoothed scores; the C3 page's bypass keeps
 // every position once the budget reaches the audio length).
 //
-// select kernel (one CTA per row; the WnW segment-wise variant takes the
-// row's segments in turn): smoothed scores become order-preserving
+// select kernel (one CTA per row; in the WnW segment-wise variant each warp
+// takes whole segments, so the row's segments are selected in parallel):
+// smoothed scores become order-preserving
 // uint32 keys (-0 folded into +0) in shared memory; an MSB-first 8-bit radix
 // select finds the k-th largest key T and how many keys equal to T are taken;
 // a warp-ballot compaction then writes the kept indices in ascending order:
@@ -19,7 +20,20 @@ namespace {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kMaxSegments = 4096;  // segments of a row in the segment-wise selection
+
+__host__ __device__ __forceinline__ int map_max_len(const RowMap& m) {
+  int x = 0;
+  for (int i = 0; i < m.n_seq; ++i) x = m.L[i] > x ? m.L[i] : x;
+  return x;
+}
+
+// Dynamic shared memory of select_kernel: the keys of the longest row, and for
+// the segment-wise variant the quotas, their prefix and the warps' histograms.
+size_t sel_smem_bytes(const RowMap& m, int nseg) {
+  size_t b = (size_t)map_max_len(m) * sizeof(uint32_t);
+  if (nseg > 0) b += 2 * (size_t)nseg * sizeof(int) + (size_t)kSelWarps * 256 * sizeof(int);
+  return b;
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -105,6 +119,74 @@ __device__ void select_range(const uint32_t* keys, int c0s, int c1s, int k, int3
   }
 }
 
+// The same selection by one warp (a segment of the segment-wise variant):
+// keys[c0, c1) -> out[0, k), 1 <= k <= c1 - c0; hist is the warp's 256 bins.
+__device__ void select_range_warp(const uint32_t* keys, int c0, int c1, int k, int32_t* __restrict__ out,
+                                  int* hist) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, mask = 0;
+  int kk = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) hist[i] = 0;
+    __syncwarp();
+    for (int j = c0 + lane; j < c1; j += 32) {
+      const uint32_t key = keys[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncwarp();
+    // lane l holds bins 255 - 8 l down to 248 - 8 l: lanes in order walk the bins from the top
+    int loc[8], tot = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      loc[t] = hist[255 - 8 * lane - t];
+      tot += loc[t];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - tot;
+    const unsigned here = __ballot_sync(0xffffffffu, excl < kk && kk <= incl);
+    const int src = __ffs(here) - 1;
+    int dg = 0, kk_new = kk;
+    if (lane == src) {
+      int cum = excl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (cum + loc[t] >= kk) {
+          dg = 255 - 8 * lane - t;
+          kk_new = kk - cum;
+          break;
+        }
+        cum += loc[t];
+      }
+    }
+    dg = __shfl_sync(0xffffffffu, dg, src);
+    kk = __shfl_sync(0xffffffffu, kk_new, src);
+    prefix |= (uint32_t)dg << shift;
+    mask |= 255u << shift;
+    __syncwarp();  // every lane has read the bins before the next round clears them
+  }
+  const uint32_t T = prefix;
+  const int take_eq = kk;
+  const unsigned lt = (1u << lane) - 1u;
+  int eq_before = 0, sel_before = 0;
+  for (int base = c0; base < c1; base += 32) {
+    const int j = base + lane;
+    const uint32_t key = j < c1 ? keys[j] : 0u;
+    const bool eq = j < c1 && key == T;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const bool sel = j < c1 && (key > T || (eq && eq_before + __popc(beq & lt) < take_eq));
+    const unsigned bsel = __ballot_sync(0xffffffffu, sel);
+    const int at = sel_before + __popc(bsel & lt);
+    if (sel && at < k) out[at] = j;
+    eq_before += __popc(beq);
+    sel_before += __popc(bsel);
+  }
+}
+
 // One CTA per row. nseg = 0: one top-(b - w) over the candidates [0, L - w);
 // nseg > 0: the candidates cut into nseg segments [floor(i n / nseg),
 // floor((i + 1) n / nseg)), segment i keeping q_i = floor(k len_i / n) plus
@@ -113,14 +195,18 @@ __device__ void select_range(const uint32_t* keys, int c0s, int c1s, int k, int3
 __global__ void __launch_bounds__(kSelThreads, 1)
     select_kernel(const RowMap map, int w, int nseg, const float* __restrict__ s_hat, const int32_t* __restrict__ b,
                   const int64_t* __restrict__ slot_off, int32_t* __restrict__ idx) {
+  // dynamic shared memory: keys [L]; with segments also q_s, at_s [nseg] and
+  // the warps' histograms [kSelWarps][256] (sel_smem_bytes)
   extern __shared__ uint32_t keys[];
   __shared__ int hist[256];
   __shared__ int wgt[kSelWarps], weq[kSelWarps];
   __shared__ uint32_t sh_prefix;
   __shared__ int sh_kk;
-  __shared__ int q_s[kMaxSegments];
 
   const int row = blockIdx.x;
+  int* q_s = reinterpret_cast<int*>(keys + map_max_len(map));
+  int* at_s = q_s + max(nseg, 0);
+  int(*whist)[256] = reinterpret_cast<int(*)[256]>(at_s + max(nseg, 0));
   const int L = row_len(map, row);
   const long long koff = row_key_off(map, row);
   const int bb = b[row];
@@ -136,7 +222,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   for (int i = threadIdx.x; i < w; i += kSelThreads) out[k + i] = n + i;
   if (k <= 0) return;
   for (int j = threadIdx.x; j < n; j += kSelThreads) keys[j] = order_key(s_hat[koff + j]);
-  if (nseg <= 0) {
+  if (nseg <= 1) {  // one top-k over the candidates (a single segment is the same selection)
     select_range(keys, 0, n, k, out, hist, wgt, weq, &sh_prefix, &sh_kk);
     return;
   }
@@ -155,12 +241,43 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     q_s[i] = (int)((long long)k * len / n) + (rank < k - sum_q ? 1 : 0);
   }
   __syncthreads();
-  int at = 0;
-  for (int i = 0; i < nseg; ++i) {
+  // each segment's first output place: the exclusive prefix of the quotas
+  // (each thread sums a run of consecutive segments, then the runs are scanned)
+  {
+    const int per = (nseg + kSelThreads - 1) / kSelThreads;
+    const int i0 = threadIdx.x * per, i1 = min(nseg, i0 + per);
+    int run = 0;
+    for (int i = i0; i < i1; ++i) run += q_s[i];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wgt[warp] = incl;
+    __syncthreads();
+    int before = incl - run;
+    for (int i = 0; i < warp; ++i) before += wgt[i];
+    for (int i = i0; i < i1; ++i) {
+      at_s[i] = before;
+      before += q_s[i];
+    }
+  }
+  __syncthreads();
+  if (nseg < kSelWarps / 4) {  // a few long segments: the whole block on each in turn
+    for (int i = 0; i < nseg; ++i) {
+      const int lo = (int)((long long)i * n / nseg), hi = (int)((long long)(i + 1) * n / nseg);
+      if (q_s[i] > 0) select_range(keys, lo, hi, q_s[i], out + at_s[i], hist, wgt, weq, &sh_prefix, &sh_kk);
+    }
+    return;
+  }
+  // many segments: one warp each, in parallel
+  const int warp = threadIdx.x >> 5;
+  for (int i = warp; i < nseg; i += kSelWarps) {
     const int lo = (int)((long long)i * n / nseg), hi = (int)((long long)(i + 1) * n / nseg);
     const int q = q_s[i];
-    if (q > 0) select_range(keys, lo, hi, q, out + at, hist, wgt, weq, &sh_prefix, &sh_kk);
-    at += q;
+    if (q > 0) select_range_warp(keys, lo, hi, q, out + at_s[i], whist[warp]);
   }
 }
 
@@ -213,15 +330,11 @@ __global__ void __launch_bounds__(256)
 int launch_select_gather(const kv_shape& sh, const RowMap& m, const float* s_hat, const void* K, const void* V,
                          const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc, int nseg,
                          cudaStream_t st) {
-  int maxL = 0;
-  for (int i = 0; i < m.n_seq; ++i) maxL = std::max(maxL, m.L[i]);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr = true;
-  }
-  select_kernel<<<m.n_rows, kSelThreads, (size_t)maxL * sizeof(uint32_t), st>>>(m, sh.w, nseg, s_hat, b, slot_off,
-                                                                                 idx);
+  // a per-device setting: made on every launch (cheap), for whichever device is current
+  const size_t smem = sel_smem_bytes(m, nseg);
+  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return KV_ERR_CUDA;
+  select_kernel<<<m.n_rows, kSelThreads, smem, st>>>(m, sh.w, nseg, s_hat, b, slot_off, idx);
   const int esz = sh.dtype == KV_BF16 ? 2 : 4;
   const int row_bytes = sh.head_dim * esz;
   gather_kernel<<<sm_count() * 8, 256, 0, st>>>(m, row_bytes, slot_off, b, idx, static_cast<const uint8_t*>(K),

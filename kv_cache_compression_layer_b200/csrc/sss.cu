@@ -424,11 +424,11 @@ int launch_sss(const RowMap& m, const float* s, float* s_hat, int32_t* kstar, fl
   cfg.numAttrs = 1;
   cudaError_t e;
   if (C == 1) {
-    cudaFuncSetAttribute(sss_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = cudaLaunchKernelEx(&cfg, sss_kernel<1>, m, s, s_hat, kstar, alpha, rho);
+    e = cudaFuncSetAttribute(sss_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sss_kernel<1>, m, s, s_hat, kstar, alpha, rho);
   } else {
-    cudaFuncSetAttribute(sss_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = cudaLaunchKernelEx(&cfg, sss_kernel<2>, m, s, s_hat, kstar, alpha, rho);
+    e = cudaFuncSetAttribute(sss_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sss_kernel<2>, m, s, s_hat, kstar, alpha, rho);
   }
   return cuda_status(e);
 }

@@ -363,12 +363,10 @@ extern "C" int kv_voxzip_pool(const int32_t* L_a, int32_t n_seq, const double* t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   const size_t plan_bytes = sizeof(SegPlan) * (size_t)std::max(max_seg, 1);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(vz_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)(sizeof(SegPlan) * KV_VZ_MAX_SEGMENTS));
-    attr = true;
-  }
+  // a per-device setting: made on every launch (cheap), for whichever device is current
+  if (cudaFuncSetAttribute(vz_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(sizeof(SegPlan) * KV_VZ_MAX_SEGMENTS)) != cudaSuccess)
+    return KV_ERR_CUDA;
   vz_plan_kernel<<<n_seq, kPlanThreads, plan_bytes, st>>>(m, conf_min, segs, (long long)n_text_rows,
                                                           E_T ? 1 : 0, src, out_len, status);
   const int slices = (d * esz + kSliceBytes - 1) / kSliceBytes;

@@ -421,12 +421,10 @@ int kv_wnw_update(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32
   const int cpc = chunks_per_cta(p->chunk_len, p->chunk_stride);
   int max_M = 0;
   for (int i = 0; i < n_seq; ++i) max_M = std::max(max_M, m.M[i]);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(wnw_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)(sizeof(float) * kStageFloats));
-    attr = true;
-  }
+  // per-device settings: made on every launch (cheap), for whichever device is current
+  if (cudaFuncSetAttribute(wnw_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(sizeof(float) * kStageFloats)) != cudaSuccess)
+    return KV_ERR_CUDA;
   wnw_score_kernel<<<dim3((max_M + cpc - 1) / cpc, n_seq), kScoreThreads, sizeof(float) * kStageFloats, cs>>>(
       m, p->chunk_len, p->chunk_stride, cpc, n_anchor, s, score);
   // stage each sequence's scores and state in shared memory when the largest fits
@@ -435,11 +433,9 @@ int kv_wnw_update(const int32_t* L, int32_t n_seq, const kv_wnw_params* p, int32
     stage_bytes = std::max(stage_bytes, sizeof(double) * m.M[i] + sizeof(int32_t) * (m.M[i] + m.nb[i] + p->n_slots));
   const size_t list_bytes = sizeof(int32_t) * (size_t)((p->n_slots + 1) & ~1);
   const int staged = list_bytes + stage_bytes <= (size_t)kUpdStageMax ? 1 : 0;
-  static bool upd_attr = false;
-  if (!upd_attr) {
-    cudaFuncSetAttribute(wnw_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUpdStageMax);
-    upd_attr = true;
-  }
+  if (cudaFuncSetAttribute(wnw_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUpdStageMax) !=
+      cudaSuccess)
+    return KV_ERR_CUDA;
   wnw_update_kernel<<<n_seq, kUpdThreads, staged ? list_bytes + stage_bytes : list_bytes, cs>>>(
       m, p->chunk_len, p->chunk_stride, p->top_c, p->release_after, p->n_slots, cap, staged, state, score, fetch,
       release, counts);

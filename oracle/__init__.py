@@ -276,6 +276,19 @@ class DecodeList:
                                     gamma, T, M, b, _p(o))
         return o, int(ev)
 
+    def remove(self, pos: int) -> None:
+        """Evicts the entry at position `pos`: the list becomes the Concat of the
+        entries before and after it (the eviction of the VoxZip second stage
+        with the evicted index given, for a tie the caller has resolved)."""
+        n = self.n.value
+        hit = np.flatnonzero(self.pos[:n] == pos)
+        if len(hit) != 1:
+            raise ValueError(f"position {pos} is not in the list")
+        i = int(hit[0])
+        for arr in (self.K, self.V, self.A, self.pos):
+            arr[i:n - 1] = arr[i + 1:n].copy()
+        self.n.value = n - 1
+
     def clone(self) -> "DecodeList":
         c = DecodeList.__new__(DecodeList)
         c.d = self.d

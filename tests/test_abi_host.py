@@ -180,3 +180,14 @@ def test_status_strings(L):
     assert kv.status_string(kv.KV_OK) == "ok"
     assert "budget" in kv.status_string(kv.KV_ERR_BUDGET)
     assert kv.status_string(99) == "unknown status"
+
+
+def test_wait_limit_round_trips(L):
+    # host-side setting only: launches made after the call take the new limit
+    prev = kv.kv_set_wait_limit_ns(12345)
+    try:
+        assert prev == kv.DEFAULT_WAIT_LIMIT_NS
+        assert kv.kv_set_wait_limit_ns(0) == 12345
+    finally:
+        kv.kv_set_wait_limit_ns(prev)
+    assert kv.kv_set_wait_limit_ns(prev) == prev

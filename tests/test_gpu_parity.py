@@ -13,7 +13,8 @@ import torch
 import kv_cache_compression_layer_b200 as kv
 import oracle as orc
 import synth
-from tests._harness import (dev, kth_exempt_mask, params_of, score_close, shape_of, tdtype, up, valid_kstars)
+from tests._harness import (KSTAR_BAND_SAME_INPUT, dev, f32, kth_exempt_mask, params_of, score_close, shape_of,
+                            tdtype, up, valid_kstars)
 
 pytestmark = pytest.mark.gpu
 
@@ -83,9 +84,10 @@ def _check_sss(L_list, s_rows, alpha, rho):
     off = np.concatenate([[0], np.cumsum(L_list)])
     for i, L in enumerate(L_list):
         srow = s32[i].astype(np.float64)
-        valid = valid_kstars(srow, rho, orc)
+        # the kernel received alpha and rho as float32: the oracle computes with those values
+        valid = valid_kstars(srow, f32(rho), orc, KSTAR_BAND_SAME_INPUT)
         assert int(g_ks[i]) in valid, (L, int(g_ks[i]), valid[:5])
-        o_hat, _ = orc.sss(srow, [L], alpha, rho, kstar_force=[int(g_ks[i])])
+        o_hat, _ = orc.sss(srow, [L], f32(alpha), f32(rho), kstar_force=[int(g_ks[i])])
         ok, worst = score_close(g_hat[off[i]:off[i + 1]], o_hat, [L])
         assert ok, (L, worst)
 

@@ -1,111 +1,44 @@
 """End-to-end parity: the whole path through the C ABI (``Compressor``, the
 same calls the benchmark times) against the oracle's chain on the same seeded
-inputs. Small workloads are checked on every row; the full 3B-class workload
-(36 layers x 2 KV heads, L = 6000, the benchmark's default) on sampled rows.
+inputs. Small workloads are checked on every row (compression, then decode in
+lock step); the full 3B-class workload (36 layers x 2 KV heads, L = 6000) on
+sampled rows. The other full-size workloads are in test_gpu_full_size.py.
 """
 import numpy as np
 import pytest
-import torch
 
-import kv_cache_compression_layer_b200 as kv
-import oracle as orc
 import synth
-from kv_cache_compression_layer_b200 import Compressor
-from tests._harness import (dev, kth_exempt_mask, params_of, score_close, shape_of, tdtype, up, valid_kstars)
+from tests._pipeline import check_compress_rows, compress, decode_lockstep
 
 pytestmark = pytest.mark.gpu
-
-
-def _run_gpu(cfg, bt, steps):
-    dt = tdtype(cfg)
-    comp = Compressor(shape_of(cfg), cfg.L, params_of(cfg))
-    spikes = None
-    if bt.spikes is not None:
-        spikes = up(np.where(bt.spikes, 10.0, 1.0).astype(np.float32), torch.float32)
-    K, V = up(bt.K, dt), up(bt.V, dt)
-    comp.compress(up(bt.qwin, dt), K, V, up(bt.S, torch.float32), spikes=spikes)
-    comp.kept_after_compress = comp.kept()  # decode steps recycle slots afterwards
-    outs = []
-    out = torch.empty(cfg.rows, cfg.group, cfg.head_dim, dtype=dt, device=dev())
-    for t in range(steps):
-        comp.decode_step(up(bt.q_dec[t], dt), up(bt.k_dec[t], dt), up(bt.v_dec[t], dt), out)
-        outs.append(out.float().cpu().numpy())
-    torch.cuda.synchronize()
-    assert kv.kv_read_device_status(comp.status) == 0
-    assert kv.kv_read_device_status(comp.ws[:4].view(torch.int32)) == 0
-    return comp, outs
-
-
-def _check_rows(cfg, bt, comp, outs, rows, steps):
-    s_gpu = comp.s.cpu().numpy()
-    h_gpu = comp.s_hat.cpu().numpy()
-    ks_gpu = comp.kstar.cpu().numpy()
-    b_gpu = comp.b.cpu().numpy()
-    kept = comp.kept_after_compress
-    b_orc = orc.allocate(bt.S, cfg.L, cfg.w, cfg.budget_pct, cfg.r).reshape(-1)
-    np.testing.assert_array_equal(b_gpu, b_orc)
-    koff = bt.key_off
-    same_sel = 0
-    for r in rows:
-        L = int(bt.L_rows[r])
-        sl = slice(koff[r], koff[r + 1])
-        s_orc = orc.score(bt.qwin[r:r + 1], bt.K[sl], [L])
-        if bt.spikes is not None:  # the harness multiplies spike positions by 10 before smoothing
-            s_orc = s_orc * np.where(bt.spikes[sl], 10.0, 1.0)
-        ok, worst = score_close(s_gpu[sl], s_orc, [L])
-        assert ok, ("score", r, worst)
-        valid = valid_kstars(s_orc, cfg.rho, orc)
-        assert int(ks_gpu[r]) in valid, ("kstar", r, int(ks_gpu[r]), valid[:4])
-        h_orc, _ = orc.sss(s_orc, [L], cfg.alpha, cfg.rho, kstar_force=[int(ks_gpu[r])])
-        ok, worst = score_close(h_gpu[sl], h_orc, [L], floor="rms")
-        assert ok, ("s_hat", r, worst)
-        idx_orc = orc.select(h_orc, [L], cfg.w, [int(b_orc[r])])[0]
-        b_r, idx_gpu, Kc, Vc = kept[r]
-        assert len(idx_gpu) == b_r == len(idx_orc)
-        assert (np.diff(idx_gpu) > 0).all() and set(range(L - cfg.w, L)) <= set(idx_gpu.tolist())
-        diff = np.setxor1d(idx_gpu, idx_orc)
-        if len(diff):
-            exempt = np.flatnonzero(kth_exempt_mask(h_orc, L, cfg.w, int(b_orc[r])))
-            assert set(diff.tolist()) <= set(exempt.tolist()), ("select", r, diff[:8])
-        else:
-            same_sel += 1
-        np.testing.assert_array_equal(Kc, bt.K[koff[r] + idx_gpu])
-        np.testing.assert_array_equal(Vc, bt.V[koff[r] + idx_gpu])
-        if len(diff) == 0 and steps:
-            lst = orc.DecodeList(bt.K[koff[r] + idx_orc], bt.V[koff[r] + idx_orc], idx_orc)
-            M = orc.recent_count(int(b_orc[r]), cfg.recent_pct)
-            for t in range(steps):
-                o, ev = lst.step(bt.q_dec[t, r], bt.k_dec[t, r], bt.v_dec[t, r], L + t, cfg.gamma, cfg.sinks_T, M,
-                                 int(b_orc[r]))
-                tol = 2e-2 if cfg.dtype == "bf16" else 1e-4 * np.abs(o).max()
-                assert np.abs(outs[t][r] - o).max() <= tol, ("decode", r, t)
-    return same_sel
-
 
 SMALL = [
     (synth.CONFIGS["tiny"], 8),
     (synth.small("3b", n_layers=2, L=(2000,)), 6),
-    (synth.small("ragged", n_layers=2, L=(1000, 3500)), 4),  # spikes, g = 7
-    (synth.small("30b", n_layers=2, L=(4000,)), 4),
-    (synth.small("long", n_layers=1, L=(8000,)), 4),  # 5% budget
+    (synth.small("ragged", n_layers=2, L=(1000, 3500)), 6),  # spikes, g = 7
+    (synth.small("30b", n_layers=2, L=(4000,)), 6),
+    (synth.small("long", n_layers=1, L=(8000,)), 6),  # 5% budget
 ]
 
 
 @pytest.mark.parametrize("cfg,steps", SMALL, ids=lambda c: getattr(c, "name", str(c)))
 def test_pipeline_small_all_rows(cfg, steps):
     bt = synth.make_batch(cfg, steps=steps)
-    comp, outs = _run_gpu(cfg, bt, steps)
-    same = _check_rows(cfg, bt, comp, outs, range(cfg.rows), steps)
-    assert same >= cfg.rows // 2
+    comp, _, _ = compress(cfg, bt)
+    kept, same = check_compress_rows(cfg, bt, comp, range(cfg.rows))
+    assert len(same) >= cfg.rows // 2
+    ls = decode_lockstep(cfg, bt, comp, kept, steps)
+    assert ls.ties <= max(1, cfg.rows // 4)
 
 
 def test_pipeline_3b_full_size_sampled_rows():
     cfg = synth.CONFIGS["3b"]
-    steps = 4
+    steps = 32
     bt = synth.make_batch(cfg, steps=steps)
-    comp, outs = _run_gpu(cfg, bt, steps)
-    _check_rows(cfg, bt, comp, outs, [0, 37, 71], steps)
-    # invariants on every row
+    comp, _, _ = compress(cfg, bt)
+    kept, _ = check_compress_rows(cfg, bt, comp, [0, 37, 71])
+    # invariant on every row: each window row's softmax sums to 1
     s = comp.s.cpu().numpy().astype(np.float64)
-    sums = np.add.reduceat(s, bt.key_off[:-1])
-    np.testing.assert_allclose(sums, cfg.R, rtol=1e-4)
+    np.testing.assert_allclose(np.add.reduceat(s, bt.key_off[:-1]), cfg.R, rtol=1e-4)
+    ls = decode_lockstep(cfg, bt, comp, kept, steps)
+    assert ls.checked == 3 * steps

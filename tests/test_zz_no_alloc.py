@@ -6,15 +6,17 @@ buffers, cannot obtain a workspace. For them the library keeps its scoring
 scratch in one fixed device array of its own. These checks call that entry
 point through the C ABI twice in a row (on two different batches, so the
 array's leftover contents from the first call are in place for the second)
-and compare each result with kv_score given a caller-owned workspace, under
-the score tolerance the other tests use. A batch whose scratch does not fit
-the array must be refused before anything is launched.
+and compare each result with the oracle's scores and with kv_score given a
+caller-owned workspace, under the score tolerance the other tests use; the
+array's status word must read clean after each call. A batch whose scratch
+does not fit the array must be refused before anything is launched.
 """
 import numpy as np
 import pytest
 import torch
 
 import kv_cache_compression_layer_b200 as kv
+import oracle as orc
 import synth
 from tests._harness import dev, score_close, shape_of, tdtype, up
 
@@ -35,7 +37,7 @@ def _with_workspace(cfg, q, K, n):
     return s
 
 
-def test_noalloc_matches_kv_score_on_two_calls_in_a_row():
+def test_noalloc_matches_oracle_and_kv_score_on_two_calls_in_a_row():
     cases = [synth.small("3b", n_layers=2), synth.small("ragged", n_layers=1, L=(2000, 3500))]
     for cfg in cases:
         sh = shape_of(cfg)
@@ -45,15 +47,17 @@ def test_noalloc_matches_kv_score_on_two_calls_in_a_row():
         bt, q, K = _inputs(cfg)
         s = torch.full((len(bt.K),), float("nan"), dtype=torch.float32, device=dev())
         kv.kv_score_noalloc(shape_of(cfg), cfg.L, q, K, s)
+        assert kv.kv_score_noalloc_status() == 0  # this call's status word (synchronises)
         got.append((cfg, bt, q, K, s))
-    torch.cuda.synchronize()
     for cfg, bt, q, K, s in got:
         ref = _with_workspace(cfg, q, K, len(bt.K))
         torch.cuda.synchronize()
-        s_h, ref_h = s.cpu().numpy(), ref.cpu().numpy().astype(np.float64)
+        s_h = s.cpu().numpy()
         assert np.isfinite(s_h).all()
-        ok, worst = score_close(s_h, ref_h, bt.L_rows)
-        assert ok, worst
+        ok, worst = score_close(s_h, orc.score(bt.qwin, bt.K, bt.L_rows), bt.L_rows)
+        assert ok, ("oracle", worst)
+        ok, worst = score_close(s_h, ref.cpu().numpy().astype(np.float64), bt.L_rows)
+        assert ok, ("kv_score", worst)
 
 
 def test_noalloc_refuses_batch_beyond_its_scratch():
