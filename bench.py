@@ -41,9 +41,14 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one decode kernel launch from an ncu capture of
 # this benchmark's workload (its summary is kept under profiles/), valid while
 # the kernel source is the one captured (its SHA-256 below); otherwise null.
-NCU_TRAFFIC = {"3b": {"bytes": 139348224,
+NCU_TRAFFIC = {"3b": {"bytes": 139746048,  # profiles/decode_cl_kernel_3b.md
                       "source": "kv_cache_compression_layer_b200/csrc/decode_cl.cu",
-                      "sha256": "78b5b0da77529123"}}
+                      "sha256": "45d44be40b24b73b"},
+               # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (257,690,624 B for
+               # 483,224 slots) scaled by the slots of the full batch (x 4)
+               "ragged": {"bytes": 1030762496,
+                          "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
+                          "sha256": "c079ebe6e00045ad"}}
 
 
 def decode_kernel(cfg: synth.Config, sms: int) -> str:
@@ -68,6 +73,15 @@ def measured_traffic(cfg_name: str):
     except OSError:
         return None
     return rec["bytes"] if rec["bytes"] and digest.startswith(rec["sha256"]) else None
+
+
+def workload(args) -> synth.Config:
+    """The named workload, or (--layers N) the same with N layers per sequence,
+    a reduced case for profiler captures."""
+    cfg = synth.CONFIGS[args.config]
+    if args.layers:
+        cfg = cfg.with_(n_layers=args.layers)
+    return cfg
 
 
 def describe(cfg: synth.Config) -> str:
@@ -217,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     init_group("nccl", world, dev)
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
     cfg = cfg.with_(seed=replica_seed(cfg.seed, rank))
     bt = synth.make_batch(cfg)
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
@@ -337,7 +351,7 @@ def run_ours(args, rank, world, local_rank):
                    "decode_bytes_alg": dec_bytes, "decode_steps": D},
         "roofline": {"kernel": decode_kernel(cfg, torch.cuda.get_device_properties(dev).multi_processor_count)
                      + " (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": measured_traffic(args.config) if tc else None,
+                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": measured_traffic(args.config) if tc and not args.layers else None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},
         "e2e": {"value": job_throughput(tokens, world, e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
@@ -661,7 +675,7 @@ def run_reference(args, rank, world):
     import oracle as orc
 
     orc.build()
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
     rows = sample_rows(cfg, args.ref_rows)
     bt = synth.make_batch(cfg)
     threads = orc.default_threads()
@@ -690,6 +704,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="ragged", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layers per sequence (default: the workload's); a reduced case for profiler captures")
     ap.add_argument("--cpu-rows", type=int, default=64,
                     help="rows of the oracle sample for cpu_baseline, spread over the batch")
     ap.add_argument("--ref-rows", type=int, default=64,

@@ -12,8 +12,11 @@
 //
 // Attention phase. Twelve warps form three groups of four. The CTA's items
 // are cut into three contiguous runs, one per group, walked as 64-slot tiles
-// (a row change then costs one group, not all three, a combine). Each group
-// feeds itself: its first thread streams its
+// (a row change then costs one group, not all three, a combine); a group
+// claims its run's items one at a time from the front, and a group that has
+// run out takes the back half of the largest unclaimed run of another group
+// (a shared (front, back) word per group, changed by compare-and-swap), so
+// the groups of a CTA end together. Each group feeds itself: its first thread streams its
 // tiles (K and V as 128-byte swizzled TMA boxes, the row's g query rows as a
 // bulk copy, a header with the row's step state) into the group's two
 // stages, and refills a stage as soon as the group has finished with it.
@@ -63,8 +66,9 @@ struct TcScratch {
 
 // The cost of a row beyond its slots when cutting the CTAs' runs, in slots: a
 // row change makes a group combine its four warps' softmax state and write a
-// partial, during which its stages wait.
-constexpr int kRowCost = 256;
+// partial, during which its stages wait, and adds a row's statistics and
+// output to the CTA's finish (measured together: about what 150 slots take).
+constexpr int kRowCost = 150;
 constexpr int kMaxCtas = 1024;
 
 struct TcArgs {
@@ -281,11 +285,73 @@ __device__ __forceinline__ bool walk_first(Walk& w, const DecArgs& a, const TcSc
   return true;
 }
 
-// Moves to the next tile of the CTA; false past the last one.
-__device__ __forceinline__ bool walk_advance(Walk& w, const DecArgs& a, int max_per_row) {
+// A group's unclaimed items [front, back) in one 64-bit word: the group
+// claims from the front, other groups steal from the back.
+__device__ __forceinline__ unsigned long long pack_range(int f, int b) {
+  return (unsigned long long)(unsigned)f | ((unsigned long long)(unsigned)b << 32);
+}
+__device__ __forceinline__ int range_front(unsigned long long c) { return (int)(unsigned)(c & 0xffffffffull); }
+__device__ __forceinline__ int range_back(unsigned long long c) { return (int)(unsigned)(c >> 32); }
+
+// Claims item u, the front of the group's range, unless it has been stolen.
+__device__ __forceinline__ bool claim_item(unsigned long long* own, int u) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(own);
+  for (;;) {
+    if (range_front(cur) != u || u >= range_back(cur)) return false;
+    const unsigned long long prev = atomicCAS(own, cur, pack_range(u + 1, range_back(cur)));
+    if (prev == cur) return true;
+    cur = prev;
+  }
+}
+
+// Takes the back half of the largest unclaimed range of another group (at
+// least two items left there); false when no group has that much left.
+__device__ __forceinline__ bool steal_range(unsigned long long* owns, int grp, int& s0, int& s1) {
+  for (;;) {
+    int v = -1, best = 1;
+    unsigned long long cv = 0;
+    for (int g = 0; g < kGroups; ++g) {
+      if (g == grp) continue;
+      const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(owns + g);
+      const int rem = range_back(c) - range_front(c);
+      if (rem > best) {
+        best = rem;
+        v = g;
+        cv = c;
+      }
+    }
+    if (v < 0) return false;
+    const int f = range_front(cv), b = range_back(cv), k = (b - f) / 2;
+    if (atomicCAS(owns + v, cv, pack_range(f, b - k)) == cv) {
+      s0 = b - k;
+      s1 = b;
+      return true;
+    }
+  }
+}
+
+// Positions the walk on the next item the group may take: the front of its
+// own range, else the first of a range stolen from another group (which
+// becomes its own). False when the CTA has no unclaimed item worth taking.
+__device__ __noinline__ bool group_take(Walk& w, const DecArgs& a, const TcScratch& sc, unsigned long long* owns,
+                                        int grp) {
+  for (;;) {
+    const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(owns + grp);
+    const int f = range_front(c);
+    if (claim_item(owns + grp, f)) return walk_first(w, a, sc, f, range_back(c));
+    int s0, s1;
+    if (!steal_range(owns, grp, s0, s1)) return false;
+    atomicExch(owns + grp, pack_range(s0, s1));
+  }
+}
+
+// Moves to the next tile of the group's claimed items; false when the next
+// item cannot be claimed (the range is used up or its rest was stolen).
+__device__ __forceinline__ bool walk_advance(Walk& w, const DecArgs& a, int max_per_row, unsigned long long* own) {
   ++w.it;
   if (++w.t < w.nt) return true;
-  if (++w.u >= w.u1) return false;
+  if (!claim_item(own, w.u + 1)) return false;
+  ++w.u;
   if (++w.chunk >= w.nchunk) {  // the next row
     w.chunk = 0;
     w.base += w.cap;
@@ -511,6 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __shared__ int dq_row[kGroups][kDefer], dq_cnt[kGroups][kDefer], dq_n[kGroups];
   __shared__ Walk walk_s[kGroups];  // each group's tile walk (its first thread's), kept out of registers
   __shared__ int more_s[kGroups], ended_s[kGroups], nreal_s[kGroups];
+  __shared__ unsigned long long owns_s[kGroups];  // each group's unclaimed items (front, back)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
@@ -537,23 +604,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     u0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
     u1 = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
   }
+  if (tid == 0)  // each group starts with a contiguous third of the CTA's items
+    for (int g = 0; g < kGroups; ++g)
+      owns_s[g] = pack_range(u0 + (int)((long long)(u1 - u0) * g / kGroups),
+                             u0 + (int)((long long)(u1 - u0) * (g + 1) / kGroups));
+  __syncthreads();
 
   // ---------------------------------------------------------------- attention
   {
     Walk& w = walk_s[grp];
     if (gt == 0) {
       const uint64_t stream_policy = make_policy_evict_first();  // K and V are read once per step
-      // this group's contiguous share of the CTA's items
-      const int gu0 = u0 + (int)((long long)(u1 - u0) * grp / kGroups);
-      const int gu1 = u0 + (int)((long long)(u1 - u0) * (grp + 1) / kGroups);
-      int more = walk_first(w, a, sc, gu0, gu1);
+      int more = group_take(w, a, sc, owns_s, grp);
       int ended = 0, n_real = 0;
       for (int s = 0; s < kGStages && !ended; ++s) {
         const int stg = grp * kGStages + s;
         if (more) {
           issue_tile<D>(w, ring + stg * STAGE, &full[stg], &hdr[stg], &tmK, &tmV, &tmQ, a, stream_policy);
           ++n_real;
-          more = walk_advance(w, a, sc.max_per_row);
+          more = walk_advance(w, a, sc.max_per_row, owns_s + grp) || group_take(w, a, sc, owns_s, grp);
         } else {
           hdr[stg].row = -1;
           mbar_arrive(&full[stg]);
@@ -620,14 +689,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
           // the group's warps add their O in warp order (a fixed summation order,
           // so a step's result does not depend on scheduling); lanes own distinct columns
-#pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
             if ((warp & 3) == w4 && g_ok) {
+              float* ogp = og + g0 * D;
+              asm volatile("" : "+l"(ogp));  // addresses formed here, not held across the turns
 #pragma unroll
               for (int i = 0; i < 2 * NDC; ++i) {
                 const int col = i * 8 + q4 * 2;
-                og[g0 * D + ogswz(g0, col)] += o[i][0] * f0;
-                og[g0 * D + ogswz(g0, col + 1)] += o[i][1] * f0;
+                ogp[ogswz(g0, col)] += o[i][0] * f0;
+                ogp[ogswz(g0, col + 1)] += o[i][1] * f0;
               }
             }
             named_bar_sync(1 + grp, 128);
@@ -786,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (more_s[grp]) {
           issue_tile<D>(w, stage, &full[stg], &hdr[stg], &tmK, &tmV, &tmQ, a, make_policy_evict_first());
           ++nreal_s[grp];
-          more_s[grp] = walk_advance(w, a, sc.max_per_row);
+          more_s[grp] = walk_advance(w, a, sc.max_per_row, owns_s + grp) || group_take(w, a, sc, owns_s, grp);
         } else if (!ended_s[grp]) {
           hdr[stg].row = -1;
           mbar_arrive(&full[stg]);
@@ -818,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const int nq = (E + kOutUnit - 1) / kOutUnit;
   const int r_lo = rlo_s, r_hi = rhi_s, own_lo = own_s;
   const long long S0 = rng_s[0], S1 = rng_s[1];
-  constexpr int UP = 8;  // slot pairs per lane in flight in the sweep
+  constexpr int UP = 12;  // slot pairs per lane in flight in the sweep
   // The first batch's slot data (logits written by this CTA, A, positions: none of it
   // waits for another CTA) is copied into the rest of the freed ring now, without
   // waiting; the sweep reads it from there.
