@@ -385,31 +385,76 @@ __global__ void __launch_bounds__(kScanThreads) c3_frontier_kernel(const RowMap 
 
 // ------------------------------------------------------------------- step --
 // sigma of every frontier node: max over the query heads of the cosine
-// (float64; products and sums rounded separately, dimensions in order).
+// (float64; products and sums rounded separately, every sum in dimension
+// order from 0, as the oracle does). A lane takes a node; its warp copies
+// the 32 nodes' centroids into shared memory 32 dimensions at a time with
+// coalesced loads (padded so the lanes' reads spread over the banks), and the
+// block copies the row's query rows as doubles. Sum c_k^2 does not depend on
+// the head and is taken once; the heads' dot products are independent
+// chains (up to kC3Heads at a time).
+constexpr int kC3ScoreWarps = 4;
+constexpr int kC3Heads = 8;
+constexpr int kC3QStage = 16;  // query heads staged in shared memory (more: read from global memory)
+
 template <typename T>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(32 * kC3ScoreWarps)
     c3_score_kernel(const RowMap m, C3Arr a, const T* __restrict__ q, int G, int d, int B) {
+  extern __shared__ double c3s[];  // [warps][32][33] centroid chunks, then [G][d] query rows if G <= kC3QStage
   const int row = blockIdx.y;
   if (row_len(m, row) <= B) return;
   const long long no = 2 * row_key_off(m, row);
   const int A = a.hdr()[(long long)row * kHdr + 1];
-  const int i = blockIdx.x * 128 + threadIdx.x;
-  if (i >= A) return;
-  const double* c = a.cent() + (no + a.front()[no + i]) * d;
+  const int i0 = blockIdx.x * 32 * kC3ScoreWarps;
+  if (i0 >= A) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double* cs = c3s + (size_t)warp * 32 * 33;
+  double* qs = c3s + (size_t)kC3ScoreWarps * 32 * 33;
   const T* qr = q + (long long)row * G * d;
-  double best = -INFINITY;
-  for (int g = 0; g < G; ++g) {
-    double ab = 0.0, aa = 0.0, bb = 0.0;
-    for (int k = 0; k < d; ++k) {
-      const double x = ld(qr + (long long)g * d + k), y = c[k];
-      ab = __dadd_rn(ab, __dmul_rn(x, y));
-      aa = __dadd_rn(aa, __dmul_rn(x, x));
-      bb = __dadd_rn(bb, __dmul_rn(y, y));
+  const bool q_staged = G <= kC3QStage;
+  if (q_staged)
+    for (int k = threadIdx.x; k < G * d; k += 32 * kC3ScoreWarps) qs[k] = ld(qr + k);
+  __syncthreads();
+  const int wi0 = i0 + warp * 32;
+  if (wi0 >= A) return;
+  const int i = wi0 + lane;
+  const int nw = min(32, A - wi0);  // nodes of this warp
+  const int my_node = i < A ? a.front()[no + i] : 0;
+  double bb = 0.0, best = -INFINITY;
+  for (int g0 = 0; g0 < G; g0 += kC3Heads) {
+    double ab[kC3Heads], aa[kC3Heads];
+#pragma unroll
+    for (int t = 0; t < kC3Heads; ++t) ab[t] = aa[t] = 0.0;
+    for (int k0 = 0; k0 < d; k0 += 32) {
+      __syncwarp();
+      for (int n = 0; n < nw; ++n) {  // node n's dimensions k0 .. k0 + 31, one per lane
+        const int node = __shfl_sync(0xffffffffu, my_node, n);
+        cs[n * 33 + lane] = a.cent()[(no + node) * d + k0 + lane];
+      }
+      __syncwarp();
+      if (i < A) {
+        for (int kk = 0; kk < 32; ++kk) {
+          const int k = k0 + kk;
+          const double yk = cs[lane * 33 + kk];
+          if (g0 == 0) bb = __dadd_rn(bb, __dmul_rn(yk, yk));
+#pragma unroll
+          for (int t = 0; t < kC3Heads; ++t)
+            if (g0 + t < G) {
+              const double x = q_staged ? qs[(g0 + t) * d + k] : ld(qr + (long long)(g0 + t) * d + k);
+              ab[t] = __dadd_rn(ab[t], __dmul_rn(x, yk));
+              aa[t] = __dadd_rn(aa[t], __dmul_rn(x, x));
+            }
+        }
+      }
     }
-    const double cs = (aa == 0.0 || bb == 0.0) ? 0.0 : __ddiv_rn(ab, __dmul_rn(__dsqrt_rn(aa), __dsqrt_rn(bb)));
-    if (cs > best) best = cs;
+#pragma unroll
+    for (int t = 0; t < kC3Heads; ++t)
+      if (g0 + t < G) {
+        const double c =
+            (aa[t] == 0.0 || bb == 0.0) ? 0.0 : __ddiv_rn(ab[t], __dmul_rn(__dsqrt_rn(aa[t]), __dsqrt_rn(bb)));
+        if (c > best) best = c;
+      }
   }
-  a.sigma()[no + i] = best;
+  if (i < A) a.sigma()[no + i] = best;
 }
 
 // Order key of a frontier entry: larger sigma first, then the lower node id.
@@ -875,11 +920,16 @@ int kv_c3_step(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int d = shape->head_dim, G = shape->group, B = p->budget;
   const int Lmax = max_len(m);
-  const dim3 sgrid((2 * Lmax + 127) / 128, m.n_rows);
+  const int per_blk = 32 * kC3ScoreWarps;
+  const dim3 sgrid((2 * Lmax + per_blk - 1) / per_blk, m.n_rows);
+  const size_t score_smem = ((G <= kC3QStage ? (size_t)G * d : 0) + (size_t)kC3ScoreWarps * 32 * 33) * sizeof(double);
   const size_t attn_smem = 2 * (size_t)B * sizeof(float);  // logits and retrieved positions
   if (shape->dtype == KV_BF16) {
     using T = __nv_bfloat16;
-    c3_score_kernel<T><<<sgrid, 128, 0, cs>>>(m, a, static_cast<const T*>(q), G, d, B);
+    if (cudaFuncSetAttribute(c3_score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)score_smem) !=
+        cudaSuccess)
+      return KV_ERR_CUDA;
+    c3_score_kernel<T><<<sgrid, 32 * kC3ScoreWarps, score_smem, cs>>>(m, a, static_cast<const T*>(q), G, d, B);
     c3_select_kernel<<<m.n_rows, kScanThreads, 0, cs>>>(m, a, B);
     if (cudaFuncSetAttribute(c3_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem) !=
         cudaSuccess)
@@ -889,7 +939,10 @@ int kv_c3_step(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_
         d, B);
   } else {
     using T = float;
-    c3_score_kernel<T><<<sgrid, 128, 0, cs>>>(m, a, static_cast<const T*>(q), G, d, B);
+    if (cudaFuncSetAttribute(c3_score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)score_smem) !=
+        cudaSuccess)
+      return KV_ERR_CUDA;
+    c3_score_kernel<T><<<sgrid, 32 * kC3ScoreWarps, score_smem, cs>>>(m, a, static_cast<const T*>(q), G, d, B);
     c3_select_kernel<<<m.n_rows, kScanThreads, 0, cs>>>(m, a, B);
     if (cudaFuncSetAttribute(c3_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem) !=
         cudaSuccess)

@@ -161,12 +161,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long key0 = row_key_off(a.map, row) + (long long)tile * kTileKeys;
         for (int c = 0; c < a.nk; ++c)
           tma_load_2d(sK + st * kKStageBytes + c * kKChunkBytes, &tmK, &full_k[st], c * 64, (int)key0);
-        k_issued[st] = true;
-        k_parity[st] = (it / kStages) & 1;
+#pragma unroll
+        for (int z = 0; z < kStages; ++z)  // constant indices: the arrays stay in registers
+          if (z == st) {
+            k_issued[z] = true;
+            k_parity[z] = (it / kStages) & 1;
+          }
       }
       // let every copy issued land before the CTA's shared memory goes away (after
       // a normal run they all have; after an abort raised anywhere some may not)
       (void)aborted;
+#pragma unroll
       for (int st = 0; st < kStages; ++st)
         if (k_issued[st]) wait_drain(&full_k[st], k_parity[st]);
       if (have_q) wait_drain(q_full, q_parity);
@@ -255,21 +260,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // chunk by chunk (chunks of keys at or beyond nvalid are skipped)
         const uint32_t hb = tbase + half * 128;
         const int r = half * 128 + quarter * 32 + lane;
-        float m = -INFINITY, Z = 0.f;
-        auto rowstats = [&](const float (&x)[32], int ch) {
-          if (ch * 32 >= nvalid) return;
-          float mx = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i < nvalid) mx = fmaxf(mx, x[i]);
+        // four partial sums (independent add chains), combined in a fixed order
+        float m = -INFINITY, Z4[4] = {0.f, 0.f, 0.f, 0.f};
+        auto rescale = [&](float mx) {
           if (mx > m) {
-            Z = m == -INFINITY ? 0.f : Z * ex2_approx((m - mx) * a.c);
+            const float f = m == -INFINITY ? 0.f : ex2_approx((m - mx) * a.c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) Z4[q] *= f;
             m = mx;
           }
-          const float mc = m * a.c;
+        };
+        auto rowstats = [&](const float (&x)[32], int ch) {
+          if (ch * 32 + 32 <= nvalid) {  // a full chunk (every tile but a row's last): no masks
+            float mx = fmaxf(x[0], x[1]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i < nvalid) Z += ex2_approx(fmaf(x[i], a.c, -mc));
+            for (int i = 2; i < 32; ++i) mx = fmaxf(mx, x[i]);
+            rescale(mx);
+            const float mc = m * a.c;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) Z4[i & 3] += ex2_approx(fmaf(x[i], a.c, -mc));
+          } else if (ch * 32 < nvalid) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (ch * 32 + i < nvalid) mx = fmaxf(mx, x[i]);
+            rescale(mx);
+            const float mc = m * a.c;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (ch * 32 + i < nvalid) Z4[i & 3] += ex2_approx(fmaf(x[i], a.c, -mc));
+          }
         };
         tmem_ld32(hb, xa);
         tc_wait_ld_regs(xa);
@@ -284,23 +304,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_wait_ld_regs(xb);
         release();
         rowstats(xb, 3);
+        const float Z = (Z4[0] + Z4[1]) + (Z4[2] + Z4[3]);
         if (r < a.R) a.partial[(long long)u * a.R + r] = make_float2(m, Z);
       } else {
         // this thread's key: the sum over its half of the window rows of
         // exp2(x c - lse_r), chunk by chunk
         const int j = quarter * 32 + lane;
         const float* lse = a.lse2 + (long long)row * a.Rs;
-        float sum = 0.f;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};  // independent add chains, combined in a fixed order
         auto colsum = [&](const float (&x)[32], int ch) {
           const int col = ch * 32;
+          if (col + 32 <= a.R) {  // a full chunk of window rows: no masks
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            if (col + i < a.R) {
+            for (int i = 0; i < 32; i += 4) {
               const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse + col + i));
-              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+              sum4[0] += ex2_approx(fmaf(x[i + 0], a.c, -l4.x));
+              sum4[1] += ex2_approx(fmaf(x[i + 1], a.c, -l4.y));
+              sum4[2] += ex2_approx(fmaf(x[i + 2], a.c, -l4.z));
+              sum4[3] += ex2_approx(fmaf(x[i + 3], a.c, -l4.w));
+            }
+          } else {
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                if (col + i + q < a.R) sum += ex2_approx(fmaf(x[i + q], a.c, -lv[q]));
+            for (int i = 0; i < 32; i += 4) {
+              if (col + i < a.R) {
+                const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse + col + i));
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (col + i + q < a.R) sum4[q] += ex2_approx(fmaf(x[i + q], a.c, -lv[q]));
+              }
             }
           }
         };
@@ -319,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (has2) tc_wait_ld_regs(xa);
           }
         }
+        float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         float* pb = part + (bf * 2 + ((it >> 1) & 1)) * kTileKeys;
         if (pair && half == 0) {  // hand the first half's sums to the second
           pb[j] = sum;

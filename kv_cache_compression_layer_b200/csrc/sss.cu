@@ -170,7 +170,9 @@ __device__ __forceinline__ void small_dft<7>(double2 (&v)[7], bool inv) {
 template <int RAD, int C>
 __device__ __noinline__ void fft_stage(const Buf& buf, int N, int Ns, int L, bool inv, const Twiddles& tw,
                                        int rank, cg::cluster_group& cl) {
-  constexpr int MAXB = (kMaxPerThread + RAD - 1) / RAD + 1;
+  // a CTA holds at most kMaxLocal points: nb / C <= kMaxLocal / RAD butterflies, at
+  // most ceil(kMaxPerThread / RAD) per thread (every one held across the barrier)
+  constexpr int MAXB = (kMaxPerThread + RAD - 1) / RAD;
   const int nb = N / RAD;
   const int jb0 = (int)((long long)nb * rank / C), jb1 = (int)((long long)nb * (rank + 1) / C);
   double2 v[MAXB][RAD];
