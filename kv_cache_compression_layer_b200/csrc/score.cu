@@ -53,7 +53,6 @@ struct TcArgs {
   RowMap map;
   int R;      // valid window rows
   int n2;     // pass-2 MMA N: R rounded up to 16
-  int nk;     // 64-element chunks of d (1 or 2)
   int total_tiles;
   float c;    // log2(e) / sqrt(d)
   int Rs;     // row stride of lse2: R rounded up to 4 (16-byte rows)
@@ -62,6 +61,35 @@ struct TcArgs {
   float* s;            // pass 2 out: [sum L]
   int* status;
   unsigned long long limit_ns;
+};
+
+// Walks a CTA's contiguous run of scoring tiles in order: the row, the tile
+// in the row, its valid keys and the row's first key, advanced without a
+// search (the sequences' rows and keys are laid out one after another).
+struct TileIter {
+  int row, tile, tpr, L;
+  long long key0;  // first key of the row
+  __device__ __forceinline__ void init(const RowMap& m, int u) {
+    int s = 0;
+    while (s + 1 < m.n_seq && m.tile_off[s + 1] <= u) ++s;
+    L = m.L[s];
+    tpr = (L + kTileKeys - 1) / kTileKeys;
+    const int local = u - m.tile_off[s];
+    row = s * m.rows_per_seq + local / tpr;
+    tile = local % tpr;
+    key0 = m.key_off[s] + (long long)(row - s * m.rows_per_seq) * L;
+  }
+  __device__ __forceinline__ void next(const RowMap& m) {
+    if (++tile < tpr) return;
+    tile = 0;
+    key0 += L;
+    ++row;
+    if (row % m.rows_per_seq == 0 && row < m.n_rows) {  // the next sequence's first row
+      L = m.L[row / m.rows_per_seq];
+      tpr = (L + kTileKeys - 1) / kTileKeys;
+    }
+  }
+  __device__ __forceinline__ int nvalid() const { return min(kTileKeys, L - tile * kTileKeys); }
 };
 
 // Epilogue warps with work per accumulator buffer: pass 1, the (row half,
@@ -78,7 +106,7 @@ __host__ __device__ constexpr int epi_active_warps(int R, int n2) {
   return ((n2 + 31) / 32) / 2 > 0 ? 8 : 4;
 }
 
-template <int PASS>
+template <int PASS, int NK>  // NK: 64-column chunks of d
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const TcArgs a) {
@@ -134,16 +162,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int it = 0, cur_row = -1;
-      uint32_t qe_phase = 0;
+      TileIter ti;
+      if (u0 < u1) ti.init(a.map, u0);
+      int cur_row = -1, st = 0;
+      uint32_t qe_phase = 0, kphase = 0;  // kphase: the parity of the stage ring's current round
       bool have_q = false;
       bool k_issued[kStages] = {false, false, false, false};
       uint32_t k_parity[kStages] = {0, 0, 0, 0};
       uint32_t q_parity = 0;
       bool aborted = false;
-      for (int u = u0; u < u1; ++u, ++it) {
-        int row, tile;
-        tile_to_row(a.map, u, row, tile);
+      for (int u = u0; u < u1; ++u, ti.next(a.map)) {
+        const int row = ti.row;
         if (row != cur_row) {
           if (have_q) {
             if (!wait_bounded(q_empty, qe_phase, g)) { aborted = true; break; }
@@ -152,21 +181,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           have_q = true;
           cur_row = row;
-          mbar_arrive_expect_tx(q_full, a.nk * kQChunkBytes);
-          for (int c = 0; c < a.nk; ++c) tma_load_2d(sQ + c * kQChunkBytes, &tmQ, q_full, c * 64, row * a.R);
+          mbar_arrive_expect_tx(q_full, NK * kQChunkBytes);
+#pragma unroll
+          for (int c = 0; c < NK; ++c) tma_load_2d(sQ + c * kQChunkBytes, &tmQ, q_full, c * 64, row * a.R);
         }
-        const int st = it % kStages;
-        if (it >= kStages && !wait_bounded(&empty_k[st], ((it / kStages) - 1) & 1, g)) { aborted = true; break; }
-        mbar_arrive_expect_tx(&full_k[st], a.nk * kKChunkBytes);
-        const long long key0 = row_key_off(a.map, row) + (long long)tile * kTileKeys;
-        for (int c = 0; c < a.nk; ++c)
-          tma_load_2d(sK + st * kKStageBytes + c * kKChunkBytes, &tmK, &full_k[st], c * 64, (int)key0);
+        // the stage's previous round has been consumed (from the second round on)
+        if (u - u0 >= kStages && !wait_bounded(&empty_k[st], kphase ^ 1, g)) { aborted = true; break; }
+        mbar_arrive_expect_tx(&full_k[st], NK * kKChunkBytes);
+        const int key0 = (int)(ti.key0 + (long long)ti.tile * kTileKeys);
+#pragma unroll
+        for (int c = 0; c < NK; ++c)
+          tma_load_2d(sK + st * kKStageBytes + c * kKChunkBytes, &tmK, &full_k[st], c * 64, key0);
 #pragma unroll
         for (int z = 0; z < kStages; ++z)  // constant indices: the arrays stay in registers
           if (z == st) {
             k_issued[z] = true;
-            k_parity[z] = (it / kStages) & 1;
+            k_parity[z] = kphase;
           }
+        if (++st == kStages) {
+          st = 0;
+          kphase ^= 1;
+        }
       }
       // let every copy issued land before the CTA's shared memory goes away (after
       // a normal run they all have; after an abort raised anywhere some may not)
@@ -179,45 +214,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0, cur_row = -1;
-      uint32_t qf_phase = 0;
-      const uint32_t qbase = smem_u32(sQ);
-      for (int u = u0; u < u1; ++u, ++it) {
-        int row, tile;
-        tile_to_row(a.map, u, row, tile);
+      // One thread issues every MMA and shares its scheduler with four busy
+      // epilogue warps, so its loop is kept short: no search for the tile's row,
+      // and the operand descriptors are fixed ones plus constant offsets (the
+      // 14-bit address field holds (address >> 4), which an added offset inside
+      // shared memory never carries out of).
+      TileIter ti;
+      if (u0 < u1) ti.init(a.map, u0);
+      int cur_row = -1, st = 0;
+      uint32_t qf_phase = 0, kphase = 0;
+      const uint64_t qdesc = sw128_kmajor_desc(smem_u32(sQ));
+      const uint64_t kdesc = sw128_kmajor_desc(smem_u32(sK));
+      const uint32_t idesc = PASS == 1 ? idesc_bf16_f32(128, 128) : idesc_bf16_f32(128, a.n2);
+      const bool upper = a.R > 128;  // pass 1: window rows in the second 128-row half
+      for (int u = u0, it = 0; u < u1; ++u, ++it) {
+        const int row = ti.row;
         if (row != cur_row) {
           if (!wait_bounded(q_full, qf_phase, g)) break;
           qf_phase ^= 1;
           cur_row = row;
         }
-        const int st = it % kStages;
-        if (!wait_bounded(&full_k[st], (it / kStages) & 1, g)) break;
+        if (!wait_bounded(&full_k[st], kphase, g)) break;
         const int acc = it & 1;
         if (it >= 2 && !wait_bounded(&acc_empty[acc], ((it >> 1) - 1) & 1, g)) break;
         tc_fence_after();
         const uint32_t d_base = tmem + acc * 256;
-        const uint32_t kbase = smem_u32(sK + st * kKStageBytes);
+        const uint64_t kd = kdesc + (uint64_t)((st * kKStageBytes) >> 4);
+        uint64_t qd = qdesc;
+        asm volatile("" : "+l"(qd));  // offsets added per tile, not all held across the loop
         if (PASS == 1) {
-          const uint32_t idesc = idesc_bf16_f32(128, 128);
-          for (int h = 0; h * 128 < a.R; ++h)
-            for (int kk = 0; kk < a.nk * 4; ++kk) {
-              const uint64_t ad = sw128_kmajor_desc(qbase + (kk >> 2) * kQChunkBytes + h * 128 * 128 + (kk & 3) * 32);
-              const uint64_t bd = sw128_kmajor_desc(kbase + (kk >> 2) * kKChunkBytes + (kk & 3) * 32);
-              tc_mma_bf16(d_base + h * 128, ad, bd, idesc, kk > 0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (h == 0 || upper) {
+#pragma unroll
+              for (int kk = 0; kk < NK * 4; ++kk)
+                tc_mma_bf16(d_base + h * 128,
+                            qd + (uint64_t)(((kk >> 2) * kQChunkBytes + h * 128 * 128 + (kk & 3) * 32) >> 4),
+                            kd + (uint64_t)(((kk >> 2) * kKChunkBytes + (kk & 3) * 32) >> 4), idesc, kk > 0);
             }
         } else {
-          const uint32_t idesc = idesc_bf16_f32(128, a.n2);
-          for (int kk = 0; kk < a.nk * 4; ++kk) {
-            const uint64_t ad = sw128_kmajor_desc(kbase + (kk >> 2) * kKChunkBytes + (kk & 3) * 32);
-            const uint64_t bd = sw128_kmajor_desc(qbase + (kk >> 2) * kQChunkBytes + (kk & 3) * 32);
-            tc_mma_bf16(d_base, ad, bd, idesc, kk > 0);
-          }
+#pragma unroll
+          for (int kk = 0; kk < NK * 4; ++kk)
+            tc_mma_bf16(d_base, kd + (uint64_t)(((kk >> 2) * kKChunkBytes + (kk & 3) * 32) >> 4),
+                        qd + (uint64_t)(((kk >> 2) * kQChunkBytes + (kk & 3) * 32) >> 4), idesc, kk > 0);
         }
         tc_commit(&empty_k[st]);
         tc_commit(&acc_full[acc]);
-        int nrow = -1, ntile;
-        if (u + 1 < u1) tile_to_row(a.map, u + 1, nrow, ntile);
-        if (nrow != row) tc_commit(q_empty);
+        ti.next(a.map);
+        if (u + 1 >= u1 || ti.row != row) tc_commit(q_empty);  // the row's last tile: Q may be replaced
+        if (++st == kStages) {
+          st = 0;
+          kphase ^= 1;
+        }
       }
       // every issued MMA has finished before TMEM is released
       tc_commit(drain);
@@ -236,11 +284,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool pair = PASS == 2 && nc / 2 > 0;  // both column halves active: hand-off through shared memory
     const int n_pair = 32 * epi_active_warps<PASS>(a.R, a.n2);  // pass 2: the buffer's threads
     float* part = reinterpret_cast<float*>(smem + kSmemPart);
+    TileIter ti;  // pass 1; pass 2 looks each tile up (its epilogue has no registers to spare)
+    if (PASS == 1 && u0 + bf < u1) ti.init(a.map, u0 + bf);
     for (int u = u0 + bf; active && u < u1; u += 2) {
       const int it = u - u0;
-      int row, tile;
-      tile_to_row(a.map, u, row, tile);
-      const int nvalid = min(kTileKeys, row_len(a.map, row) - tile * kTileKeys);
+      int row, tile, nvalid;
+      if (PASS == 1) {
+        row = ti.row;
+        tile = ti.tile;
+        nvalid = ti.nvalid();
+        ti.next(a.map);  // this buffer's next tile is two on
+        ti.next(a.map);
+      } else {
+        tile_to_row(a.map, u, row, tile);
+        nvalid = min(kTileKeys, row_len(a.map, row) - tile * kTileKeys);
+      }
       // the warp (pass 2: the buffer's warps) leave together: tensor-memory loads are
       // warp-wide and the column halves meet at a barrier
       bool ok = __all_sync(0xffffffffu, wait_bounded(&acc_full[bf], (it >> 1) & 1, g));
@@ -495,17 +553,16 @@ int launch_score(const kv_shape& sh, const RowMap& m, const void* qwin, const vo
     if (!encode_rows_bf16(&tmQ, qwin, d, (long long)m.n_rows * R, kQRows)) return KV_ERR_CUDA;
     if (!encode_rows_bf16(&tmK, K, d, total_keys(m), kTileKeys)) return KV_ERR_CUDA;
     // per-device settings: made on every launch (cheap), for whichever device is current
-    if (cudaFuncSetAttribute(score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(score_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
-            cudaSuccess)
+    auto k1 = d == 128 ? score_tc_kernel<1, 2> : score_tc_kernel<1, 1>;
+    auto k2 = d == 128 ? score_tc_kernel<2, 2> : score_tc_kernel<2, 1>;
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) != cudaSuccess)
       return KV_ERR_CUDA;
     TcArgs a;
     a.map = m;
     a.R = R;
     a.Rs = (R + 3) & ~3;
     a.n2 = ((R + 15) / 16) * 16;
-    a.nk = d / 64;
     a.total_tiles = total_tiles;
     a.c = c;
     a.partial = partial;
@@ -514,9 +571,9 @@ int launch_score(const kv_shape& sh, const RowMap& m, const void* qwin, const vo
     a.status = status;
     a.limit_ns = wait_limit_ns();
     const int grid = std::min(sm_count(), total_tiles);
-    score_tc_kernel<1><<<grid, kThreads, kSmemAlloc, st>>>(tmQ, tmK, a);
+    k1<<<grid, kThreads, kSmemAlloc, st>>>(tmQ, tmK, a);
     score_merge_kernel<<<m.n_rows, merge_threads, 0, st>>>(m, R, (R + 3) & ~3, c, partial, lse2);
-    score_tc_kernel<2><<<grid, kThreads, kSmemAlloc, st>>>(tmQ, tmK, a);
+    k2<<<grid, kThreads, kSmemAlloc, st>>>(tmQ, tmK, a);
   } else {
     const size_t sm1 = (size_t)(kTileKeys + R) * (d + 1) * sizeof(float);
     const size_t sm2 = sm1 + (size_t)R * sizeof(float);
