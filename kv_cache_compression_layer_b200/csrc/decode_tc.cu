@@ -888,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const int nq = (E + kOutUnit - 1) / kOutUnit;
   const int r_lo = rlo_s, r_hi = rhi_s, own_lo = own_s;
   const long long S0 = rng_s[0], S1 = rng_s[1];
-  constexpr int UP = 12;  // slot pairs per lane in flight in the sweep
+  constexpr int UP = 6;  // slots per lane in flight in the sweep
   // The first batch's slot data (logits written by this CTA, A, positions: none of it
   // waits for another CTA) is copied into the rest of the freed ring now, without
   // waiting; the sweep reads it from there.
@@ -963,44 +963,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         float lse[kTcMaxG];
 #pragma unroll
         for (int g = 0; g < kTcMaxG; ++g) lse[g] = g < G ? rs[ri].lse[g] : 0.f;
-        // lane pairs share a slot: each lane loads 4 of its 8 logits, so a warp's
-        // request is 512 contiguous bytes
+        // one slot per lane (all eight logits, A and the position), U slots per lane
+        // with every load issued before the first use
         constexpr int U = UP;
-        const int half = lane & 1, sl = lane >> 1;
-        float lh[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) lh[k] = half ? lse[4 + k] : lse[k];
-        for (long long s0 = p0; s0 < p1; s0 += 16 * U) {
-          float4 lv[U];
+        for (long long s0 = p0; s0 < p1; s0 += 32 * U) {
+          float4 la[U], lb[U];
           float Av[U];
           int pv[U];
-          if (s0 >= stg0 && min(s0 + 16 * U, p1) <= stg0 + nst) {  // staged in shared memory
+          if (s0 >= stg0 && min(s0 + 32 * U, p1) <= stg0 + nst) {  // staged in shared memory
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {
-              const int k = (int)(min(s0 + uu * 16 + sl, p1 - 1) - stg0);
-              lv[uu] = *reinterpret_cast<const float4*>(st_lg + k * kTcMaxG + half * 4);
+              const int k = (int)(min(s0 + uu * 32 + lane, p1 - 1) - stg0);
+              la[uu] = *reinterpret_cast<const float4*>(st_lg + k * kTcMaxG);
+              lb[uu] = *reinterpret_cast<const float4*>(st_lg + k * kTcMaxG + 4);
               Av[uu] = st_A[k];
               pv[uu] = st_pos[k];
             }
           } else {
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {  // every load first, addresses clamped into the piece
-              const long long s = min(s0 + uu * 16 + sl, p1 - 1);
-              lv[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + half);
+              const long long s = min(s0 + uu * 32 + lane, p1 - 1);
+              la[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG));
+              lb[uu] = __ldcg(reinterpret_cast<const float4*>(sc.logits + s * kTcMaxG) + 1);
               Av[uu] = __ldcg(a.A + s);
               pv[uu] = __ldcg(a.pos + s);
             }
           }
+          const int jb = (int)(s0 - rbase) + lane;
 #pragma unroll
           for (int uu = 0; uu < U; ++uu) {
-            float ps = ex2_approx(lv[uu].x - lh[0]) + ex2_approx(lv[uu].y - lh[1]) + ex2_approx(lv[uu].z - lh[2]) +
-                       ex2_approx(lv[uu].w - lh[3]);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-            const long long s = s0 + uu * 16 + sl;
-            const int j = (int)(s - rbase);
-            if (half == 0 && s < p1 && j < rn_) {
+            const float ps =
+                (((ex2_approx(la[uu].x - lse[0]) + ex2_approx(la[uu].y - lse[1])) + ex2_approx(la[uu].z - lse[2])) +
+                 ex2_approx(la[uu].w - lse[3])) +
+                (((ex2_approx(lb[uu].x - lse[4]) + ex2_approx(lb[uu].y - lse[5])) + ex2_approx(lb[uu].z - lse[6])) +
+                 ex2_approx(lb[uu].w - lse[7]));
+            const int j = jb + uu * 32;
+            if (j < (int)(p1 - rbase) && j < rn_) {
               const float Anew = (j == rnext ? 0.f : a.gamma * Av[uu]) + ps;
-              st_f32_hint_nc(a.A + s, Anew, keep);  // read again by the next step
+              st_f32_hint_nc(a.A + rbase + j, Anew, keep);  // read again by the next step
               const int pj = j == rnext ? rpos_new : pv[uu];
               if (j >= a.T && pj < rpos_thr) {
                 const Best c{Anew, pj, j};
