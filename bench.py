@@ -44,11 +44,11 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {"3b": {"bytes": 139746048,  # profiles/decode_cl_kernel_3b.md
                       "source": "kv_cache_compression_layer_b200/csrc/decode_cl.cu",
                       "sha256": "45d44be40b24b73b"},
-               # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (257,690,624 B for
+               # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (256,964,096 B for
                # 483,224 slots) scaled by the slots of the full batch (x 4)
-               "ragged": {"bytes": 1030762496,
+               "ragged": {"bytes": 1027856384,
                           "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
-                          "sha256": "c079ebe6e00045ad"}}
+                          "sha256": "51c4a6b218d8429a"}}
 
 
 def decode_kernel(cfg: synth.Config, sms: int) -> str:

@@ -46,7 +46,10 @@ constexpr int kSmemBar = kSmemK + kStages * kKStageBytes;
 constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int kSmemMisc = kSmemBar + kNumBars * 8;
 constexpr int kSmemPart = kSmemMisc + 16;                  // pass 2: [buffer][parity][128 keys] float
-constexpr int kSmemTotal = kSmemPart + 2 * 2 * kTileKeys * 4;
+// pass 2: [epilogue warp][128 columns] float, read as float4 (16-byte aligned)
+constexpr int kSmemLse = (kSmemPart + 2 * 2 * kTileKeys * 4 + 127) & ~127;
+static_assert(kSmemLse % 16 == 0, "float4 reads of the staged lse2");
+constexpr int kSmemTotal = kSmemLse + kEpiWarps * 128 * 4;
 constexpr int kSmemAlloc = kSmemTotal + 1024;  // slack for 1024-byte alignment
 
 struct TcArgs {
@@ -284,6 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool pair = PASS == 2 && nc / 2 > 0;  // both column halves active: hand-off through shared memory
     const int n_pair = 32 * epi_active_warps<PASS>(a.R, a.n2);  // pass 2: the buffer's threads
     float* part = reinterpret_cast<float*>(smem + kSmemPart);
+    // pass 2: this warp's columns of the current row's lse2, staged once per row
+    float* lse_s = reinterpret_cast<float*>(smem + kSmemLse) + e * 128;
+    int lrow = -1;
     TileIter ti;  // pass 1; pass 2 looks each tile up (its epilogue has no registers to spare)
     if (PASS == 1 && u0 + bf < u1) ti.init(a.map, u0 + bf);
     for (int u = u0 + bf; active && u < u1; u += 2) {
@@ -298,6 +304,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         tile_to_row(a.map, u, row, tile);
         nvalid = min(kTileKeys, row_len(a.map, row) - tile * kTileKeys);
+      }
+      if (PASS == 2 && row != lrow) {
+        __syncwarp();  // the previous row's values are no longer read
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int col = (c_lo + k) * 32 + lane;
+          if (c_lo + k < c_hi) lse_s[k * 32 + lane] = col < a.R ? __ldg(a.lse2 + (long long)row * a.Rs + col) : 0.f;
+        }
+        __syncwarp();
+        lrow = row;
       }
       // the warp (pass 2: the buffer's warps) leave together: tensor-memory loads are
       // warp-wide and the column halves meet at a barrier
@@ -368,14 +384,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this thread's key: the sum over its half of the window rows of
         // exp2(x c - lse_r), chunk by chunk
         const int j = quarter * 32 + lane;
-        const float* lse = a.lse2 + (long long)row * a.Rs;
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};  // independent add chains, combined in a fixed order
         auto colsum = [&](const float (&x)[32], int ch) {
           const int col = ch * 32;
+          const float* lc = lse_s + (ch - c_lo) * 32;
           if (col + 32 <= a.R) {  // a full chunk of window rows: no masks
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-              const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse + col + i));
+              const float4 l4 = *reinterpret_cast<const float4*>(lc + i);
               sum4[0] += ex2_approx(fmaf(x[i + 0], a.c, -l4.x));
               sum4[1] += ex2_approx(fmaf(x[i + 1], a.c, -l4.y));
               sum4[2] += ex2_approx(fmaf(x[i + 2], a.c, -l4.z));
@@ -385,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               if (col + i < a.R) {
-                const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse + col + i));
+                const float4 l4 = *reinterpret_cast<const float4*>(lc + i);
                 const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
