@@ -196,14 +196,16 @@ int kv_allocate_global(const kv_shape* shape, const int32_t* L, int32_t n_seq, c
  *   keep the last w positions and the top-(b - w) positions of s_hat over
  *   [0, L - w) (ties to the lower index), in ascending order; then
  *   Kc[slot_off_i + t] = K[koff_i + idx_t], same for V.
- *   s_hat : device, [sum L] float32;  K, V : device, [sum L][d] dtype.
+ *   s_hat : device, [sum L] float32;  K, V : [sum L][d] dtype, device memory or
+ *           pinned (page-locked) host memory: only the b kept rows of each row are
+ *           read, so K or V left on the host cross the host link b rows at a time.
  *   b, slot_off : device, from kv_allocate.
  *   idx   : device, [total_slots] int32 (output; row i writes b_i entries at
  *           slot_off[i]; the spare slot is left untouched). idx doubles as
  *           the initial `pos` array of the decode cache.
  *   Kc, Vc : device, [total_slots][d] dtype (output, same slots).
  *   A row with b < w (never produced by kv_allocate) is left unwritten.
- * Errors: KV_ERR_ARG, KV_ERR_UNSUPPORTED_L, KV_ERR_CUDA.
+ * Errors: KV_ERR_ARG (also for K or V in pageable host memory), KV_ERR_UNSUPPORTED_L, KV_ERR_CUDA.
  */
 int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat, const void* K,
                      const void* V, const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
@@ -218,9 +220,9 @@ int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, con
  * q_i = floor(k len_i / (L - w)) of the k = b - w kept candidates, plus one
  * for the (k - sum q) segments with the largest remainders k len_i mod (L - w)
  * (ties to the lower segment), choosing its top-q_i by s_hat (ties to the
- * lower index). The window, the b >= L bypass, the outputs and the gather
- * are those of kv_select_gather. 1 <= n_segments <= 4096; n_segments = 1 is
- * kv_select_gather.
+ * lower index). The window, the b >= L bypass, the outputs, the gather and
+ * where K and V may live are those of kv_select_gather. 1 <= n_segments <=
+ * 4096; n_segments = 1 is kv_select_gather.
  * Errors: KV_ERR_ARG, KV_ERR_CUDA.
  */
 int kv_select_gather_segmented(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat,

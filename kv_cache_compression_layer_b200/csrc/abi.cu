@@ -201,6 +201,20 @@ int kv_allocate_global(const kv_shape* shape, const int32_t* L, int32_t n_seq, c
   return launch_allocate(*shape, m, *params, S, b, slot_off, true, static_cast<cudaStream_t>(stream));
 }
 
+// The address a kernel reads a gather source at: device or managed memory as
+// is, pinned host memory at its device mapping; nullptr for memory the device
+// cannot read (pageable host memory).
+static const void* gather_source(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return p;
+  if (at.type == cudaMemoryTypeHost && at.devicePointer) return at.devicePointer;
+  return nullptr;
+}
+
 int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, const float* s_hat, const void* K,
                      const void* V, const int32_t* b, const int64_t* slot_off, int32_t* idx, void* Kc, void* Vc,
                      void* stream) {
@@ -212,6 +226,9 @@ int kv_select_gather(const kv_shape* shape, const int32_t* L, int32_t n_seq, con
   for (const void* p : {(const void*)s_hat, K, V, (const void*)b, (const void*)slot_off, (const void*)idx,
                         (const void*)Kc, (const void*)Vc})
     if (!aligned16(p)) return KV_ERR_ARG;
+  K = gather_source(K);
+  V = gather_source(V);
+  if (!K || !V) return KV_ERR_ARG;
   return launch_select_gather(*shape, m, s_hat, K, V, b, slot_off, idx, Kc, Vc, 0, static_cast<cudaStream_t>(stream));
 }
 
@@ -226,6 +243,9 @@ int kv_select_gather_segmented(const kv_shape* shape, const int32_t* L, int32_t 
   for (const void* p : {(const void*)s_hat, K, V, (const void*)b, (const void*)slot_off, (const void*)idx,
                         (const void*)Kc, (const void*)Vc})
     if (!aligned16(p)) return KV_ERR_ARG;
+  K = gather_source(K);
+  V = gather_source(V);
+  if (!K || !V) return KV_ERR_ARG;
   return launch_select_gather(*shape, m, s_hat, K, V, b, slot_off, idx, Kc, Vc, n_segments,
                               static_cast<cudaStream_t>(stream));
 }

@@ -82,9 +82,95 @@ class Compressor:
         self.select_gather(K, V, stream)
         self.decode_init(stream)
 
+    def compress_from_host(self, host: dict, dev: dict, stream=None, copy_stream=None) -> int:
+        """The same path with its inputs in pinned host memory, the copies overlapped with the work.
+
+        ``host`` holds pinned CPU tensors qwin, K, V, S (and the harness's spikes); ``dev`` device
+        buffers of the same shapes for qwin, K, S (and spikes). On ``copy_stream`` S and the window
+        queries are copied first, then K one sequence at a time; on ``stream`` each sequence is
+        scored and smoothed as soon as its keys have arrived (every row is an independent problem,
+        so a sequence is a batch of its own for kv_score and kv_sss). V is not copied: select +
+        gather reads the kept rows straight from the pinned host tensor over the host link (the
+        path needs only those b rows of each row's L). Returns the host bytes the device reads.
+        """
+        dev_ = self.device
+        stream = stream if stream is not None else torch.cuda.current_stream(dev_)
+        copy_stream = copy_stream if copy_stream is not None else torch.cuda.Stream(dev_)
+        copy_stream.wait_stream(stream)  # the device buffers are no longer in use
+        rps = self.shape.n_layers * self.shape.n_kv_heads
+        spikes = "spikes" in host
+        nbytes = 0
+
+        def copy(name, lo=None, hi=None):
+            nonlocal nbytes
+            src = host[name] if lo is None else host[name][lo:hi]
+            dst = dev[name] if lo is None else dev[name][lo:hi]
+            dst.copy_(src, non_blocking=True)
+            nbytes += src.numel() * src.element_size()
+
+        with torch.cuda.stream(copy_stream):
+            copy("S")
+            copy("qwin")
+        ev = torch.cuda.Event()
+        ev.record(copy_stream)
+        stream.wait_event(ev)
+        self.allocate(dev["S"], stream)
+        key0 = 0
+        for sq, L in enumerate(self.L):
+            key1 = key0 + rps * L
+            with torch.cuda.stream(copy_stream):
+                copy("K", key0, key1)
+                if spikes:
+                    copy("spikes", key0, key1)
+            ev = torch.cuda.Event()
+            ev.record(copy_stream)
+            stream.wait_event(ev)
+            r0, r1 = sq * rps, (sq + 1) * rps
+            kv_score(self.shape, [L], dev["qwin"][r0:r1], dev["K"][key0:key1], self.s[key0:key1], self.ws,
+                     self.ws_bytes, stream)
+            if spikes:
+                with torch.cuda.stream(stream):
+                    self.s[key0:key1].mul_(dev["spikes"][key0:key1])
+            kv_sss(self.shape, [L], self.s[key0:key1], self.s_hat[key0:key1], self.kstar[r0:r1], self.params.alpha,
+                   self.params.rho, stream)
+            key0 = key1
+        self.select_gather(dev["K"], host["V"], stream)
+        self.decode_init(stream)
+        return nbytes
+
     # -- decode ----------------------------------------------------------------
     def decode_step(self, q_t, k_t, v_t, out, stream=None):
         kv_decode_attn_update(self.shape, self.L, self.params, self.cache, q_t, k_t, v_t, out, stream)
+
+    def decode_from_host(self, q, k, v, out_host, dq, dk, dv, out, stream=None, copy_stream=None, d2h_stream=None):
+        """Decode steps t = 0.. with their inputs q[t], k[t], v[t] in pinned host memory and each
+        step's output read back into out_host[t]: the inputs go over the host link on ``copy_stream``
+        (after the work already queued on ``stream``) and the outputs on ``d2h_stream``, both
+        overlapped with the steps. dq, dk, dv, out: device buffers shaped like q, k, v, out_host."""
+        dev_ = self.device
+        stream = stream if stream is not None else torch.cuda.current_stream(dev_)
+        copy_stream = copy_stream if copy_stream is not None else torch.cuda.Stream(dev_)
+        d2h_stream = d2h_stream if d2h_stream is not None else torch.cuda.Stream(dev_)
+        copy_stream.wait_stream(stream)
+        d2h_stream.wait_stream(stream)
+        ev_in = []
+        with torch.cuda.stream(copy_stream):
+            for t in range(q.shape[0]):
+                dq[t].copy_(q[t], non_blocking=True)
+                dk[t].copy_(k[t], non_blocking=True)
+                dv[t].copy_(v[t], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_stream)
+                ev_in.append(ev)
+        for t in range(q.shape[0]):
+            stream.wait_event(ev_in[t])
+            self.decode_step(dq[t], dk[t], dv[t], out[t], stream)
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            d2h_stream.wait_event(ev)
+            with torch.cuda.stream(d2h_stream):
+                out_host[t].copy_(out[t], non_blocking=True)
+        stream.wait_stream(d2h_stream)  # the caller's later work on stream sees every output on the host
 
     # -- host views for checks -------------------------------------------------
     def kept(self):
