@@ -333,6 +333,8 @@ __global__ void __launch_bounds__(kSssThreads, 1)
   uint16_t* rev = reinterpret_cast<uint16_t*>(sss_smem + Lay::kTwBytes);
   double2* zb = reinterpret_cast<double2*>(sss_smem + Lay::kDataOff);
   __shared__ int rad_s[kMaxStages];
+  __shared__ unsigned mg_s[kMaxStages];  // per stage: ceil(2^32 / radix), for k / radix by a multiply-high
+  __shared__ int blk_s[kMaxStages];      // per stage: N over the product of the radices up to it
   __shared__ int m_s;
   __shared__ double wsum[kSssWarps];
   __shared__ double gsum[4];
@@ -363,8 +365,10 @@ __global__ void __launch_bounds__(kSssThreads, 1)
       else if (rest % 3 == 0) r = 3;
       else if (rest % 5 == 0) r = 5;
       else r = 7;  // lengths with other prime factors are rejected on the host
-      rad_s[m++] = r;
+      rad_s[m] = r;
+      mg_s[m] = (unsigned)((0x100000000ull + (unsigned)r - 1) / (unsigned)r);
       rest /= r;
+      blk_s[m++] = rest;
     }
     m_s = m;
   }
@@ -396,11 +400,9 @@ __global__ void __launch_bounds__(kSssThreads, 1)
       kk[j] = k0 + (int)threadIdx.x + j * kSssThreads;
       pos[j] = 0;
     }
-    int B = N;
     for (int i = 0; i < m; ++i) {
-      const int r = rad_s[i];
-      const unsigned mg = (unsigned)((0x100000000ull + (unsigned)r - 1) / (unsigned)r);  // kk / r for kk < 2^16
-      B /= r;
+      const int r = rad_s[i], B = blk_s[i];
+      const unsigned mg = mg_s[i];  // kk / r for kk < 2^16
 #pragma unroll
       for (int j = 0; j < kRevPer; ++j) {
         const int q = (int)__umulhi((unsigned)kk[j], mg);
