@@ -362,7 +362,10 @@ def run_ours(args, rank, world, local_rank):
                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": measured_traffic(args.config) if tc and not args.layers else None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},
         "e2e": {"value": job_throughput(tokens, world, e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
+                "path": "pinned host inputs; K copied a sequence at a time under the scoring of the sequences "
+                        "already on the device, the kept V rows read over the host link by select + gather, "
+                        "decode inputs and outputs crossing during the decode steps"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
