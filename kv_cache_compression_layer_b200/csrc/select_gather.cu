@@ -27,12 +27,12 @@ __host__ __device__ __forceinline__ int map_max_len(const RowMap& m) {
   return x;
 }
 
-// Dynamic shared memory of select_kernel: the keys of the longest row, and for
-// the segment-wise variant the quotas, their prefix and the warps' histograms.
+// Dynamic shared memory of select_kernel: the keys of the longest row, for the
+// segment-wise variant the quotas and their prefix, and the warps' histograms.
 size_t sel_smem_bytes(const RowMap& m, int nseg) {
   size_t b = (size_t)map_max_len(m) * sizeof(uint32_t);
-  if (nseg > 0) b += 2 * (size_t)nseg * sizeof(int) + (size_t)kSelWarps * 256 * sizeof(int);
-  return b;
+  if (nseg > 0) b += 2 * (size_t)nseg * sizeof(int);
+  return b + (size_t)kSelWarps * 256 * sizeof(int);
 }
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -41,10 +41,50 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The bin of the kk-th largest key from a 256-bin histogram, by one warp: lane
+// l holds bins 255 - 8 l down to 248 - 8 l, so lanes in order walk the bins
+// from the top. Returns the bin; kk becomes the rank within it.
+__device__ __forceinline__ int top_bin(const int* hist, int& kk) {
+  const int lane = threadIdx.x & 31;
+  int loc[8], tot = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    loc[t] = hist[255 - 8 * lane - t];
+    tot += loc[t];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - tot;
+  const unsigned here = __ballot_sync(0xffffffffu, excl < kk && kk <= incl);
+  const int src = __ffs(here) - 1;
+  int dg = 0, kk_new = kk;
+  if (lane == src) {
+    int cum = excl;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (cum + loc[t] >= kk) {
+        dg = 255 - 8 * lane - t;
+        kk_new = kk - cum;
+        break;
+      }
+      cum += loc[t];
+    }
+  }
+  dg = __shfl_sync(0xffffffffu, dg, src);
+  kk = __shfl_sync(0xffffffffu, kk_new, src);
+  return dg;
+}
+
 // The k largest keys of keys[c0s, c1s) (ties to the lower index) written to
-// out[0, k) in ascending index order; called by the whole block.
+// out[0, k) in ascending index order; called by the whole block. Each radix
+// round counts into per-warp histograms (no atomics between warps: the
+// scores' top bytes take few values), merged once per round.
 __device__ void select_range(const uint32_t* keys, int c0s, int c1s, int k, int32_t* __restrict__ out, int* hist,
-                             int* wgt, int* weq, uint32_t* sh_prefix, int* sh_kk) {
+                             int (*whist)[256], int* wgt, int* weq, uint32_t* sh_prefix, int* sh_kk) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = c1s - c0s;
   __syncthreads();  // the keys are in place, the previous range's scratch is free
@@ -56,22 +96,27 @@ __device__ void select_range(const uint32_t* keys, int c0s, int c1s, int k, int3
   // radix select of the k-th largest key, most significant byte first
   uint32_t mask = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < kSelWarps * 256; i += kSelThreads) (&whist[0][0])[i] = 0;
     __syncthreads();
     const uint32_t prefix = *sh_prefix;
     for (int j = c0s + threadIdx.x; j < c1s; j += kSelThreads) {
       const uint32_t key = keys[j];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+      if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int kk = *sh_kk, cum = 0, dg = 0;
-      for (dg = 255; dg > 0; --dg) {
-        if (cum + hist[dg] >= kk) break;
-        cum += hist[dg];
+    for (int b = threadIdx.x; b < 256; b += kSelThreads) {  // warp order: a fixed sum
+      int t = 0;
+      for (int w = 0; w < kSelWarps; ++w) t += whist[w][b];
+      hist[b] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int kk = *sh_kk;
+      const int dg = top_bin(hist, kk);
+      if (lane == 0) {
+        *sh_kk = kk;
+        *sh_prefix = prefix | ((uint32_t)dg << shift);
       }
-      *sh_kk = kk - cum;
-      *sh_prefix = prefix | ((uint32_t)dg << shift);
     }
     mask |= 255u << shift;
     __syncthreads();
@@ -134,37 +179,7 @@ __device__ void select_range_warp(const uint32_t* keys, int c0, int c1, int k, i
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
     __syncwarp();
-    // lane l holds bins 255 - 8 l down to 248 - 8 l: lanes in order walk the bins from the top
-    int loc[8], tot = 0;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      loc[t] = hist[255 - 8 * lane - t];
-      tot += loc[t];
-    }
-    int incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int excl = incl - tot;
-    const unsigned here = __ballot_sync(0xffffffffu, excl < kk && kk <= incl);
-    const int src = __ffs(here) - 1;
-    int dg = 0, kk_new = kk;
-    if (lane == src) {
-      int cum = excl;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (cum + loc[t] >= kk) {
-          dg = 255 - 8 * lane - t;
-          kk_new = kk - cum;
-          break;
-        }
-        cum += loc[t];
-      }
-    }
-    dg = __shfl_sync(0xffffffffu, dg, src);
-    kk = __shfl_sync(0xffffffffu, kk_new, src);
+    const int dg = top_bin(hist, kk);
     prefix |= (uint32_t)dg << shift;
     mask |= 255u << shift;
     __syncwarp();  // every lane has read the bins before the next round clears them
@@ -223,7 +238,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (k <= 0) return;
   for (int j = threadIdx.x; j < n; j += kSelThreads) keys[j] = order_key(s_hat[koff + j]);
   if (nseg <= 1) {  // one top-k over the candidates (a single segment is the same selection)
-    select_range(keys, 0, n, k, out, hist, wgt, weq, &sh_prefix, &sh_kk);
+    select_range(keys, 0, n, k, out, hist, whist, wgt, weq, &sh_prefix, &sh_kk);
     return;
   }
   // segment quotas: q_i = floor(k len_i / n), the remainder by largest k len_i mod n
@@ -268,7 +283,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (nseg < kSelWarps / 4) {  // a few long segments: the whole block on each in turn
     for (int i = 0; i < nseg; ++i) {
       const int lo = (int)((long long)i * n / nseg), hi = (int)((long long)(i + 1) * n / nseg);
-      if (q_s[i] > 0) select_range(keys, lo, hi, q_s[i], out + at_s[i], hist, wgt, weq, &sh_prefix, &sh_kk);
+      if (q_s[i] > 0) select_range(keys, lo, hi, q_s[i], out + at_s[i], hist, whist, wgt, weq, &sh_prefix, &sh_kk);
     }
     return;
   }
