@@ -454,10 +454,19 @@ __global__ void __launch_bounds__(kSssThreads, 1)
         sync();
       }
     };
-#pragma unroll 4
-    for (int i = pm0 + tid; i < pm1; i += step) {
-      const float2 x = srow[i];
-      z0.at(i) = make_double2(x.x, x.y);
+#pragma unroll 1
+    for (int j0 = 0; j0 < kMaxPer; j0 += 8) {  // eight of the thread's points' loads in flight at a time
+      float2 x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = pm0 + tid + (j0 + j) * step;
+        if (i < pm1) x[j] = srow[i];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = pm0 + tid + (j0 + j) * step;
+        if (i < pm1) z0.at(i) = make_double2(x[j].x, x[j].y);
+      }
     }
     sync();
     fft<false>(z0, N, L, rad_s, m, tw, bnum, bden, tid, step, sync);
