@@ -91,7 +91,8 @@ class Compressor:
         scored and smoothed as soon as its keys have arrived (every row is an independent problem,
         so a sequence is a batch of its own for kv_score and kv_sss). V is not copied: select +
         gather reads the kept rows straight from the pinned host tensor over the host link (the
-        path needs only those b rows of each row's L). Returns the host bytes the device reads.
+        path needs only those b rows of each row's L). Errors of the scoring calls are OR-ed into
+        the batch's device status word (``self.status``). Returns the host bytes the device reads.
         """
         dev_ = self.device
         stream = stream if stream is not None else torch.cuda.current_stream(dev_)
@@ -128,8 +129,10 @@ class Compressor:
             r0, r1 = sq * rps, (sq + 1) * rps
             kv_score(self.shape, [L], dev["qwin"][r0:r1], dev["K"][key0:key1], self.s[key0:key1], self.ws,
                      self.ws_bytes, stream)
-            if spikes:
-                with torch.cuda.stream(stream):
+            with torch.cuda.stream(stream):
+                # each kv_score call restarts its workspace status word: keep every call's in the batch's
+                self.status[:1].bitwise_or_(self.ws[:4].view(torch.int32))
+                if spikes:
                     self.s[key0:key1].mul_(dev["spikes"][key0:key1])
             kv_sss(self.shape, [L], self.s[key0:key1], self.s_hat[key0:key1], self.kstar[r0:r1], self.params.alpha,
                    self.params.rho, stream)
