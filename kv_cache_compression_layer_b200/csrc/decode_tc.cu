@@ -687,18 +687,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           if (g_ok)
             for (int w4 = 0; w4 < 4; ++w4) M0 = fmaxf(M0, red_m[grp * 4 + w4][g0]);
           const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
-          // the group's warps add their O in warp order (a fixed summation order,
-          // so a step's result does not depend on scheduling); lanes own distinct columns
-          for (int w4 = 0; w4 < 4; ++w4) {
-            if ((warp & 3) == w4 && g_ok) {
+          // the group's warps add their O in four turns; in turn t warp w adds its quarter
+          // (w + t) mod 4 of the columns, so every turn all four warps work and each
+          // column still receives the warps in a fixed order (the step's result does not
+          // depend on scheduling); lanes own distinct columns
+          constexpr int QI = 2 * NDC / 4;  // i-values of a quarter
+          for (int t4 = 0; t4 < 4; ++t4) {
+            if (g_ok) {
+              const int qb = ((warp & 3) + t4) & 3;
               float* ogp = og + g0 * D;
               asm volatile("" : "+l"(ogp));  // addresses formed here, not held across the turns
 #pragma unroll
-              for (int i = 0; i < 2 * NDC; ++i) {
-                const int col = i * 8 + q4 * 2;
-                ogp[ogswz(g0, col)] += o[i][0] * f0;
-                ogp[ogswz(g0, col + 1)] += o[i][1] * f0;
-              }
+              for (int b = 0; b < 4; ++b)
+                if (b == qb) {
+#pragma unroll
+                  for (int ii = 0; ii < QI; ++ii) {
+                    const int i = b * QI + ii;
+                    const int col = i * 8 + q4 * 2;
+                    ogp[ogswz(g0, col)] += o[i][0] * f0;
+                    ogp[ogswz(g0, col + 1)] += o[i][1] * f0;
+                  }
+                }
             }
             named_bar_sync(1 + grp, 128);
           }
