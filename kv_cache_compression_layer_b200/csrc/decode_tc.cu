@@ -687,30 +687,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           if (g_ok)
             for (int w4 = 0; w4 < 4; ++w4) M0 = fmaxf(M0, red_m[grp * 4 + w4][g0]);
           const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
-          // the group's warps add their O in four turns; in turn t warp w adds its quarter
-          // (w + t) mod 4 of the columns, so every turn all four warps work and each
-          // column still receives the warps in a fixed order (the step's result does not
-          // depend on scheduling); lanes own distinct columns
-          constexpr int QI = 2 * NDC / 4;  // i-values of a quarter
-          for (int t4 = 0; t4 < 4; ++t4) {
-            if (g_ok) {
-              const int qb = ((warp & 3) + t4) & 3;
-              float* ogp = og + g0 * D;
-              asm volatile("" : "+l"(ogp));  // addresses formed here, not held across the turns
-#pragma unroll
-              for (int b = 0; b < 4; ++b)
-                if (b == qb) {
-#pragma unroll
-                  for (int ii = 0; ii < QI; ++ii) {
-                    const int i = b * QI + ii;
-                    const int col = i * 8 + q4 * 2;
-                    ogp[ogswz(g0, col)] += o[i][0] * f0;
-                    ogp[ogswz(g0, col + 1)] += o[i][1] * f0;
-                  }
-                }
-            }
-            named_bar_sync(1 + grp, 128);
-          }
           const int pidx = seg_u * kGroups + grp;
           float* part = sc.part + (long long)pidx * sc.stride;
           // the row's list place of this partial: (the segment's first item in the row, group)
@@ -734,12 +710,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             ent->pidx = pidx;
             ent->stamp = segs_s[grp] + 1;
           }
-          for (int i = gt; i < G * D; i += 128) {
-            const int og_i = (i / D) * D + ogswz(i / D, i % D);
-            part[kPartO + i] = og[og_i];
-            og[og_i] = 0.f;
+          // the group's warps add their O in four turns; in turn t warp w adds its quarter
+          // (w + t) mod 4 of the columns, so every turn all four warps work and each
+          // column still receives the warps in a fixed order (the step's result does not
+          // depend on scheduling); in the last turn a column's sum is complete and goes
+          // to the partial, and the buffer is cleared; lanes own distinct columns
+          constexpr int QI = 2 * NDC / 4;  // i-values of a quarter
+          for (int t4 = 0; t4 < 4; ++t4) {
+            if (g_ok) {
+              const int qb = ((warp & 3) + t4) & 3;
+              float* ogp = og + g0 * D;
+              float* pgp = part + kPartO + g0 * D;
+              asm volatile("" : "+l"(ogp), "+l"(pgp));  // addresses formed here, not held across the turns
+#pragma unroll
+              for (int b = 0; b < 4; ++b)
+                if (b == qb) {
+#pragma unroll
+                  for (int ii = 0; ii < QI; ++ii) {
+                    const int i = b * QI + ii;
+                    const int col = i * 8 + q4 * 2;
+                    const int c0 = ogswz(g0, col), c1 = ogswz(g0, col + 1);
+                    if (t4 < 3) {
+                      ogp[c0] += o[i][0] * f0;
+                      ogp[c1] += o[i][1] * f0;
+                    } else {
+                      *reinterpret_cast<float2*>(pgp + col) = make_float2(ogp[c0] + o[i][0] * f0, ogp[c1] + o[i][1] * f0);
+                      ogp[c0] = 0.f;
+                      ogp[c1] = 0.f;
+                    }
+                  }
+                }
+            }
+            named_bar_sync(1 + grp, 128);  // after the last turn: the partial is written
           }
-          named_bar_sync(1 + grp, 128);
           if (gt == 0) {  // count the slots the partial covers, once it is visible (at the end)
             const int qn = dq_n[grp];
             if (qn < kDefer) {
