@@ -44,11 +44,11 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {"3b": {"bytes": 139746048,  # profiles/decode_cl_kernel_3b.md
                       "source": "kv_cache_compression_layer_b200/csrc/decode_cl.cu",
                       "sha256": "45d44be40b24b73b"},
-               # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (256,964,096 B for
+               # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (257,023,232 B for
                # 483,224 slots) scaled by the slots of the full batch (x 4)
-               "ragged": {"bytes": 1027856384,
+               "ragged": {"bytes": 1028092928,
                           "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
-                          "sha256": "51c4a6b218d8429a"}}
+                          "sha256": "683f49d231d41696"}}
 
 
 def decode_kernel(cfg: synth.Config, sms: int) -> str:
