@@ -41,9 +41,9 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one decode kernel launch from an ncu capture of
 # this benchmark's workload (its summary is kept under profiles/), valid while
 # the kernel source is the one captured (its SHA-256 below); otherwise null.
-NCU_TRAFFIC = {"3b": {"bytes": 139746048,  # profiles/decode_cl_kernel_3b.md
-                      "source": "kv_cache_compression_layer_b200/csrc/decode_cl.cu",
-                      "sha256": "45d44be40b24b73b"},
+NCU_TRAFFIC = {"3b": {"bytes": 140328704,  # profiles/decode_tc_kernel_3b.md (the full workload)
+                      "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
+                      "sha256": "683f49d231d41696"},
                # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (257,023,232 B for
                # 483,224 slots) scaled by the slots of the full batch (x 4)
                "ragged": {"bytes": 1028092928,
@@ -51,14 +51,10 @@ NCU_TRAFFIC = {"3b": {"bytes": 139746048,  # profiles/decode_cl_kernel_3b.md
                           "sha256": "683f49d231d41696"}}
 
 
-def decode_kernel(cfg: synth.Config, sms: int) -> str:
+def decode_kernel(cfg: synth.Config) -> str:
     """The decode kernel kv_decode_attn_update launches for this workload (the library's rule)."""
     if cfg.dtype != "bf16" or cfg.group > 8:
         return "decode_simple_kernel"
-    for C in (8, 4, 2, 1):
-        ctas = cfg.rows * C
-        if ctas <= sms and ctas * 8 >= sms * 7:
-            return "decode_cl_kernel"
     return "decode_tc_kernel"
 
 
@@ -357,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
                    "compress_bytes_alg": comp_bytes, "compress_gbs": comp_gbs,
                    "compress_hbm_frac": comp_gbs / peak, "decode_us_per_step": dec_avg_us,
                    "decode_bytes_alg": dec_bytes, "decode_steps": D},
-        "roofline": {"kernel": decode_kernel(cfg, torch.cuda.get_device_properties(dev).multi_processor_count)
+        "roofline": {"kernel": decode_kernel(cfg)
                      + " (kv_decode_attn_update)", "bound": "hbm", "achieved": dec_gbs,
                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak, "traffic": measured_traffic(args.config) if tc and not args.layers else None,
                      "peak_kind": peak_kind + " (hbm_gbs copy)"},

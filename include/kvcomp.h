@@ -253,14 +253,11 @@ int kv_decode_init(const kv_shape* shape, const int32_t* L, int32_t n_seq, const
  *   evict the larger position — and its slot becomes the next free slot.
  *   q_t : device, [rows][g][d] dtype;  k_t, v_t : device, [rows][d] dtype.
  *   out : device, [rows][g][d] dtype.
- * bf16 caches with g <= 8: when the rows fill the GPU as thread-block
- * clusters (rows x C between 7/8 of the SM count and the SM count, C <= 8)
- * each row is one cluster of C CTAs and nothing leaves it; otherwise one
- * persistent launch of one CTA per SM, whose CTAs that share a row wait for
- * each other (bounded: a wait that runs out sets KV_DEV_TIMEOUT, and the
- * decode state is then undefined until kv_decode_init runs again). Steps on
- * one stream are ordered; steps of one cache must not overlap on different
- * streams.
+ * bf16 caches with g <= 8: one persistent launch of one CTA per SM, whose
+ * CTAs that share a row wait for each other (bounded: a wait that runs out
+ * sets KV_DEV_TIMEOUT, and the decode state is then undefined until
+ * kv_decode_init runs again). Steps on one stream are ordered; steps of one
+ * cache must not overlap on different streams.
  * Errors: KV_ERR_ARG, KV_ERR_WORKSPACE, KV_ERR_CUDA.
  */
 int kv_decode_attn_update(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_params* params,

@@ -396,8 +396,6 @@ int launch_decode(const kv_shape& sh, const RowMap& m, const kv_params& p, const
   if (tc_path(sh)) {
     a.C = 1;
     a.S_cap = 0;
-    const int C = cl_cluster_size(sh, m, capb);
-    if (C > 0) return launch_cl(sh, m, capb, C, cache_slots(sh, m, p, c), a, c, st);
     return launch_tc(sh, m, capb, cache_slots(sh, m, p, c), a, c, st);
   }
   cudaError_t e;

@@ -52,9 +52,4 @@ int launch_tc_init(const kv_shape& sh, const RowMap& m, int capb, long long tota
 int launch_tc(const kv_shape& sh, const RowMap& m, int capb, long long total_slots, const DecArgs& a,
               const kv_cache& c, cudaStream_t st);
 
-// Cluster path (decode_cl.cu): the cluster size for this batch, 0 when it does not apply.
-int cl_cluster_size(const kv_shape& sh, const RowMap& m, int capb);
-int launch_cl(const kv_shape& sh, const RowMap& m, int capb, int C, long long total_slots, const DecArgs& a,
-              const kv_cache& c, cudaStream_t st);
-
 }  // namespace kvc

@@ -53,7 +53,7 @@ DECODE_CASES = [
     (synth.CONFIGS["tiny"], 32),
     (synth.small("3b", n_layers=1, L=(2000,)), 24),
     (synth.small("ragged", n_layers=1, L=(1000, 2000), budget_pct=10), 40),  # g = 7, small budgets
-    # enough rows to fill the GPU as clusters: one cluster of 4 (36 rows) or 2 (72 rows) CTAs per row
+    # many rows: 36 (g = 8) and 72 (g = 7), several rows per CTA of the persistent kernel
     (synth.small("3b", n_layers=18, L=(2000,)), 12),
     (synth.small("ragged", n_layers=9, L=(1000, 2000), budget_pct=10), 12),  # g = 7
 ]

@@ -39,7 +39,7 @@ def _steps(cfg, bt, cache, t, steps, first):
     return outs, metas
 
 
-# a batch that fills the GPU as clusters (36 rows x 4 CTAs) and one on the persistent kernel (g = 7)
+# a batch of 36 rows (g = 8) and a ragged one of 16 rows (g = 7)
 RESUME_CASES = [synth.small("3b", n_layers=18, L=(2000,)), synth.small("ragged", n_layers=2, L=(1000, 3500))]
 
 

@@ -6,8 +6,7 @@ land, releases its tensor memory and returns, so the context stays usable:
 with the default limit back, the same calls match the oracle again (decode
 after kv_decode_init, which the header requires after a timed-out step).
 Covered: kv_score (its tensor-core passes) and one step of the persistent
-decode kernel (the work-item path every batch that does not fill the GPU as
-clusters takes).
+decode kernel (the path of every bf16 batch with g <= 8).
 """
 import numpy as np
 import pytest
