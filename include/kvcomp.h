@@ -61,6 +61,7 @@ enum {
 #define KV_DEV_TIMEOUT 0x1
 #define KV_DEV_BUDGET 0x2
 #define KV_DEV_CAPACITY 0x4 /* a row holds more slots than the launch was sized for */
+#define KV_DEV_BOUNDS 0x10  /* debug builds: a checked index fell outside its buffer */
 
 enum { KV_F32 = 0, KV_BF16 = 1 };
 
@@ -308,6 +309,24 @@ uint64_t kv_set_wait_limit_ns(uint64_t limit_ns);
 /* Copies the device status word to the host (synchronises `stream`);
  * returns KV_OK or KV_ERR_CUDA. */
 int kv_read_device_status(const int32_t* status_dev, int32_t* status_host, void* stream);
+
+/*
+ * Debug builds (libkvcomp_debug.so: the same sources compiled with
+ * -DKV_DEBUG_CHECKS). Every kernel checks the indices it takes from data
+ * (kept positions, slot numbers and slot ranges, cluster, node and member
+ * ids, pooled row ranges, recalled blocks) against the extent of the
+ * buffer or row they address; a failed check skips that access (and, where
+ * the rest of the row depends on it, the row) and sets KV_DEV_BOUNDS in the
+ * library's check word. Release builds compile the checks away.
+ * kv_debug_checks returns 1 in a debug build and 0 in a release build.
+ */
+int kv_debug_checks(void);
+
+/* The library's check word (KV_DEV_BOUNDS or 0; always 0 in a release
+ * build) copied to *word_host after all earlier work on the current device
+ * (synchronises the device); clear != 0 resets it to 0 afterwards.
+ * Errors: KV_ERR_ARG (null word_host), KV_ERR_CUDA. */
+int kv_debug_check_word(int32_t* word_host, int32_t clear);
 
 /* Human-readable name of a status code. */
 const char* kv_status_string(int status);

@@ -6,7 +6,10 @@ sm_100a kernels. Functions take torch tensors (or raw device addresses as
 ints) and the current CUDA stream, and raise ``KvError`` on a non-zero
 status. The library must be built (``python -m
 kv_cache_compression_layer_b200.build``); importing the binding without it
-fails loudly, there is no fallback.
+fails loudly, there is no fallback. With KV_DEBUG_CHECKS=1 in the
+environment the binding loads the debug build, libkvcomp_debug.so (built by
+``python -m kv_cache_compression_layer_b200.build --debug``), whose kernels
+check their data-dependent indices (see kv_debug_check_word).
 """
 from __future__ import annotations
 
@@ -15,10 +18,11 @@ import os
 from typing import Optional, Sequence
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libkvcomp.so")
+DEBUG_CHECKS = os.environ.get("KV_DEBUG_CHECKS", "0") not in ("", "0")
+LIB_PATH = os.path.join(HERE, "libkvcomp_debug.so" if DEBUG_CHECKS else "libkvcomp.so")
 
 KV_OK, KV_ERR_ARG, KV_ERR_UNSUPPORTED_L, KV_ERR_BUDGET, KV_ERR_WORKSPACE, KV_ERR_CUDA, KV_ERR_TIMEOUT = range(7)
-KV_DEV_TIMEOUT, KV_DEV_BUDGET, KV_DEV_CAPACITY, KV_DEV_RANGE = 0x1, 0x2, 0x4, 0x8
+KV_DEV_TIMEOUT, KV_DEV_BUDGET, KV_DEV_CAPACITY, KV_DEV_RANGE, KV_DEV_BOUNDS = 0x1, 0x2, 0x4, 0x8, 0x10
 KV_F32, KV_BF16 = 0, 1
 KV_MAX_SEQ = 64
 META_INTS = 8
@@ -29,7 +33,7 @@ EXPORTS = ("kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots"
            "kv_status_string", "kv_score_noalloc", "kv_decode_scratch_bytes", "kv_allocate_global",
            "kv_select_gather_segmented", "kv_voxzip_pool", "kv_wnw_chunk_count", "kv_wnw_state_ints",
            "kv_wnw_init", "kv_wnw_update", "kv_wnw_recall", "kv_c3_index_layout", "kv_c3_build", "kv_c3_step",
-           "kv_set_wait_limit_ns", "kv_score_noalloc_status")
+           "kv_set_wait_limit_ns", "kv_score_noalloc_status", "kv_debug_checks", "kv_debug_check_word")
 KV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -102,6 +106,8 @@ def lib():
             "kv_score_noalloc": (C.c_int, [Ps, P, I32, P, P, P, P]),
             "kv_score_noalloc_status": (C.c_int, [P, P]),
             "kv_set_wait_limit_ns": (C.c_uint64, [C.c_uint64]),
+            "kv_debug_checks": (C.c_int, []),
+            "kv_debug_check_word": (C.c_int, [P, I32]),
             "kv_decode_scratch_bytes": (SZ, [Ps, P, I32, Pp, I64]),
             "kv_voxzip_pool": (C.c_int, [P, I32, P, P, I32, I32, C.c_float, P, P, P, I64, P, P, P, P, P]),
             "kv_wnw_chunk_count": (I64, [P, I32, Pw]),
@@ -366,11 +372,25 @@ def kv_read_device_status(status_dev, stream=None) -> int:
     return host.value
 
 
+def kv_debug_checks() -> bool:
+    """True when the loaded library is the debug build (index checks compiled in)."""
+    return bool(lib().kv_debug_checks())
+
+
+def kv_debug_check_word(clear: bool = False) -> int:
+    """The debug build's check word (KV_DEV_BOUNDS or 0; 0 in a release build),
+    read after all earlier work on the current device; clear resets it."""
+    host = C.c_int32(0)
+    _check("kv_debug_check_word", lib().kv_debug_check_word(C.byref(host), 1 if clear else 0))
+    return host.value
+
+
 from .pipeline import Compressor  # noqa: E402  (the torch-side convenience wrapper)
 
 __all__ = ["kv_shape", "kv_params", "kv_cache", "KvError", "lib", "make_shape", "make_params", "make_cache",
            "kv_rows", "kv_check_lengths", "kv_workspace_bytes", "kv_total_slots", "kv_score", "kv_score_noalloc",
            "kv_score_noalloc_status", "kv_set_wait_limit_ns", "DEFAULT_WAIT_LIMIT_NS", "kv_sss",
+           "kv_debug_checks", "kv_debug_check_word",
            "kv_allocate", "kv_select_gather", "kv_decode_init", "kv_decode_attn_update", "kv_read_device_status",
            "kv_decode_scratch_bytes", "kv_allocate_global", "kv_select_gather_segmented", "kv_voxzip_pool",
            "pack_segments", "ASR_SEGMENT_BYTES", "kv_wnw_params", "make_wnw_params", "kv_wnw_chunk_count",

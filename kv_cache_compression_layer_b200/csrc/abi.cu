@@ -96,6 +96,21 @@ static bool fault_injected(const char* name) {
   return v && std::strcmp(v, name) == 0;
 }
 
+// Readers of the kernel files' check words (debug builds register one per
+// file while the library loads; release builds register none).
+struct CheckReaders {
+  int n = 0;
+  int (*fn[32])(bool);
+};
+CheckReaders& check_readers() {
+  static CheckReaders r;
+  return r;
+}
+void register_check_word(int (*reader)(bool)) {
+  CheckReaders& r = check_readers();
+  if (r.n < 32) r.fn[r.n++] = reader;
+}
+
 }  // namespace kvc
 
 using namespace kvc;
@@ -292,6 +307,27 @@ int kv_read_device_status(const int32_t* status_dev, int32_t* status_host, void*
   if (cudaMemcpyAsync(status_host, status_dev, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return KV_ERR_CUDA;
   return cudaStreamSynchronize(st) == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+int kv_debug_checks(void) {
+#ifdef KV_DEBUG_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int kv_debug_check_word(int32_t* word_host, int32_t clear) {
+  if (!word_host) return KV_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return KV_ERR_CUDA;
+  int w = 0;
+  for (int i = 0; i < kvc::check_readers().n; ++i) {
+    const int v = kvc::check_readers().fn[i](clear != 0);
+    if (v < 0) return KV_ERR_CUDA;
+    w |= v;
+  }
+  *word_host = w;
+  return KV_OK;
 }
 
 const char* kv_status_string(int status) {

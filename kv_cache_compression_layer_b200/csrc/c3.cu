@@ -126,6 +126,7 @@ __device__ __forceinline__ double ld<__nv_bfloat16>(const __nv_bfloat16* p) {
 }
 
 constexpr int kScanThreads = 1024;
+constexpr int kC3SelReg = 4;  // frontier entries a select thread keeps in registers
 
 // Exclusive sum over a block of kScanThreads threads; *total = the block's sum.
 __device__ int scan_excl(int v, int* total, int* sh) {
@@ -388,73 +389,98 @@ __global__ void __launch_bounds__(kScanThreads) c3_frontier_kernel(const RowMap 
 // (float64; products and sums rounded separately, every sum in dimension
 // order from 0, as the oracle does). A lane takes a node; its warp copies
 // the 32 nodes' centroids into shared memory 32 dimensions at a time with
-// coalesced loads (padded so the lanes' reads spread over the banks), and the
-// block copies the row's query rows as doubles. Sum c_k^2 does not depend on
-// the head and is taken once; the heads' dot products are independent
-// chains (up to kC3Heads at a time).
+// coalesced loads (eight in flight per lane; padded so the lanes' reads
+// spread over the banks), and the block copies the row's query rows as
+// doubles. The query norms sum q_k^2 and the centroid norm sum c_k^2 are
+// each taken once (the same chains as per cosine, so the same values); the
+// heads' dot products are independent chains (up to kC3Heads at a time).
+// A row's blocks stride over its frontier, so the grid holds no blocks
+// beyond the frontier's possible size.
 constexpr int kC3ScoreWarps = 4;
 constexpr int kC3Heads = 8;
 constexpr int kC3QStage = 16;  // query heads staged in shared memory (more: read from global memory)
+constexpr int kC3FillBatch = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(32 * kC3ScoreWarps)
     c3_score_kernel(const RowMap m, C3Arr a, const T* __restrict__ q, int G, int d, int B) {
-  extern __shared__ double c3s[];  // [warps][32][33] centroid chunks, then [G][d] query rows if G <= kC3QStage
+  // [warps][32][33] centroid chunks, then [G] query norms, then [G][d] query rows if G <= kC3QStage
+  extern __shared__ double c3s[];
   const int row = blockIdx.y;
   if (row_len(m, row) <= B) return;
   const long long no = 2 * row_key_off(m, row);
-  const int A = a.hdr()[(long long)row * kHdr + 1];
-  const int i0 = blockIdx.x * 32 * kC3ScoreWarps;
-  if (i0 >= A) return;
+  const int nodes = a.hdr()[(long long)row * kHdr], A = a.hdr()[(long long)row * kHdr + 1];
+  if (!kv_check(A >= 0 && A <= 2 * row_len(m, row) && nodes <= 2 * row_len(m, row))) return;
+  const int per_blk = 32 * kC3ScoreWarps;
+  if (blockIdx.x * per_blk >= A) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double* cs = c3s + (size_t)warp * 32 * 33;
-  double* qs = c3s + (size_t)kC3ScoreWarps * 32 * 33;
+  double* qn = c3s + (size_t)kC3ScoreWarps * 32 * 33;
+  double* qs = qn + G;
   const T* qr = q + (long long)row * G * d;
   const bool q_staged = G <= kC3QStage;
   if (q_staged)
-    for (int k = threadIdx.x; k < G * d; k += 32 * kC3ScoreWarps) qs[k] = ld(qr + k);
+    for (int k = threadIdx.x; k < G * d; k += per_blk) qs[k] = ld(qr + k);
   __syncthreads();
-  const int wi0 = i0 + warp * 32;
-  if (wi0 >= A) return;
-  const int i = wi0 + lane;
-  const int nw = min(32, A - wi0);  // nodes of this warp
-  const int my_node = i < A ? a.front()[no + i] : 0;
-  double bb = 0.0, best = -INFINITY;
-  for (int g0 = 0; g0 < G; g0 += kC3Heads) {
-    double ab[kC3Heads], aa[kC3Heads];
+  for (int g = threadIdx.x; g < G; g += per_blk) {
+    double aa = 0.0;
+    for (int k = 0; k < d; ++k) {
+      const double x = q_staged ? qs[g * d + k] : ld(qr + (long long)g * d + k);
+      aa = __dadd_rn(aa, __dmul_rn(x, x));
+    }
+    qn[g] = aa;
+  }
+  __syncthreads();
+  for (int i0 = blockIdx.x * per_blk; i0 < A; i0 += gridDim.x * per_blk) {
+    const int wi0 = i0 + warp * 32;
+    if (wi0 >= A) break;
+    const int i = wi0 + lane;
+    const int nw = min(32, A - wi0);  // nodes of this warp
+    int my_node = i < A ? a.front()[no + i] : 0;
+    if (!kv_check(my_node >= 0 && my_node < nodes)) my_node = 0;
+    double bb = 0.0, best = -INFINITY;
+    for (int g0 = 0; g0 < G; g0 += kC3Heads) {
+      double ab[kC3Heads];
 #pragma unroll
-    for (int t = 0; t < kC3Heads; ++t) ab[t] = aa[t] = 0.0;
-    for (int k0 = 0; k0 < d; k0 += 32) {
-      __syncwarp();
-      for (int n = 0; n < nw; ++n) {  // node n's dimensions k0 .. k0 + 31, one per lane
-        const int node = __shfl_sync(0xffffffffu, my_node, n);
-        cs[n * 33 + lane] = a.cent()[(no + node) * d + k0 + lane];
-      }
-      __syncwarp();
-      if (i < A) {
-        for (int kk = 0; kk < 32; ++kk) {
-          const int k = k0 + kk;
-          const double yk = cs[lane * 33 + kk];
-          if (g0 == 0) bb = __dadd_rn(bb, __dmul_rn(yk, yk));
+      for (int t = 0; t < kC3Heads; ++t) ab[t] = 0.0;
+      for (int k0 = 0; k0 < d; k0 += 32) {
+        __syncwarp();
+        for (int n0 = 0; n0 < nw; n0 += kC3FillBatch) {  // node n's dimensions k0 .. k0 + 31, one per lane
+          double v[kC3FillBatch];
 #pragma unroll
-          for (int t = 0; t < kC3Heads; ++t)
-            if (g0 + t < G) {
-              const double x = q_staged ? qs[(g0 + t) * d + k] : ld(qr + (long long)(g0 + t) * d + k);
-              ab[t] = __dadd_rn(ab[t], __dmul_rn(x, yk));
-              aa[t] = __dadd_rn(aa[t], __dmul_rn(x, x));
-            }
+          for (int u = 0; u < kC3FillBatch; ++u) {
+            const int node = __shfl_sync(0xffffffffu, my_node, (n0 + u) & 31);
+            v[u] = n0 + u < nw ? a.cent()[(no + node) * d + k0 + lane] : 0.0;
+          }
+#pragma unroll
+          for (int u = 0; u < kC3FillBatch; ++u)
+            if (n0 + u < nw) cs[(n0 + u) * 33 + lane] = v[u];
+        }
+        __syncwarp();
+        if (i < A) {
+          for (int kk = 0; kk < 32; ++kk) {
+            const int k = k0 + kk;
+            const double yk = cs[lane * 33 + kk];
+            if (g0 == 0) bb = __dadd_rn(bb, __dmul_rn(yk, yk));
+#pragma unroll
+            for (int t = 0; t < kC3Heads; ++t)
+              if (g0 + t < G) {
+                const double x = q_staged ? qs[(g0 + t) * d + k] : ld(qr + (long long)(g0 + t) * d + k);
+                ab[t] = __dadd_rn(ab[t], __dmul_rn(x, yk));
+              }
+          }
         }
       }
-    }
 #pragma unroll
-    for (int t = 0; t < kC3Heads; ++t)
-      if (g0 + t < G) {
-        const double c =
-            (aa[t] == 0.0 || bb == 0.0) ? 0.0 : __ddiv_rn(ab[t], __dmul_rn(__dsqrt_rn(aa[t]), __dsqrt_rn(bb)));
-        if (c > best) best = c;
-      }
+      for (int t = 0; t < kC3Heads; ++t)
+        if (g0 + t < G) {
+          const double aa = qn[g0 + t];
+          const double c = (aa == 0.0 || bb == 0.0) ? 0.0 : __ddiv_rn(ab[t], __dmul_rn(__dsqrt_rn(aa), __dsqrt_rn(bb)));
+          if (c > best) best = c;
+        }
+    }
+    if (i < A) a.sigma()[no + i] = best;
   }
-  if (i < A) a.sigma()[no + i] = best;
 }
 
 // Order key of a frontier entry: larger sigma first, then the lower node id.
@@ -481,23 +507,49 @@ __global__ void __launch_bounds__(kScanThreads) c3_select_kernel(const RowMap m,
     if (threadIdx.x == 0) h[2] = L;
     return;
   }
-  const int A = h[1];
+  const int nodes = h[0], A = h[1];
   const int32_t* fr = a.front() + no;
   const double* sg = a.sigma() + no;
+  if (kDebugChecks) {  // the row's frontier: its size and node ids, and each node's members
+    bool bad = !kv_check(A >= 0 && A <= 2 * L && nodes <= 2 * L);
+    for (int i = threadIdx.x; !bad && i < A; i += kScanThreads) {
+      const int n = fr[i];
+      bad = !kv_check(n >= 0 && n < nodes && a.lo()[no + n] >= 0 && a.cnt()[no + n] >= 0 &&
+                      a.lo()[no + n] + a.cnt()[no + n] <= L);
+    }
+    if (__syncthreads_or(bad)) return;
+  }
   if (threadIdx.x == 0) {
     thi_s = 0;
     tlo_s = 0;
     need_s = B;
   }
-  // weighted radix select over the 96-bit keys (sigma key, ~node id), 8 bits a round
+  // weighted radix select over the 96-bit keys (sigma key, ~node id), 8 bits a
+  // round; a thread keeps its first kC3SelReg entries in registers, and warp 0
+  // finds each round's bin (the entries' weights, the clusters' sizes, add up
+  // to L > B, so the bins always hold `need`)
+  uint64_t khi[kC3SelReg];
+  uint32_t klo[kC3SelReg];
+  int kcnt[kC3SelReg];
+#pragma unroll
+  for (int u = 0; u < kC3SelReg; ++u) {
+    const int i = threadIdx.x + u * kScanThreads;
+    khi[u] = 0;
+    klo[u] = 0;
+    kcnt[u] = 0;
+    if (i < A) {
+      const int n = fr[i];
+      khi[u] = sigma_key(sg[i]);
+      klo[u] = ~(uint32_t)n;
+      kcnt[u] = a.cnt()[no + n];
+    }
+  }
   for (int round = 0; round < 12; ++round) {
     for (int i = threadIdx.x; i < 256; i += kScanThreads) hist[i] = 0;
     __syncthreads();
     const unsigned long long phi = thi_s;
     const unsigned int plo = tlo_s;
-    for (int i = threadIdx.x; i < A; i += kScanThreads) {
-      const uint64_t hi = sigma_key(sg[i]);
-      const uint32_t lo = ~(uint32_t)fr[i];
+    auto count = [&](uint64_t hi, uint32_t lo, int c) {
       bool match;
       int digit;
       if (round < 8) {
@@ -511,18 +563,22 @@ __global__ void __launch_bounds__(kScanThreads) c3_select_kernel(const RowMap m,
         match = hi == phi && (lo & mask) == (plo & mask);
         digit = (int)((lo >> sh_lo) & 255u);
       }
-      if (match) atomicAdd(&hist[digit], a.cnt()[no + fr[i]]);
-    }
+      if (match) atomicAdd(&hist[digit], c);
+    };
+#pragma unroll
+    for (int u = 0; u < kC3SelReg; ++u)
+      if (threadIdx.x + u * kScanThreads < A) count(khi[u], klo[u], kcnt[u]);
+    for (int i = threadIdx.x + kC3SelReg * kScanThreads; i < A; i += kScanThreads)
+      count(sigma_key(sg[i]), ~(uint32_t)fr[i], a.cnt()[no + fr[i]]);
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int need = need_s, cum = 0, dg = 255;
-      for (; dg > 0; --dg) {
-        if (cum + hist[dg] >= need) break;
-        cum += hist[dg];
+    if (threadIdx.x < 32) {
+      int need = need_s;
+      const int dg = top_bin(hist, need);
+      if (threadIdx.x == 0) {
+        need_s = need;
+        if (round < 8) thi_s = phi | ((unsigned long long)dg << (56 - 8 * round));
+        else tlo_s = plo | ((unsigned int)dg << (24 - 8 * (round - 8)));
       }
-      need_s = need - cum;
-      if (round < 8) thi_s = phi | ((unsigned long long)dg << (56 - 8 * round));
-      else tlo_s = plo | ((unsigned int)dg << (24 - 8 * (round - 8)));
     }
     __syncthreads();
   }
@@ -539,7 +595,8 @@ __global__ void __launch_bounds__(kScanThreads) c3_select_kernel(const RowMap m,
     if (hi > thi || (hi == thi && lo > tlo)) take = a.cnt()[no + n];
     else if (hi == thi && lo == tlo) take = need;
     const int32_t* mem = a.perm() + ko + a.lo()[no + n];
-    for (int j = 0; j < take; ++j) a.taken[ko + mem[j]] = 1;
+    for (int j = 0; j < take; ++j)
+      if (kv_check(mem[j] >= 0 && mem[j] < L)) a.taken[ko + mem[j]] = 1;
   }
   __syncthreads();
   int carry = 0;
@@ -616,7 +673,10 @@ __global__ void __launch_bounds__(kAttnThreads)
   const int per = d / 32;  // elements per lane: 2 or 4
   const T* qr = q + ((long long)row * G + g) * d;
   for (int k = threadIdx.x; k < d; k += kAttnThreads) qv[k] = (float)ld(qr + k);
-  for (int i = threadIdx.x; i < n; i += kAttnThreads) sel_s[i] = sel[i];
+  for (int i = threadIdx.x; i < n; i += kAttnThreads) {
+    const int p = sel[i];
+    sel_s[i] = kv_check(p >= 0 && p < row_len(m, row)) ? p : 0;
+  }
   __syncthreads();
   const float scale = rsqrtf((float)d);
   float qa[4];
@@ -738,6 +798,12 @@ __global__ void __launch_bounds__(kScanThreads)
   int32_t* h = a.hdr() + (long long)row * kHdr;
   const int nodes = h[0], A = h[1];
   int32_t* fr = a.front() + no;
+  if (kDebugChecks) {  // the row's frontier: its size and node ids
+    const int L = row_len(m, row);
+    bool bad = !kv_check(A >= 0 && A <= 2 * L && nodes <= 2 * L);
+    for (int i = threadIdx.x; !bad && i < A; i += kScanThreads) bad = !kv_check(fr[i] >= 0 && fr[i] < nodes);
+    if (__syncthreads_or(bad)) return;
+  }
   double* e = a.e() + no;
   const int32_t* left = a.left() + no;
   uint8_t* on = a.on + no;
@@ -920,9 +986,14 @@ int kv_c3_step(const kv_shape* shape, const int32_t* L, int32_t n_seq, const kv_
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int d = shape->head_dim, G = shape->group, B = p->budget;
   const int Lmax = max_len(m);
+  // blocks per row: the frontier's largest possible size (2 L nodes), capped so
+  // that the grid is about four waves of resident blocks; the blocks stride
   const int per_blk = 32 * kC3ScoreWarps;
-  const dim3 sgrid((2 * Lmax + per_blk - 1) / per_blk, m.n_rows);
-  const size_t score_smem = ((G <= kC3QStage ? (size_t)G * d : 0) + (size_t)kC3ScoreWarps * 32 * 33) * sizeof(double);
+  const size_t score_smem =
+      ((G <= kC3QStage ? (size_t)G * d : 0) + (size_t)G + (size_t)kC3ScoreWarps * 32 * 33) * sizeof(double);
+  const int resident = sm_count() * (int)std::max<size_t>(1, (228u << 10) / (score_smem + 1024));
+  const int sx = std::max(1, std::min((2 * Lmax + per_blk - 1) / per_blk, (4 * resident + m.n_rows - 1) / m.n_rows));
+  const dim3 sgrid(sx, m.n_rows);
   const size_t attn_smem = 2 * (size_t)B * sizeof(float);  // logits and retrieved positions
   if (shape->dtype == KV_BF16) {
     using T = __nv_bfloat16;

@@ -14,6 +14,40 @@ namespace kvc {
 
 constexpr int kTileKeys = 128;  // keys per scoring tile (the MMA's M or N)
 
+// Index checks of debug builds. kv_check(ok) returns ok; when it is false it
+// sets KV_DEV_BOUNDS in this file's check word, and the caller skips the
+// access. Each kernel file has its own word (a device variable is local to
+// its file without relocatable device code) and registers a reader with the
+// C-ABI layer, which ORs them. Release builds compile kv_check to `true`.
+#ifdef KV_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+namespace {
+__device__ int kv_check_word_;
+int read_check_word(bool clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, kv_check_word_, sizeof(int)) != cudaSuccess) return -1;
+  if (clear) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(kv_check_word_, &z, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+}  // namespace
+void register_check_word(int (*reader)(bool));
+namespace {
+struct CheckWordRegistration {
+  CheckWordRegistration() { register_check_word(&read_check_word); }
+} check_word_registration_;
+}  // namespace
+__device__ __forceinline__ bool kv_check(bool ok) {
+  if (!ok) atomicOr(&kv_check_word_, KV_DEV_BOUNDS);
+  return ok;
+}
+#else
+constexpr bool kDebugChecks = false;
+__device__ __forceinline__ bool kv_check(bool) { return true; }
+#endif
+
 // Where every row of a ragged batch lives. Rows of sequence s are
 // rows_per_seq consecutive rows of length L[s].
 struct RowMap {
@@ -137,6 +171,45 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
       : "r"(id), "r"(nthreads), "r"((uint32_t)pred)
       : "memory");
   return r != 0;
+}
+
+// The bin of the kk-th largest key from a 256-bin histogram, by one warp: lane
+// l holds bins 255 - 8 l down to 248 - 8 l, so lanes in order walk the bins
+// from the top. Returns the bin; kk becomes the rank within it. The bins must
+// hold at least kk keys in all.
+__device__ __forceinline__ int top_bin(const int* hist, int& kk) {
+  const int lane = threadIdx.x & 31;
+  int loc[8], tot = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    loc[t] = hist[255 - 8 * lane - t];
+    tot += loc[t];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - tot;
+  const unsigned here = __ballot_sync(0xffffffffu, excl < kk && kk <= incl);
+  const int src = __ffs(here) - 1;
+  int dg = 0, kk_new = kk;
+  if (lane == src) {
+    int cum = excl;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (cum + loc[t] >= kk) {
+        dg = 255 - 8 * lane - t;
+        kk_new = kk - cum;
+        break;
+      }
+      cum += loc[t];
+    }
+  }
+  dg = __shfl_sync(0xffffffffu, dg, src);
+  kk = __shfl_sync(0xffffffffu, kk_new, src);
+  return dg;
 }
 
 // ---------------------------------------------------------------------- TMA

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(const DecArg
   const bool evict = n > bb;
   const int S = (cap + a.C - 1) / a.C;
   const int j0 = rank * S, j1 = min(j0 + S, n);
-  const bool ok = S <= a.S_cap && count < cap && (!evict || bb >= a.T + M);
+  const bool ok = S <= a.S_cap && count < cap && (!evict || bb >= a.T + M) && kv_check(next >= 0 && next < cap);
   const int cnt = ok ? max(0, j1 - j0) : 0;
   if (!ok && rank == 0 && tid == 0) atomicOr(a.status, S > a.S_cap ? KV_DEV_CAPACITY : KV_DEV_BUDGET);
 
@@ -254,9 +254,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(const DecArg
       f[g] = 0.f;
       if (g < G && m_s[g] > -INFINITY) f[g] = exp2f(m_s[g] - *cluster.map_shared_rank(&lse_s[g], 0));
     }
-    int pos_thr;
-    if (appended >= M) pos_thr = pos_new - M + 1;
-    else pos_thr = pos[max(0, count0 - (M - appended))];
+    int pos_thr = pos_new - M + 1;
+    if (appended < M && kv_check(count0 - (M - appended) < cap)) pos_thr = pos[max(0, count0 - (M - appended))];
     if (ok) {
       for (int jl = tid; jl < cnt; jl += kDecThreads) {
         const int j = j0 + jl;
@@ -298,7 +297,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(const DecArg
       const Best y = *cluster.map_shared_rank(&best_s, r);
       if (better(y, bst)) bst = y;
     }
-    if (evict && bst.slot >= 0) {
+    if (evict && bst.slot >= 0 && kv_check(bst.slot < cap)) {
       meta[0] = bb;
       meta[1] = bst.slot;
       meta[3] = bst.slot;

@@ -530,7 +530,8 @@ __device__ __forceinline__ void row_consts(const DecArgs& a, int row, RowC& R) {
   // the M most recent positions are >= pos_thr: the appended ones and, early on,
   // the last prefill entries (never evicted while recent, so their pos is stable)
   int pos_thr = pos_new - Mr + 1;
-  if (ok && appended < Mr) pos_thr = a.pos[base + max(0, count0 - (Mr - appended))];
+  if (ok && appended < Mr && kv_check(count0 - (Mr - appended) < cap))
+    pos_thr = a.pos[base + max(0, count0 - (Mr - appended))];
   R.base = base;
   R.cap = cap;
   R.n = n;
@@ -1066,7 +1067,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           } else if ((R.flags & 4) || nb > sc.max_bests) {
             atomicOr(a.status, KV_DEV_CAPACITY);
           } else {
-            if ((R.flags & 2) && bst.slot >= 0) {
+            if ((R.flags & 2) && bst.slot >= 0 && kv_check(bst.slot < R.cap)) {
               meta[0] = R.bb;
               meta[1] = bst.slot;
               meta[3] = bst.slot;

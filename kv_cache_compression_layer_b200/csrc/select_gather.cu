@@ -41,44 +41,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// The bin of the kk-th largest key from a 256-bin histogram, by one warp: lane
-// l holds bins 255 - 8 l down to 248 - 8 l, so lanes in order walk the bins
-// from the top. Returns the bin; kk becomes the rank within it.
-__device__ __forceinline__ int top_bin(const int* hist, int& kk) {
-  const int lane = threadIdx.x & 31;
-  int loc[8], tot = 0;
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    loc[t] = hist[255 - 8 * lane - t];
-    tot += loc[t];
-  }
-  int incl = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int excl = incl - tot;
-  const unsigned here = __ballot_sync(0xffffffffu, excl < kk && kk <= incl);
-  const int src = __ffs(here) - 1;
-  int dg = 0, kk_new = kk;
-  if (lane == src) {
-    int cum = excl;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      if (cum + loc[t] >= kk) {
-        dg = 255 - 8 * lane - t;
-        kk_new = kk - cum;
-        break;
-      }
-      cum += loc[t];
-    }
-  }
-  dg = __shfl_sync(0xffffffffu, dg, src);
-  kk = __shfl_sync(0xffffffffu, kk_new, src);
-  return dg;
-}
-
 // The k largest keys of keys[c0s, c1s) (ties to the lower index) written to
 // out[0, k) in ascending index order; called by the whole block. Each radix
 // round counts into per-warp histograms (no atomics between warps: the
@@ -226,6 +188,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   const long long koff = row_key_off(map, row);
   const int bb = b[row];
   int32_t* out = idx + slot_off[row];
+  // debug builds: the row writes min(b, L) entries into its b + 1 slots
+  if (!kv_check(bb < 0 || min(bb, L) <= slot_off[row + 1] - slot_off[row])) return;
 
   if (bb >= L) {
     for (int j = threadIdx.x; j < L; j += kSelThreads) out[j] = j;

@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(kPoolThreads)
     const long long r = R - m.row_off[lo_s];
     if (r >= __ldg(out_len + lo_s)) continue;
     const int first = __ldg(src + 3 * R), cnt = __ldg(src + 3 * R + 1), tr = __ldg(src + 3 * R + 2);
+    if (!kv_check(first >= 0 && cnt >= 0 && (long long)first + cnt <= m.L[lo_s])) continue;
     const int c0 = slice * (kSliceBytes / (int)sizeof(T)) + lane * N;  // first piece
     const int c1 = c0 + 32 * N;                                        // second piece
     const bool p0 = c0 < d, p1 = c1 < d;

@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kRecThreads)
     const int b = __ldg(fetch + ((long long)sq * cap + f) * 2), slot = __ldg(fetch + ((long long)sq * cap + f) * 2 + 1);
     const int L = m.L[sq];
     const long long row0 = (long long)b * S;
-    if (b < 0 || row0 >= L || slot < 0 || slot >= n_slots) continue;
+    if (!kv_check(b >= 0 && row0 < L && slot >= 0 && slot < n_slots)) continue;
     const int rows = (int)min((long long)S, L - row0);
     const uint4* src = reinterpret_cast<const uint4*>((kv ? V_host : K_host) +
                                                       (m.s_off[sq] + (long long)r * L + row0) * row_bytes);

@@ -191,3 +191,14 @@ def test_wait_limit_round_trips(L):
     finally:
         kv.kv_set_wait_limit_ns(prev)
     assert kv.kv_set_wait_limit_ns(prev) == prev
+
+
+def test_debug_build_exports_and_reports_itself(L):
+    # the debug build (index checks compiled in) exports the same symbols and
+    # says it is one; the release build loaded by the binding says it is not
+    D = C.CDLL(kvbuild.build(debug=True))
+    for n in _declared():
+        assert hasattr(D, n), n
+    D.kv_debug_checks.restype = C.c_int
+    assert D.kv_debug_checks() == 1
+    assert kv.kv_debug_checks() == kv.DEBUG_CHECKS
