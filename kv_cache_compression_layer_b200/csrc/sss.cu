@@ -25,7 +25,8 @@
 //
 // Rows with N <= 2048 are taken four to a CTA and N <= 4096 two (a named
 // barrier per row), N <= 8192 one; longer rows are split over a 2-CTA cluster
-// whose halves are addressed through distributed shared memory. Sequences are
+// whose halves are addressed through distributed shared memory. A batch that
+// would leave SMs idle that way (fewer CTAs than SMs) gets one row per CTA. Sequences are
 // launched longest first. Prior art on the pages uses cuFFT (AudioKV blog
 // §3.2); this is a hand-written transform.
 #include <algorithm>
@@ -604,15 +605,23 @@ __global__ void __launch_bounds__(kSssThreads, 1)
 
 int launch_sss(const RowMap& m, const float* s, float* s_hat, int32_t* kstar, float alpha, float rho,
                cudaStream_t st) {
-  // sequences longest first; rows per CTA by length; rows past kMaxLocal points on a cluster
+  // sequences longest first; rows per CTA by length (one when the batch is too
+  // small to fill the SMs otherwise); rows past kMaxLocal points on a cluster
   int order[KV_MAX_SEQ];
   for (int i = 0; i < m.n_seq; ++i) order[i] = i;
   std::stable_sort(order, order + m.n_seq, [&](int x, int y) { return m.L[x] > m.L[y]; });
   SssPlan p1 = {}, p2 = {};
+  int ctas = 0;
+  for (int i = 0; i < m.n_seq; ++i) {
+    const int N = m.L[i] / 2;
+    const int per = N > kMaxLocal ? 1 : N > 4096 ? 1 : N > 2048 ? 2 : 4;
+    ctas += (N > kMaxLocal ? 2 : 1) * ((m.rows_per_seq + per - 1) / per);
+  }
+  const bool few = ctas < sm_count();
   for (int i = 0; i < m.n_seq; ++i) {
     const int sq = order[i], N = m.L[sq] / 2;
     SssPlan& p = N > kMaxLocal ? p2 : p1;
-    const int per = N > 4096 ? 1 : N > 2048 ? 2 : 4;
+    const int per = few || N > 4096 ? 1 : N > 2048 ? 2 : 4;
     p.seq[p.n] = sq;
     p.per[p.n] = N > kMaxLocal ? 1 : per;
     p.first[p.n + 1] = p.first[p.n] + (m.rows_per_seq + p.per[p.n] - 1) / p.per[p.n];
