@@ -82,7 +82,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with python -m kv_cache_compression_layer_b200.build")
+            flag = " --debug" if DEBUG_CHECKS else ""
+            raise ImportError(f"{LIB_PATH} is missing: build it with python -m kv_cache_compression_layer_b200.build{flag}")
         L = C.CDLL(LIB_PATH)
         P, I32, SZ, I64 = C.c_void_p, C.c_int32, C.c_size_t, C.c_int64
         Ps, Pp, Pc = C.POINTER(kv_shape), C.POINTER(kv_params), C.POINTER(kv_cache)
